@@ -1,0 +1,204 @@
+"""Python binding for libattn, the B200 (sm_100a) fused exact-attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind ``include/libattn.h``.  PyTorch supplies device memory and the
+current stream.  There is no CPU or library fallback: if ``libattn.so`` is
+missing, importing the entry points raises.
+
+The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
+``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_workspace_bytes``,
+``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
+``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_MISALIGNED = 3
+ATTN_ERR_WORKSPACE = 4
+ATTN_ERR_CUDA = 5
+ATTN_ERR_TIMEOUT = 6
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: libattn status {code}: {attn_strerror(code)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so from the package directory (built by ``build.py``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libattn.so not found at {LIB_PATH}; build it with "
+                           "`python -m exact_attention_123_b200.build` (no fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
+    L.attn_fwd_masked.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp]
+    L.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
+    L.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    L.attn_bwd_workspace_bytes.restype = sz
+    L.attn_bwd_varlen_workspace_bytes.argtypes = [i, i, i]
+    L.attn_bwd_varlen_workspace_bytes.restype = sz
+    L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp, sz, vp]
+    L.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
+    L.attn_status.argtypes = [vp]
+    L.attn_strerror.argtypes = [i]
+    L.attn_strerror.restype = ctypes.c_char_p
+    L.attn_set_wait_limit_ms.argtypes = [i]
+    L.attn_debug_skip_load.argtypes = [i]
+    for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen",
+                 "attn_status", "attn_set_wait_limit_ms", "attn_debug_skip_load"):
+        getattr(L, name).restype = i
+    _lib = L
+    return L
+
+
+def attn_strerror(code: int) -> str:
+    return lib().attn_strerror(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, where: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, where)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def attn_fwd(q, k, v, o=None, lse=None, *, scale: Optional[float] = None, causal: bool = True,
+             cu_seqlens: Optional[torch.Tensor] = None, key_keep: Optional[torch.Tensor] = None,
+             max_seqlen: Optional[int] = None, stream=None):
+    """Forward pass.  Dense q/k/v are [B,H,N,d]; packed ones are [total,H,d] with
+    ``cu_seqlens`` (int32, device).  Returns (o, lse)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, n)
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if cu_seqlens is not None:
+        total, H = q.shape[0], q.shape[1]
+        B = cu_seqlens.numel() - 1
+        if lse is None:
+            lse = torch.empty((total, H), device=q.device, dtype=torch.float32)
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, total, int(max_seqlen), H, d,
+                                   float(scale), int(causal), _ptr(cu_seqlens), _ptr(key_keep), _stream(stream))
+        _check(rc, "attn_fwd_varlen")
+        return o, lse
+    B, H, N, _ = q.shape
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    if key_keep is None:
+        rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal),
+                            None, _stream(stream))
+        _check(rc, "attn_fwd")
+    else:
+        rc = lib().attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                   int(causal), None, _ptr(key_keep), _stream(stream))
+        _check(rc, "attn_fwd_masked")
+    return o, lse
+
+
+def attn_fwd_masked(q, k, v, key_keep, **kw):
+    return attn_fwd(q, k, v, key_keep=key_keep, **kw)
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, **kw):
+    return attn_fwd(q, k, v, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen, **kw)
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().attn_bwd_workspace_bytes(B, H, N, d))
+
+
+def attn_bwd_varlen_workspace_bytes(total: int, H: int, d: int) -> int:
+    return int(lib().attn_bwd_varlen_workspace_bytes(total, H, d))
+
+
+def workspace_for(q: torch.Tensor, cu_seqlens=None) -> torch.Tensor:
+    """Allocate (with torch) a backward workspace sized for q's shape."""
+    if cu_seqlens is not None:
+        n = attn_bwd_varlen_workspace_bytes(q.shape[0], q.shape[1], q.shape[2])
+    else:
+        B, H, N, d = q.shape
+        n = attn_bwd_workspace_bytes(B, H, N, d)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
+def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[float] = None,
+             causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
+             workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward pass.  Returns (dq, dk, dv)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(q, cu_seqlens)
+    if cu_seqlens is not None:
+        total, H = q.shape[0], q.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        rc = lib().attn_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, total, int(max_seqlen), H, d, float(scale), int(causal),
+                                   _ptr(cu_seqlens), _ptr(key_keep), _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
+        _check(rc, "attn_bwd_varlen")
+    else:
+        B, H, N, _ = q.shape
+        rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                            B, H, N, d, float(scale), int(causal), None, _ptr(key_keep), _ptr(workspace),
+                            workspace.numel(), _stream(stream))
+        _check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word."""
+    return int(lib().attn_status(_stream(stream)))
+
+
+def attn_set_wait_limit_ms(ms: int) -> int:
+    return int(lib().attn_set_wait_limit_ms(int(ms)))
+
+
+def attn_debug_skip_load(index: int) -> int:
+    return int(lib().attn_debug_skip_load(int(index)))

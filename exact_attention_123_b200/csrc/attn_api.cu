@@ -1,0 +1,281 @@
+// attn_api.cu -- the libattn C ABI: argument validation, TMA tensor-map
+// construction, the device status word, and dispatch to the sm_100a launchers.
+// No entry point allocates memory or synchronises, except attn_status().
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/libattn.h"
+#include "attn_launch.h"
+
+namespace {
+
+__device__ int g_attn_status = 0;
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::atomic<int> g_wait_limit_ms{4000};
+std::atomic<int> g_skip_load{-1};
+
+struct DeviceState {
+    std::once_flag once;
+    int supported = 0;  // 1 if sm_100
+    int *status = nullptr;
+    cudaError_t err = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// Per-device one-time setup: architecture check and the status word's address.
+int device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+    DeviceState &s = g_dev[dev];
+    std::call_once(s.once, [&] {
+        int major = 0, minor = 0;
+        s.err = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        s.supported = (major == 10 && minor == 0);
+        if (s.err == cudaSuccess && s.supported) s.err = cudaGetSymbolAddress(reinterpret_cast<void **>(&s.status), g_attn_status);
+    });
+    if (s.err != cudaSuccess) return ATTN_ERR_CUDA;
+    if (!s.supported) return ATTN_ERR_UNSUPPORTED;
+    *out = &s;
+    return ATTN_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D map (col, row, slab) over a bf16 tensor; box = 64 columns x 128 rows x 1.
+int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long slabs, long long row_stride,
+             long long slab_stride) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return ATTN_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2, static_cast<cuuint64_t>(slab_stride) * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+struct Shape {
+    int B, H, N, d;
+    long long total;  // packed token rows, or 0 for dense
+    const int32_t *cu;
+};
+
+int map_for(CUtensorMap *m, const void *base, const Shape &s) {
+    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d);
+    return make_map(m, base, s.d, s.N, static_cast<long long>(s.B) * s.H, s.d, static_cast<long long>(s.N) * s.d);
+}
+
+int check_common(const Shape &s, float scale) {
+    if (s.B <= 0 || s.H <= 0 || s.N <= 0 || s.d <= 0) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (s.cu && s.total < 0) return ATTN_ERR_INVALID_ARG;
+    if (s.d != 64 && s.d != 128) return ATTN_ERR_UNSUPPORTED;
+    // grid limits: B <= 65535 (grid y), H <= 2^31-1, N/256 <= 65535 (grid z)
+    if (s.B > 65535 || (s.N + 255) / 256 > 65535) return ATTN_ERR_UNSUPPORTED;
+    // TMA extents are 32-bit
+    if (s.cu ? s.total > 0x7fffffffLL : static_cast<long long>(s.B) * s.H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+attn::Geom geom_of(const Shape &s, const uint8_t *key_keep) {
+    attn::Geom g{};
+    g.B = s.B;
+    g.H = s.H;
+    g.N = s.N;
+    g.d = s.d;
+    g.varlen = s.cu != nullptr;
+    g.cu_seqlens = s.cu;
+    g.key_keep = key_keep;
+    return g;
+}
+
+attn::SyncCtl ctl_of(DeviceState *ds) {
+    attn::SyncCtl c{};
+    c.status = ds->status;
+    c.wait_limit_ns = static_cast<unsigned long long>(g_wait_limit_ms.load()) * 1000000ull;
+    c.inject_skip_load = g_skip_load.load();
+    return c;
+}
+
+int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, const Shape &s, float scale,
+             int is_causal, const uint8_t *key_keep, void *stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    int rc = check_common(s, scale);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_MISALIGNED;
+    DeviceState *ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    if (s.cu && s.total == 0) return ATTN_OK;  // nothing to do
+    attn::FwdLaunch a{};
+    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s))) return rc;
+    a.g = geom_of(s, key_keep);
+    a.ctl = ctl_of(ds);
+    a.o = o;
+    a.lse = lse;
+    a.scale = scale;
+    a.causal = is_causal ? 1 : 0;
+    return attn::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t bwd_ws_bytes(long long rows_x_heads, int d) {
+    // dQ fp32 accumulator, then D and lse2 (fp32 each), each region 256-byte aligned
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return up(static_cast<size_t>(rows_x_heads) * d * 4) + 2 * up(static_cast<size_t>(rows_x_heads) * 4);
+}
+
+int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+             void *dq, void *dk, void *dv, const Shape &s, float scale, int is_causal, const uint8_t *key_keep,
+             void *workspace, size_t workspace_bytes, void *stream) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+    int rc = check_common(s, scale);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return ATTN_ERR_MISALIGNED;
+    const long long rows = s.cu ? s.total * s.H : static_cast<long long>(s.B) * s.H * s.N;
+    const size_t need = bwd_ws_bytes(rows, s.d);
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
+    DeviceState *ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    if (s.cu && s.total == 0) return ATTN_OK;
+    attn::BwdLaunch a{};
+    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
+        (rc = map_for(&a.tm_do, dout, s)))
+        return rc;
+    a.g = geom_of(s, key_keep);
+    a.ctl = ctl_of(ds);
+    a.o = o;
+    a.dout = dout;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    char *w = static_cast<char *>(workspace);
+    a.dq_acc = reinterpret_cast<float *>(w);
+    a.dvec = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4));
+    a.lse2 = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4) + up(static_cast<size_t>(rows) * 4));
+    a.rows_total = rows;
+    a.scale = scale;
+    a.causal = is_causal ? 1 : 0;
+    return attn::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+             float scale, int is_causal, const int32_t *cu_seqlens, void *stream) {
+    Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
+    return fwd_impl(q, k, v, o, lse, s, scale, is_causal, nullptr, stream);
+}
+
+int attn_fwd_masked(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+                    float scale, int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep, void *stream) {
+    Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
+    return fwd_impl(q, k, v, o, lse, s, scale, is_causal, key_keep, stream);
+}
+
+int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, int num_seqs, int total_tokens,
+                    int max_seqlen, int H, int d, float scale, int is_causal, const int32_t *cu_seqlens,
+                    const uint8_t *key_keep, void *stream) {
+    if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
+    Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
+    return fwd_impl(q, k, v, o, lse, s, scale, is_causal, key_keep, stream);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
+    if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+    return bwd_ws_bytes(static_cast<long long>(B) * H * N, d);
+}
+
+size_t attn_bwd_varlen_workspace_bytes(int total_tokens, int H, int d) {
+    if (total_tokens < 0 || H <= 0 || (d != 64 && d != 128)) return 0;
+    return bwd_ws_bytes(static_cast<long long>(total_tokens) * H, d);
+}
+
+int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout, void *dq,
+             void *dk, void *dv, int B, int H, int N, int d, float scale, int is_causal, const int32_t *cu_seqlens,
+             const uint8_t *key_keep, void *workspace, size_t workspace_bytes, void *stream) {
+    Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
+                    stream);
+}
+
+int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+                    void *dq, void *dk, void *dv, int num_seqs, int total_tokens, int max_seqlen, int H, int d,
+                    float scale, int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+    if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
+    Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
+                    stream);
+}
+
+int attn_status(void *stream) {
+    DeviceState *ds = nullptr;
+    int rc = device_state(&ds);
+    if (rc) return rc;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, ds->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    return v;
+}
+
+const char *attn_strerror(int code) {
+    switch (code) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument (null pointer, non-positive size or bad scale)";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported (head_dim must be 64 or 128; device must be sm_100)";
+        case ATTN_ERR_MISALIGNED: return "a base pointer is not 16-byte aligned (workspace: 256-byte)";
+        case ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
+        case ATTN_ERR_CUDA: return "a CUDA call or kernel launch failed";
+        case ATTN_ERR_TIMEOUT: return "a device-side pipeline wait exceeded its time limit";
+        default: return "unknown status code";
+    }
+}
+
+int attn_set_wait_limit_ms(int ms) {
+    return g_wait_limit_ms.exchange(ms > 0 ? ms : 4000);
+}
+
+int attn_debug_skip_load(int load_index) {
+    return g_skip_load.exchange(load_index < 0 ? -1 : load_index);
+}
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// attn_common.cuh -- parameter blocks and the bounded-wait / status machinery
+// shared by the forward and backward kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 6;  // ATTN_ERR_TIMEOUT
+
+// Geometry of one (sequence, head) slice, common to dense and packed layouts.
+// A tensor element (row r, column c) of slice (b, h) sits at
+//   base + seq_off(b) + h * head_stride + r * row_stride + c
+// Dense [B,H,N,d]:   seq_off = b*H*N*d, head_stride = N*d, row_stride = d.
+// Packed [total,H,d]: seq_off = cu[b]*H*d, head_stride = d, row_stride = H*d.
+// lse uses the same scheme with d = 1.
+struct Geom {
+    int B, H, N, d;
+    int varlen;                 // 0 dense, 1 packed (cu_seqlens)
+    const int32_t *cu_seqlens;  // device, B+1 entries (packed only)
+    const uint8_t *key_keep;    // device, nullable
+    __device__ __forceinline__ void slice(int b, int &start, int &len) const {
+        if (varlen) {
+            start = cu_seqlens[b];
+            len = cu_seqlens[b + 1] - start;
+        } else {
+            start = 0;
+            len = N;
+        }
+    }
+    // Element offset of (b, h, row 0, col 0) in a [.., d]-wide tensor.
+    __device__ __forceinline__ long long base(int b, int h, int start, int width) const {
+        if (varlen) return (static_cast<long long>(start) * H + h) * width;
+        return (static_cast<long long>(b) * H + h) * static_cast<long long>(N) * width;
+    }
+    __device__ __forceinline__ long long row_stride(int width) const {
+        return varlen ? static_cast<long long>(H) * width : width;
+    }
+    // Key-mask offset of key 0 of sequence b.
+    __device__ __forceinline__ long long keep_base(int b, int start) const {
+        return varlen ? start : static_cast<long long>(b) * N;
+    }
+    // TMA row coordinate of row 0 of (b, h): the maps are 3-D (col, row, slab).
+    __device__ __forceinline__ int tma_row0(int start) const { return varlen ? start : 0; }
+    __device__ __forceinline__ int tma_slab(int b, int h) const { return varlen ? h : b * H + h; }
+};
+
+struct SyncCtl {
+    int *status;             // device status word (first error wins)
+    unsigned long long wait_limit_ns;
+    int inject_skip_load;    // test hook: index of a pipeline load to skip, or -1
+};
+
+// Record an error once and raise the CTA-wide abort flag.
+__device__ __forceinline__ void raise_abort(const SyncCtl &ctl, volatile int *abort_flag, int code) {
+    atomicCAS(ctl.status, 0, code);
+    *abort_flag = 1;
+    __threadfence_block();
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the abort flag on
+// expiry) if the wait gave up, either because the limit passed or because another
+// role of the CTA already aborted.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const SyncCtl &ctl,
+                                           volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > ctl.wait_limit_ns) {
+                raise_abort(ctl, abort_flag, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait used during teardown: ignores the abort flag (the hardware must be
+// drained before shared memory / tensor memory are released), still time-limited.
+__device__ __forceinline__ bool drain_phase(uint32_t bar, uint32_t parity, const SyncCtl &ctl,
+                                            volatile int *abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0 && globaltimer_ns() - t0 > ctl.wait_limit_ns) {
+            raise_abort(ctl, abort_flag, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+}  // namespace attn

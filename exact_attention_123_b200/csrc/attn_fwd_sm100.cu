@@ -1,0 +1,394 @@
+// attn_fwd_sm100.cu -- fused exact-attention forward for B200 (sm_100a).
+//
+// One CTA owns 256 query rows of one (sequence, head) slice, as two 128-row
+// tiles Q0 and Q1, and sweeps the key/value tiles of 128 keys with the online
+// softmax recurrence ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", 第三步 §1;
+// codechina FlashAttention article §3.2): per query row a running max m, a running
+// sum l and an un-normalised output accumulator, rescaled when m moves, divided by
+// l at the end.  The 128 x 128 score tile lives only in tensor memory.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for Q0 (warp w owns TMEM lanes 32*(w%4)..+31, one row/thread)
+//   warps 4-7  softmax for Q1
+//   warp  8    TMA producer: Q0/Q1 once, then K_j, V_j into a ring of shared-memory
+//              slots guarded by full/empty mbarriers (the pages' double buffering,
+//              done by the copy engine instead of the SMs)
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   S0 = cols [0,128)  S1 = [128,256)   fp32 scores Q_t K_j^T;
+//   P_t (bf16, packed 2 per column) overwrites the first 64 columns of S_t;
+//   O0 = [256, 256+d)  O1 = [256+d, 256+2d)   fp32 output accumulators.
+//
+// MMA issue order per key tile j (single thread, in order):
+//   PV0(j) [O0 += P0 V_j], S0(j+1), PV1(j), S1(j+1)
+// so the tensor core computes tile 1's product while the Q0 softmax warps work
+// on S0(j+1) and vice versa.  Because tcgen05 operations issued by one thread
+// complete in order, the commit that publishes S_t(j+1) also proves PV_t(j) is
+// done, which is what makes reading/rescaling O_t and overwriting P_t safe.
+//
+// Exponentials are base 2: p = 2^(s * scale * log2(e) - m).  The running max is
+// only moved when a row's new max exceeds the one in use by more than 8 (log2
+// units), so O is rescaled rarely (lazy correction); O, l and lse always refer to
+// the same m, which keeps the final O / l and lse = (m + log2 l) ln 2 exact.
+// A row that sees no key keeps m = -inf and l = 0 and writes O = 0, lse = -inf
+// (the _safe_softmax rule of "Profiling in PyTorch (part 3)", math backend).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "attn_common.cuh"
+#include "attn_launch.h"
+
+namespace attn {
+
+template <int D>
+struct FwdCfg {
+    static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
+    static constexpr int kBoxes = D / 64;           // 128-byte-swizzle boxes per tile
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kThreads = 320;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+    // barrier indices
+    static constexpr int kBarQ = 0;
+    static constexpr int kBarFull = 1;                       // + slot
+    static constexpr int kBarEmpty = 1 + kStages;            // + slot
+    static constexpr int kBarS = 1 + 2 * kStages;            // + tile
+    static constexpr int kBarP = 3 + 2 * kStages;            // + tile
+    static constexpr int kBarO = 5 + 2 * kStages;            // + tile
+    static constexpr int kBarDone = 7 + 2 * kStages;
+    static constexpr int kNumBars = 8 + 2 * kStages;
+    static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
+    static constexpr int kSmemBytes = 1024 + kSmemTiles + kNumBars * 8 + 16;
+};
+
+struct FwdParams {
+    Geom g;
+    SyncCtl ctl;
+    __nv_bfloat16 *o;
+    float *lse;
+    float scale_log2;  // scale * log2(e)
+    int causal;
+    int n_pairs;       // 256-row query blocks per slice (grid z)
+};
+
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+    uint8_t *sptr = smem_raw + (sbase - raw_u32);
+    const uint32_t bars = sbase + C::kSmemTiles;
+    auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+    auto slot = [&](int s) -> uint32_t { return sbase + static_cast<uint32_t>(2 + s) * C::kTileBytes; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kSmemTiles + C::kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.z);  // heaviest causal blocks first
+    int start, len;
+    p.g.slice(b, start, len);
+    const int m0 = pair * 256;
+    if (m0 >= len) return;  // uniform for the CTA, before any barrier or allocation
+
+    const int nkv_all = (len + 127) / 128;
+    int nkv[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int r0 = m0 + 128 * t;
+        nkv[t] = (r0 >= len) ? 0 : (p.causal ? min(nkv_all, r0 / 128 + 1) : nkv_all);
+    }
+    const int nkv_max = max(nkv[0], nkv[1]);
+
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kNumBars; ++i) {
+            uint32_t cnt = 1;
+            if (i == C::kBarP || i == C::kBarP + 1) cnt = 128;
+            mbar_init(bar(i), cnt);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
+            mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTileBytes);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int x = 0; x < C::kBoxes; ++x)
+                    tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
+                                row0 + m0 + 128 * t, slab);
+            int n_issued = 0;  // loads 0 .. n_issued-1 were started (except a skipped one)
+            bool ok = true;
+            for (int j = 0; j < nkv_max && ok; ++j) {
+#pragma unroll
+                for (int kv = 0; kv < 2; ++kv) {
+                    const int idx = 2 * j + kv, s = idx % C::kStages;
+                    if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
+                    mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
+#pragma unroll
+                    for (int x = 0; x < C::kBoxes; ++x)
+                        tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
+                                    row0 + 128 * j, slab);
+                    n_issued = idx + 1;
+                }
+            }
+            if (*abort_flag) {
+                // Drain: every copy this thread started must land before the CTA exits.
+                for (int s = 0; s < C::kStages; ++s) {
+                    // newest load started in slot s
+                    int last = n_issued - 1 - ((n_issued - 1 - s) % C::kStages + C::kStages) % C::kStages;
+                    if (last == p.ctl.inject_skip_load) last -= C::kStages;
+                    if (last >= 0) drain_phase(bar(C::kBarFull + s), (last / C::kStages) & 1, p.ctl, abort_flag);
+                }
+                drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t colS[2] = {C::kColS0, C::kColS1};
+            const uint32_t colO[2] = {C::kColO0, C::kColO1};
+            auto issue_S = [&](int t, int j) {
+                const uint32_t qs = sbase + t * C::kTileBytes;
+                const uint32_t ks = slot((2 * j) % C::kStages);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024), idS,
+                           kk > 0);
+                }
+                tc_commit(bar(C::kBarS + t));
+            };
+            auto issue_PV = [&](int t, int j) {
+                const uint32_t vs = slot((2 * j + 1) % C::kStages);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sw128_desc(vs + kk * 2048, 16384, 1024), idPV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = wait_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+            if (ok) ok = wait_phase(bar(C::kBarFull + 0), 0, p.ctl, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t)
+                    if (nkv[t] > 0) issue_S(t, 0);
+                tc_commit(bar(C::kBarEmpty + 0));
+            }
+            for (int j = 0; ok && j < nkv_max; ++j) {
+                const int vidx = 2 * j + 1, kidx = 2 * j + 2;
+                ok = wait_phase(bar(C::kBarFull + vidx % C::kStages), (vidx / C::kStages) & 1, p.ctl, abort_flag);
+                if (!ok) break;
+                bool k_next = false;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j < nkv[t]) {
+                        ok = wait_phase(bar(C::kBarP + t), j & 1, p.ctl, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_PV(t, j);
+                        if (j == nkv[t] - 1) tc_commit(bar(C::kBarO + t));
+                    }
+                    if (j + 1 < nkv[t]) {
+                        if (!k_next) {
+                            ok = wait_phase(bar(C::kBarFull + kidx % C::kStages), (kidx / C::kStages) & 1, p.ctl,
+                                            abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            k_next = true;
+                        }
+                        issue_S(t, j + 1);
+                    }
+                }
+                if (!ok) break;
+                tc_commit(bar(C::kBarEmpty + vidx % C::kStages));
+                if (k_next) tc_commit(bar(C::kBarEmpty + kidx % C::kStages));
+            }
+            // Every MMA issued above must have finished before TMEM / smem go away.
+            tc_commit(bar(C::kBarDone));
+            drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int t = warp >> 2, q4 = warp & 3;
+        const int row = m0 + 128 * t + q4 * 32 + lane;  // query row within the slice
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const uint32_t tS = tmem + lane_off + (t ? C::kColS1 : C::kColS0);
+        const uint32_t tO = tmem + lane_off + (t ? C::kColO1 : C::kColO0);
+        const float c2 = p.scale_log2;
+        const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(b, start) : nullptr;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv[t]; ++j) {
+            ok = wait_phase(bar(C::kBarS + t), j & 1, p.ctl, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+            tmem_wait_ld();
+            float s[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+
+            // ---- masking: keys outside the sequence, above the diagonal, or padded
+            const int kbase = j * 128;
+            int limit = len - kbase;
+            if (p.causal) limit = min(limit, row - kbase + 1);
+            if (limit < 128) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= limit) s[c] = -INFINITY;
+            }
+            if (keep != nullptr) {
+                const int kl = len - kbase;  // keys of this tile inside the sequence
+                uint32_t kmask[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = q * 32 + lane;
+                    const bool kept = (c < kl) && keep[kbase + c] != 0;
+                    kmask[q] = __ballot_sync(0xffffffffu, kept);
+                }
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (!((kmask[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+            }
+
+            // ---- running max with lazy correction
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            const float m_cand = mx * c2;
+            const bool need = m_cand > m_used + kRescaleThreshold;
+            const bool warp_rescale = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (need) {
+                alpha = ex2_approx(m_used - m_cand);  // m_used == -inf gives 0
+                m_used = m_cand;
+                l *= alpha;
+            }
+            const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+
+            // ---- probabilities (bf16) into TMEM over S, and the row sum
+            float sum = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * c], c2, -m_use));
+                    const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * c + 1], c2, -m_use));
+                    sum += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS + half * 32, pk);
+            }
+            l += sum;
+            // Lazy correction of O_t, after the scores are dead (fewer live registers)
+            // but before P_t is published: PV_t(j) is issued only after the arrive.
+            if (warp_rescale && j > 0) {
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + q * 32, orr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+                    tmem_st32(tO + q * 32, orr);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarP + t));
+        }
+
+        // ---- epilogue: O / l in bf16, lse in natural log
+        if (ok && nkv[t] > 0) ok = wait_phase(bar(C::kBarO + t), 0, p.ctl, abort_flag);
+        if (ok && nkv[t] > 0) {
+            tc_fence_after();
+            const bool valid = row < len;
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+            __nv_bfloat16 *orow = p.o + p.g.base(b, h, start, D) + static_cast<long long>(row) * p.g.row_stride(D);
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t orr[32];
+                tmem_ld32(tO + q * 32, orr);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(__uint_as_float(orr[2 * c]) * inv, __uint_as_float(orr[2 * c + 1]) * inv);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            }
+            if (valid) p.lse[p.g.base(b, h, start, 1) + static_cast<long long>(row) * p.g.row_stride(1)] = lse_v;
+        }
+    }
+
+    __syncwarp();  // reconverge the single-lane roles before the CTA barrier
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
+    using C = FwdCfg<D>;
+    FwdParams p{};
+    p.g = a.g;
+    p.ctl = a.ctl;
+    p.o = static_cast<__nv_bfloat16 *>(a.o);
+    p.lse = a.lse;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.causal = a.causal;
+    p.n_pairs = (a.g.N + 255) / 256;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.g.H, a.g.B, p.n_pairs);
+    attn_fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {
+    if (a.g.d == 128) return launch_fwd_d<128>(a, stream);
+    return launch_fwd_d<64>(a, stream);
+}
+
+}  // namespace attn

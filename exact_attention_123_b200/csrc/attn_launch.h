@@ -1,0 +1,39 @@
+// attn_launch.h -- host-side launch descriptors passed from the C ABI layer to the
+// kernel launchers.  Internal to the library.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "attn_common.cuh"
+
+namespace attn {
+
+struct FwdLaunch {
+    CUtensorMap tm_q, tm_k, tm_v;  // 3-D bf16 maps, box {64, 128, 1}, 128-byte swizzle
+    Geom g;
+    SyncCtl ctl;
+    void *o;
+    float *lse;
+    float scale;
+    int causal;
+};
+
+struct BwdLaunch {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;  // same map shape as the forward
+    Geom g;
+    SyncCtl ctl;
+    const void *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    float *dq_acc;     // fp32 [rows, H, d] or [B, H, N, d] accumulator (workspace)
+    float *dvec;       // fp32 D_i = rowsum(dO o O), lse layout (workspace)
+    float *lse2;       // fp32 lse * log2(e), +inf for empty rows, lse layout (workspace)
+    long long rows_total;  // token rows (packed) or B*H*N (dense) of the lse layout
+    float scale;
+    int causal;
+};
+
+cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream);
+
+}  // namespace attn

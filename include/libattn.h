@@ -1,0 +1,181 @@
+/*
+ * libattn.h -- C ABI of a B200 (sm_100a) fused exact attention library.
+ *
+ * The operation is exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T + mask) V
+ *
+ * as stated by the standard_attention listing of "4.5 注意力优化实战：从PyTorch到
+ * CUDA的完整流程" (第一步 §1): Q, K, V of shape (batch, heads, seq_len, head_dim),
+ * scores scaled once, masked entries set to -inf, a row softmax, then a product
+ * with V.  It is computed as one fused, tiled pass with the running-max /
+ * running-sum ("online softmax") recurrence of the same page (第三步 §1) and of the
+ * codechina FlashAttention article (§3.2), so the [N, N] score matrix never
+ * reaches device memory.  The forward pass also saves, per query row, the
+ * natural-log logsumexp of the masked scaled scores; the backward pass uses it to
+ * recompute the probabilities ("4.5 注意力优化实战" 第四步 §2: the backward needs the
+ * softmax normaliser kept from the forward).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Element types: q, k, v, o, dout, dq, dk, dv are bf16 (2 bytes, IEEE-style
+ *   bfloat16); lse is fp32.  Accumulation is fp32.
+ * - head_dim d must be 64 or 128 (anything else returns ATTN_ERR_UNSUPPORTED).
+ * - scale must be finite and > 0 (typically 1/sqrt(d)).
+ * - Dense layout (cu_seqlens == NULL): tensors are contiguous [B, H, N, d];
+ *   lse is [B, H, N]; key_keep is [B, N].  N >= 1 is arbitrary.
+ * - Packed variable-length layout (cu_seqlens != NULL): B is the number of
+ *   sequences, N is an upper bound on every sequence length, cu_seqlens is a
+ *   DEVICE int32 array of B+1 non-decreasing offsets starting at 0; tensors are
+ *   token-major [total, H, d] with total = cu_seqlens[B]; lse is [total, H];
+ *   key_keep is [total].  Causal indices are local to each sequence.
+ *   The tile loader needs the token count on the host: the *_varlen entry
+ *   points take it as `total_tokens`; attn_fwd / attn_fwd_masked / attn_bwd
+ *   called with a non-NULL cu_seqlens assume total_tokens = B*N, i.e. the packed
+ *   buffers must then be allocated for B*N token rows (rows past
+ *   cu_seqlens[B] are read as padding but never written).
+ * - Causal masking: key j is visible to query i iff j <= i (lower triangle,
+ *   equal query/key lengths; "Profiling in PyTorch (part 3)", math backend
+ *   section, tril mask).
+ * - key_keep (nullable, DEVICE uint8): 1 = the key may be attended, 0 = masked
+ *   for every query.  A query row that sees no key at all gets O = 0 and
+ *   lse = -inf (never NaN), as the _safe_softmax discussion of the same page
+ *   asks; its gradients are 0 and it contributes nothing to dK/dV.
+ * - Ownership: every pointer is caller-owned DEVICE memory (except where noted);
+ *   the library allocates nothing per call and keeps no per-call state, so calls
+ *   on different streams are independent.  Base pointers must be 16-byte aligned.
+ * - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Every compute call is asynchronous on that stream.
+ * - Errors: a non-OK code returned from a call means nothing was launched
+ *   (argument errors) or a launch failed (ATTN_ERR_CUDA).  Faults detected on the
+ *   device (a bounded wait that expired) are reported by attn_status().  After a
+ *   non-OK status the outputs are unspecified.
+ */
+#ifndef LIBATTN_H
+#define LIBATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad scale       */
+    ATTN_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, or device is not sm_100      */
+    ATTN_ERR_MISALIGNED = 3,  /* a base pointer is not 16-byte aligned             */
+    ATTN_ERR_WORKSPACE = 4,   /* backward workspace missing or too small           */
+    ATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed       */
+    ATTN_ERR_TIMEOUT = 6      /* a device-side bounded wait expired (attn_status)  */
+} attn_status_t;
+
+/*
+ * Forward pass without a key mask.
+ *   q, k, v : inputs (bf16), layout per the conventions above.
+ *   o       : output (bf16), same layout as q.
+ *   lse     : output (fp32), natural-log logsumexp per query row; -inf for rows
+ *             that see no key.
+ *   B, H, N, d, scale, is_causal, cu_seqlens : as above (cu_seqlens nullable).
+ * Returns an attn_status_t code.
+ */
+ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int N, int d, float scale, int is_causal,
+             const int32_t *cu_seqlens, void *stream);
+
+/* Forward pass with an optional per-key padding mask (key_keep, nullable). */
+ATTN_API int attn_fwd_masked(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int B, int H, int N, int d, float scale, int is_causal,
+                    const int32_t *cu_seqlens, const uint8_t *key_keep, void *stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs for these sizes (for packed inputs,
+ * pass the same B and N as to attn_bwd; the bound B*N >= total is used).
+ * Returns 0 for invalid sizes.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass.  Recomputes the probabilities from q, k and the forward's lse,
+ * and writes the input gradients:
+ *   dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,
+ *   dK = scale dS^T Q.
+ *   o, lse     : the forward's outputs for the same inputs and masking.
+ *   dout       : upstream gradient dL/dO (bf16, layout of o).
+ *   dq, dk, dv : outputs (bf16, layout of q).
+ *   workspace  : caller-owned device memory of at least
+ *                attn_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
+ *                its contents are scratch (fp32 dQ accumulator and per-row
+ *                terms) and need no initialisation.
+ * Returns an attn_status_t code.
+ */
+ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+             const void *dout, void *dq, void *dk, void *dv,
+             int B, int H, int N, int d, float scale, int is_causal,
+             const int32_t *cu_seqlens, const uint8_t *key_keep,
+             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Packed variable-length forward with an exact token count.
+ *   num_seqs     : number of sequences (cu_seqlens has num_seqs+1 entries)
+ *   total_tokens : rows of the packed tensors (== cu_seqlens[num_seqs]); the
+ *                  tile loader never reads past this row
+ *   max_seqlen   : upper bound on every sequence length (grid sizing)
+ *   key_keep     : nullable, [total_tokens] uint8
+ * Other arguments as for attn_fwd_masked.
+ */
+ATTN_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int num_seqs, int total_tokens, int max_seqlen, int H, int d, float scale,
+                    int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
+                    void *stream);
+
+/* Workspace bytes for attn_bwd_varlen. Returns 0 for invalid sizes. */
+ATTN_API size_t attn_bwd_varlen_workspace_bytes(int total_tokens, int H, int d);
+
+/* Packed variable-length backward with an exact token count (see attn_fwd_varlen). */
+ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                    const void *dout, void *dq, void *dk, void *dv,
+                    int num_seqs, int total_tokens, int max_seqlen, int H, int d, float scale,
+                    int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait
+ * expired since the last call, or ATTN_ERR_CUDA if synchronisation failed.
+ */
+ATTN_API int attn_status(void *stream);
+
+/* Static, human-readable text for a status code (never NULL). */
+ATTN_API const char *attn_strerror(int code);
+
+/*
+ * Sets the device-side wait limit in milliseconds for later launches from this
+ * process (default 4000).  A kernel whose wait on a pipeline barrier exceeds the
+ * limit stops, records ATTN_ERR_TIMEOUT and returns.  ms <= 0 restores the
+ * default.  Returns the previous value.
+ */
+ATTN_API int attn_set_wait_limit_ms(int ms);
+
+/*
+ * Test hook for the failure-detection path.  For later forward launches from this
+ * process, the tile loader skips pipeline load number `load_index` (counting the
+ * K and V tile loads of one CTA from 0), so that slot never fills and the
+ * consumer's bounded wait expires; every kernel then stops cleanly and
+ * attn_status() reports ATTN_ERR_TIMEOUT.  -1 (the default) disables it.
+ * Returns the previous value.  Nothing faults: all waits are time-limited.
+ */
+ATTN_API int attn_debug_skip_load(int load_index);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBATTN_H */

@@ -1,0 +1,109 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "libattn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_attention_123_b200 import build
+    build.build()
+    import exact_attention_123_b200 as ea
+    return ea.lib()
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
+              "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(ROOT, "exact_attention_123_b200", "libattn.so")],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(L, n)
+    # nothing else of ours leaks out of the library
+    ours = {e for e in exported if e.startswith("attn")}
+    assert ours == set(declared_functions())
+
+
+def test_header_compiles_as_c(tmp_path):
+    c = tmp_path / "t.c"
+    c.write_text('#include "libattn.h"\nint main(void){return ATTN_OK;}\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-c", str(c),
+                    "-o", str(tmp_path / "t.o")], check=True)
+
+
+def test_strerror_and_workspace_sizes(L):
+    import exact_attention_123_b200 as ea
+    for code in range(0, 8):
+        assert isinstance(ea.attn_strerror(code), str) and ea.attn_strerror(code)
+    assert ea.attn_bwd_workspace_bytes(2, 16, 4096, 128) >= 2 * 16 * 4096 * 128 * 4 + 2 * 2 * 16 * 4096 * 4
+    assert ea.attn_bwd_workspace_bytes(1, 1, 1, 96) == 0
+    assert ea.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
+    assert ea.attn_bwd_varlen_workspace_bytes(1000, 4, 64) >= 1000 * 4 * 64 * 4
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails host validation first
+
+
+def fwd(L, ptrs, B=1, H=1, N=16, d=64, scale=0.125):
+    vp = [ctypes.c_void_p(p) if p else None for p in ptrs]
+    return L.attn_fwd(*vp, B, H, N, d, ctypes.c_float(scale), 1, None, None)
+
+
+def test_host_argument_errors(L):
+    import exact_attention_123_b200 as ea
+    good = [FAKE] * 5
+    assert fwd(L, [0, FAKE, FAKE, FAKE, FAKE]) == ea.ATTN_ERR_INVALID_ARG
+    assert fwd(L, good, B=0) == ea.ATTN_ERR_INVALID_ARG
+    assert fwd(L, good, N=-3) == ea.ATTN_ERR_INVALID_ARG
+    assert fwd(L, good, scale=0.0) == ea.ATTN_ERR_INVALID_ARG
+    assert fwd(L, good, scale=float("nan")) == ea.ATTN_ERR_INVALID_ARG
+    assert fwd(L, good, d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert fwd(L, good, d=256) == ea.ATTN_ERR_UNSUPPORTED
+    assert fwd(L, [FAKE + 8] + [FAKE] * 4) == ea.ATTN_ERR_MISALIGNED
+    vp = ctypes.c_void_p
+    # varlen entry points need cu_seqlens
+    assert L.attn_fwd_varlen(vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), 2, 10, 8, 1, 64,
+                             ctypes.c_float(0.1), 1, None, None, None) == ea.ATTN_ERR_INVALID_ARG
+    # backward: workspace missing / too small / misaligned
+    args = [vp(FAKE)] * 9 + [1, 1, 16, 64, ctypes.c_float(0.125), 1, None, None]
+    assert L.attn_bwd(*args, None, 0, None) == ea.ATTN_ERR_WORKSPACE
+    assert L.attn_bwd(*args, vp(FAKE), 16, None) == ea.ATTN_ERR_WORKSPACE
+    need = ea.attn_bwd_workspace_bytes(1, 1, 16, 64)
+    assert L.attn_bwd(*args, vp(FAKE + 16), need, None) == ea.ATTN_ERR_MISALIGNED
+
+
+def test_wait_limit_and_fault_hook_setters(L):
+    import exact_attention_123_b200 as ea
+    prev = ea.attn_set_wait_limit_ms(1234)
+    assert ea.attn_set_wait_limit_ms(prev) == 1234
+    assert ea.attn_debug_skip_load(5) == -1
+    assert ea.attn_debug_skip_load(-1) == 5
+
+
+def test_product_package_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "exact_attention_123_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", txt, re.M), f
+                assert "liboracle" not in txt, f
