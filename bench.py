@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Throughput of the fused exact-attention hot path (forward + backward) on B200.
+
+One step = one forward and one backward pass of causal bf16 attention over one
+batch of B=2, H=16, N=4096, d=128 (Q, K, V, dO ~ N(0,1), seeded), i.e. every
+kernel of the path: the fused forward, the backward's preprocessing, main and
+dQ-conversion kernels.  FLOPs follow the usual convention: forward
+2*B*H*N^2*d for causal (4*B*H*N^2*d non-causal), backward 2.5x the forward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own batch
+(weak scaling, no data-path collective); times are the max over ranks.
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same
+workload instead (the only other place this script runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+B, H, N, D = 2, 16, 4096, 128
+CAUSAL = True
+SEED = 5
+METRIC = "causal bf16 attention fwd/bwd TFLOPS at N=4096,d=128; % of B200 tensor peak"
+UNIT = "TFLOPS"
+WORKLOAD = "causal attention fwd+bwd B2 H16 N4096 d128 bf16, Q/K/V/dO ~ N(0,1)"
+
+
+def flops_fwd(b=B, h=H, n=N, d=D, causal=CAUSAL):
+    return (2.0 if causal else 4.0) * b * h * n * n * d
+
+
+def flops_bwd(b=B, h=H, n=N, d=D, causal=CAUSAL):
+    return 2.5 * flops_fwd(b, h, n, d, causal)
+
+
+def measured_peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # no NVML: clocks reported as unavailable
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+def time_oracle_sample(n_heads: int):
+    """float64 oracle forward + backward on the first n_heads (b, h) slices of the
+    workload, all host cores.  Returns (TFLOPS, seconds, cores, sample text)."""
+    import oracle
+    from attn_inputs import make_dense
+    inp = make_dense(B, H, N, D, seed=SEED, causal=CAUSAL, with_grad=True)
+    threads = oracle.default_threads()
+    picks = list(range(n_heads))
+    t0 = time.perf_counter()
+    oracle.fwd(inp.q, inp.k, inp.v, inp.scale, CAUSAL, slices=picks, nthreads=threads)
+    oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, CAUSAL, slices=picks, nthreads=threads)
+    dt = time.perf_counter() - t0
+    fl = flops_fwd(1, n_heads) + flops_bwd(1, n_heads)
+    return fl / dt / 1e12, dt, threads, f"{n_heads} of {B * H} (b,h) slices at N={N}, d={D}, fwd+bwd"
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    threads = oracle.default_threads()
+    vals = []
+    for s in range(args.warmup + args.steps):
+        v, dt, cores, sample = time_oracle_sample(1)
+        if s >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.median(v for v, _ in vals)
+    total_s = sum(dt for _, dt in vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / max(1, len(vals)), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "causal": CAUSAL},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "per step: 1 of 32 (b,h) slices at N=4096, d=128, fwd+bwd, float64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def source_digest():
+    h = hashlib.sha256()
+    for f in ("attn_bwd_sm100.cu", "attn_fwd_sm100.cu", "sm100_ptx.cuh", "attn_common.cuh"):
+        with open(os.path.join(HERE, "exact_attention_123_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on the
+    current kernel sources; otherwise None."""
+    p = os.path.join(HERE, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(kernel)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from exact_attention_123_b200 import build
+    if rank == 0:
+        build.build()
+    if ws > 1:
+        dist.barrier()
+    import exact_attention_123_b200 as ea
+    from attn_inputs import make_dense
+
+    inp = make_dense(B, H, N, D, seed=SEED + 1000 * rank, causal=CAUSAL, with_grad=True)
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.do))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsbuf = ea.workspace_for(q)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(scale=inp.scale, causal=CAUSAL, stream=stream)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ea.attn_fwd(q, k, v, o, lse, **kw)
+        if ev is not None:
+            ev[1].record(stream)
+        ea.attn_bwd_phase(0, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
+        if ev is not None:
+            ev[2].record(stream)
+        ea.attn_bwd_phase(1, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
+        if ev is not None:
+            ev[3].record(stream)
+        ea.attn_bwd_phase(2, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = ea.attn_status(stream)
+    if st != ea.ATTN_OK:
+        raise RuntimeError(f"warm-up reported status {st}: {ea.attn_strerror(st)}")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for s in range(args.steps):
+            flush.zero_()          # L2 flushed before every step, outside the event bracket
+            step(events[s])
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    if ws > 1:
+        dist.barrier()
+    st = ea.attn_status(stream)
+    if st != ea.ATTN_OK:
+        raise RuntimeError(f"timed steps reported status {st}: {ea.attn_strerror(st)}")
+
+    seg = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events]  # ms: fwd, pre, main, dq
+    step_ms = [sum(x) for x in seg]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    pin = {n: x.cpu().pin_memory() for n, x in (("q", q), ("k", k), ("v", v), ("do", do))}
+    outs = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for n, x in (("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(x.numel() * x.element_size() for x in pin.values())
+    d2h = sum(x.numel() * x.element_size() for x in outs.values())
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        do.copy_(pin["do"], non_blocking=True)
+        ea.attn_fwd(q, k, v, o, lse, **kw)
+        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
+        outs["dq"].copy_(dq, non_blocking=True)
+        outs["dk"].copy_(dk, non_blocking=True)
+        outs["dv"].copy_(dv, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_n = max(3, args.e2e_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_n):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    st = ea.attn_status(stream)
+    if st != ea.ATTN_OK:
+        raise RuntimeError(f"end-to-end steps reported status {st}")
+
+    step_flops = flops_fwd() + flops_bwd()
+    value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12
+    e2e_value = step_flops * e2e_n * ws / (float(e2e_ms.item()) * 1e-3) / 1e12
+
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    fwd_ms = statistics.mean(x[0] for x in seg)
+    pre_ms = statistics.mean(x[1] for x in seg)
+    main_ms = statistics.mean(x[2] for x in seg)
+    dq_ms = statistics.mean(x[3] for x in seg)
+    fwd_tf = flops_fwd() / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = flops_bwd() / ((pre_ms + main_ms + dq_ms) * 1e-3) / 1e12
+    main_tf = flops_bwd() / (main_ms * 1e-3) / 1e12
+    dominant = "attn_bwd_main_kernel" if main_ms >= fwd_ms else "attn_fwd_sm100_kernel"
+    dom_tf = main_tf if dominant == "attn_bwd_main_kernel" else fwd_tf
+
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if ws == 1 and not args.no_cpu_baseline:
+        cv, cdt, cores, sample = time_oracle_sample(args.cpu_heads)
+        cpu = {"value": cv, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(cdt, 3)}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "causal": CAUSAL, "seed": SEED,
+                   "l2": "flushed (256 MiB write) before every timed step, outside the timed bracket",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "breakdown_ms": {"fwd": fwd_ms, "bwd_pre": pre_ms, "bwd_main": main_ms, "bwd_dq": dq_ms},
+        "tflops": {"fwd": fwd_tf, "bwd": bwd_tf, "bwd_main": main_tf},
+        "pct_of_peak": {"fwd": 100 * fwd_tf / peak, "bwd": 100 * bwd_tf / peak, "step": 100 * value / ws / peak,
+                        "peak": f"{peak} TFLOPS bf16 dense ({peak_src}, burst)"},
+        "roofline": {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": dom_tf / peak, "traffic": recorded_traffic(dominant),
+                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src}, burst)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_n},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": wall,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-heads", type=int, default=4, help="(b,h) slices in the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

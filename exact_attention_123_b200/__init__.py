@@ -6,7 +6,7 @@ current stream.  There is no CPU or library fallback: if ``libattn.so`` is
 missing, importing the entry points raises.
 
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
-``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_workspace_bytes``,
+``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
 ``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
 """
@@ -58,12 +58,13 @@ def lib() -> ctypes.CDLL:
     L.attn_bwd_varlen_workspace_bytes.restype = sz
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
+    L.attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
     L.attn_strerror.restype = ctypes.c_char_p
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
-    for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen",
+    for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen", "attn_bwd_phase",
                  "attn_status", "attn_set_wait_limit_ms", "attn_debug_skip_load"):
         getattr(L, name).restype = i
     _lib = L
@@ -189,6 +190,24 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
                             workspace.numel(), _stream(stream))
         _check(rc, "attn_bwd")
     return dq, dk, dv
+
+
+def attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, *, workspace, scale: Optional[float] = None,
+                   causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
+                   stream=None):
+    """Launch one backward phase (0 preprocess, 1 main, 2 dQ conversion)."""
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if cu_seqlens is not None:
+        nseq, total, H, N = cu_seqlens.numel() - 1, q.shape[0], q.shape[1], int(max_seqlen)
+    else:
+        nseq, H, N, _ = q.shape
+        total = 0
+    rc = lib().attn_bwd_phase(int(phase), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                              _ptr(dk), _ptr(dv), nseq, total, N, H, d, float(scale), int(causal), _ptr(cu_seqlens),
+                              _ptr(key_keep), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "attn_bwd_phase")
 
 
 def attn_status(stream=None) -> int:

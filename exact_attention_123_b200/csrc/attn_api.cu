@@ -67,14 +67,14 @@ int device_state(DeviceState **out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 3-D map (col, row, slab) over a bf16 tensor; box = 64 columns x 128 rows x 1.
+// 3-D map (col, row, slab) over a bf16 tensor; box = 64 columns x box_rows rows x 1.
 int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long slabs, long long row_stride,
-             long long slab_stride) {
+             long long slab_stride, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return ATTN_ERR_CUDA;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2, static_cast<cuuint64_t>(slab_stride) * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -88,9 +88,10 @@ struct Shape {
     const int32_t *cu;
 };
 
-int map_for(CUtensorMap *m, const void *base, const Shape &s) {
-    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d);
-    return make_map(m, base, s.d, s.N, static_cast<long long>(s.B) * s.H, s.d, static_cast<long long>(s.N) * s.d);
+int map_for(CUtensorMap *m, const void *base, const Shape &s, int box_rows = 128) {
+    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d, box_rows);
+    return make_map(m, base, s.d, s.N, static_cast<long long>(s.B) * s.H, s.d, static_cast<long long>(s.N) * s.d,
+                    box_rows);
 }
 
 int check_common(const Shape &s, float scale) {
@@ -98,8 +99,8 @@ int check_common(const Shape &s, float scale) {
     if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     if (s.cu && s.total < 0) return ATTN_ERR_INVALID_ARG;
     if (s.d != 64 && s.d != 128) return ATTN_ERR_UNSUPPORTED;
-    // grid limits: B <= 65535 (grid y), H <= 2^31-1, N/256 <= 65535 (grid z)
-    if (s.B > 65535 || (s.N + 255) / 256 > 65535) return ATTN_ERR_UNSUPPORTED;
+    // grid limits: B <= 65535 (grid y), H <= 2^31-1, N/128 <= 65535 (grid z)
+    if (s.B > 65535 || (s.N + 127) / 128 > 65535) return ATTN_ERR_UNSUPPORTED;
     // TMA extents are 32-bit
     if (s.cu ? s.total > 0x7fffffffLL : static_cast<long long>(s.B) * s.H > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     return ATTN_OK;
@@ -154,7 +155,7 @@ size_t bwd_ws_bytes(long long rows_x_heads, int d) {
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
              void *dq, void *dk, void *dv, const Shape &s, float scale, int is_causal, const uint8_t *key_keep,
-             void *workspace, size_t workspace_bytes, void *stream) {
+             void *workspace, size_t workspace_bytes, void *stream, int phases = 7) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -169,8 +170,9 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     if ((rc = device_state(&ds))) return rc;
     if (s.cu && s.total == 0) return ATTN_OK;
     attn::BwdLaunch a{};
-    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
-        (rc = map_for(&a.tm_do, dout, s)))
+    // the backward sweeps 64-row query tiles against 128-row key tiles
+    if ((rc = map_for(&a.tm_q, q, s, 64)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
+        (rc = map_for(&a.tm_do, dout, s, 64)))
         return rc;
     a.g = geom_of(s, key_keep);
     a.ctl = ctl_of(ds);
@@ -188,6 +190,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     a.rows_total = rows;
     a.scale = scale;
     a.causal = is_causal ? 1 : 0;
+    a.phases = phases;
     return attn::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -241,6 +244,16 @@ int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, 
     Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
                     stream);
+}
+
+int attn_bwd_phase(int phase, const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, int num_seqs, int total_tokens, int max_seqlen,
+                   int H, int d, float scale, int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
+                   void *workspace, size_t workspace_bytes, void *stream) {
+    if (phase < 0 || phase > 2) return ATTN_ERR_INVALID_ARG;
+    Shape s{num_seqs, H, max_seqlen, d, cu_seqlens ? static_cast<long long>(total_tokens) : 0, cu_seqlens};
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
+                    stream, 1 << phase);
 }
 
 int attn_status(void *stream) {

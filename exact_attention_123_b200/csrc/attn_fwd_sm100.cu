@@ -126,6 +126,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    int n_issued = 0;  // producer: ring loads 0 .. n_issued-1 were started (except a skipped one)
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
@@ -141,7 +142,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int x = 0; x < C::kBoxes; ++x)
                     tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
                                 row0 + m0 + 128 * t, slab);
-            int n_issued = 0;  // loads 0 .. n_issued-1 were started (except a skipped one)
             bool ok = true;
             for (int j = 0; j < nkv_max && ok; ++j) {
 #pragma unroll
@@ -159,16 +159,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                     row0 + 128 * j, slab);
                     n_issued = idx + 1;
                 }
-            }
-            if (*abort_flag) {
-                // Drain: every copy this thread started must land before the CTA exits.
-                for (int s = 0; s < C::kStages; ++s) {
-                    // newest load started in slot s
-                    int last = n_issued - 1 - ((n_issued - 1 - s) % C::kStages + C::kStages) % C::kStages;
-                    if (last == p.ctl.inject_skip_load) last -= C::kStages;
-                    if (last >= 0) drain_phase(bar(C::kBarFull + s), (last / C::kStages) & 1, p.ctl, abort_flag);
-                }
-                drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
             }
         }
     } else if (warp == 9) {
@@ -361,6 +351,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncwarp();  // reconverge the single-lane roles before the CTA barrier
     tc_fence_before();
     __syncthreads();
+    if (warp == 8 && lane == 0 && *abort_flag) {
+        // After an abort, every copy the producer started must land before the CTA
+        // exits (the flag is final here: every role has finished).
+        for (int s = 0; s < C::kStages; ++s) {
+            int last = n_issued - 1 - ((n_issued - 1 - s) % C::kStages + C::kStages) % C::kStages;
+            if (last == p.ctl.inject_skip_load) last -= C::kStages;
+            if (last >= 0) drain_phase(bar(C::kBarFull + s), (last / C::kStages) & 1, p.ctl, abort_flag);
+        }
+        drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+    }
     if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

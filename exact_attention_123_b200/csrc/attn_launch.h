@@ -19,7 +19,7 @@ struct FwdLaunch {
 };
 
 struct BwdLaunch {
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;  // same map shape as the forward
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;  // K, V: 128-row boxes; Q, dO: 64-row boxes
     Geom g;
     SyncCtl ctl;
     const void *o, *dout;
@@ -31,6 +31,7 @@ struct BwdLaunch {
     long long rows_total;  // token rows (packed) or B*H*N (dense) of the lse layout
     float scale;
     int causal;
+    int phases;        // bit 0: preprocess, bit 1: main kernel, bit 2: dQ conversion
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);

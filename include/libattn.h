@@ -147,6 +147,23 @@ ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const 
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * One of the backward's three kernels (attn_bwd / attn_bwd_varlen launch all three
+ * in this order); lets a caller time or schedule them separately.
+ *   phase 0 : per-row terms D_i = rowsum(dO o O) and lse2 = lse*log2(e), and a
+ *             zeroed fp32 dQ accumulator, all in `workspace`
+ *   phase 1 : main kernel: dK, dV (written) and dQ (accumulated in `workspace`)
+ *   phase 2 : dQ = scale * accumulator, written as bf16
+ * Phases must run in order on the same workspace and stream.  Other arguments as
+ * attn_bwd_varlen; for the dense layout pass cu_seqlens = NULL, num_seqs = B,
+ * max_seqlen = N and total_tokens = 0.
+ */
+ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void *v, const void *o,
+                            const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                            int num_seqs, int total_tokens, int max_seqlen, int H, int d, float scale,
+                            int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait
  * expired since the last call, or ATTN_ERR_CUDA if synchronisation failed.

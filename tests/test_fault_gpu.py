@@ -1,0 +1,44 @@
+"""Failure detection without a GPU fault.
+
+The loader is told (through a test hook) to skip one pipeline load, so the slot
+it would have filled never fills.  The consumer's bounded wait expires after the
+short limit set here, every role of the kernel stops cleanly, and the host reads
+ATTN_ERR_TIMEOUT from attn_status().  The context stays usable: the next call
+succeeds and matches the oracle.  Nothing traps, faults or waits forever.
+"""
+import pytest
+import torch
+
+import oracle
+from attn_inputs import make_dense
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ea():
+    from exact_attention_123_b200 import build
+    build.build()
+    import exact_attention_123_b200 as m
+    return m
+
+
+@pytest.mark.parametrize("skip", [0, 1, 3])
+def test_expired_wait_reports_timeout_and_context_survives(ea, skip):
+    inp = make_dense(1, 2, 384, 128, seed=7000)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    assert ea.attn_status() == ea.ATTN_OK
+    prev_limit = ea.attn_set_wait_limit_ms(200)
+    ea.attn_debug_skip_load(skip)
+    try:
+        ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
+        assert ea.attn_status() == ea.ATTN_ERR_TIMEOUT
+        assert ea.attn_status() == ea.ATTN_OK  # reading clears it
+    finally:
+        ea.attn_debug_skip_load(-1)
+        ea.attn_set_wait_limit_ms(prev_limit)
+    o, lse = ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
+    assert ea.attn_status() == ea.ATTN_OK
+    ro, _ = oracle.fwd(inp.q, inp.k, inp.v, inp.scale, True)
+    err = (o.double().cpu().numpy() - ro)
+    assert abs(err).max() < 2e-2
