@@ -67,18 +67,20 @@ int device_state(DeviceState **out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 3-D map (col, row, slab) over a bf16 tensor; box = 64 columns x box_rows rows x 1.
+// 3-D map (col, row, slab) with a 128-byte swizzle; box = one 128-byte column group
+// (64 bf16 or 32 fp32 elements) x box_rows rows x 1.  Strides are in elements.
 int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long slabs, long long row_stride,
-             long long slab_stride, int box_rows) {
+             long long slab_stride, int box_rows, bool fp32 = false) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return ATTN_ERR_CUDA;
+    const cuuint64_t esz = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2, static_cast<cuuint64_t>(slab_stride) * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * esz, static_cast<cuuint64_t>(slab_stride) * esz};
+    cuuint32_t box[3] = {fp32 ? 32u : 64u, static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -88,10 +90,10 @@ struct Shape {
     const int32_t *cu;
 };
 
-int map_for(CUtensorMap *m, const void *base, const Shape &s, int box_rows = 128) {
-    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d, box_rows);
+int map_for(CUtensorMap *m, const void *base, const Shape &s, int box_rows = 128, bool fp32 = false) {
+    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d, box_rows, fp32);
     return make_map(m, base, s.d, s.N, static_cast<long long>(s.B) * s.H, s.d, static_cast<long long>(s.N) * s.d,
-                    box_rows);
+                    box_rows, fp32);
 }
 
 int check_common(const Shape &s, float scale) {
@@ -185,6 +187,8 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     char *w = static_cast<char *>(workspace);
     a.dq_acc = reinterpret_cast<float *>(w);
+    // the accumulator has the layout of q (row pitch d), in fp32
+    if ((rc = map_for(&a.tm_dqacc, a.dq_acc, s, 64, true))) return rc;
     a.dvec = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4));
     a.lse2 = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4) + up(static_cast<size_t>(rows) * 4));
     a.rows_total = rows;

@@ -23,7 +23,8 @@
 //        dV  += P^T  dO_i      (M=128, N=d, K=64)                   -> TMEM
 //        dK  += dS^T Q_i       (M=128, N=d, K=64)                   -> TMEM
 //        dQ_i = dS K_j         (M=64,  N=d, K=128)                  -> TMEM, then
-//               added into the fp32 accumulator with vector atomics by 4 warps
+//               staged in shared memory by 4 warps and added into the fp32
+//               accumulator with bulk tensor reduce-adds (TMA)
 //      and finally writes dV and scale*dK in bf16.
 //   3. attn_bwd_dq_kernel    dQ = bf16(scale * accumulator).  HBM-bound.
 //
@@ -33,7 +34,8 @@
 // copied the current ones into registers, and overlap its softmax work.
 //
 // Warp roles (448 threads): warps 0-7 probabilities/dS (warp w: key rows
-// 32*(w%4).., query columns 32*(w/4)..), warps 8-11 dQ drain and the dK/dV
+// 32*(w%4).., query columns 32*(w/4)..), warps 8-11 dQ drain (thread 256 issues
+// the bulk reductions) and the dK/dV
 // epilogue, warp 12 loader (TMA for K, V, Q, dO; plain loads for lse2/D),
 // warp 13 TMEM allocator and MMA issuer.
 #include <cuda_bf16.h>
@@ -133,7 +135,9 @@ struct BwdCfg {
     static constexpr int kOffP = kOffDO + kStages * kQBytes;           // + b * kPSBytes
     static constexpr int kOffDS = kOffP + 2 * kPSBytes;                // + b * kPSBytes
     static constexpr int kOffVec = kOffDS + 2 * kPSBytes;              // + st * 512: lse2[64], D[64]
-    static constexpr int kOffBar = kOffVec + kStages * 512;
+    static constexpr int kOffDQ = kOffVec + kStages * 512;             // fp32 dQ stage: d/32 boxes of 64x32
+    static constexpr int kDQBox = 64 * 128;
+    static constexpr int kOffBar = kOffDQ + (D / 32) * kDQBox;
     // barriers
     static constexpr int kBarKV = 0;
     static constexpr int kBarQFull = 1;    // + st
@@ -146,7 +150,9 @@ struct BwdCfg {
     static constexpr int kBarDqEmpty = 12;
     static constexpr int kBarKdv = 13;
     static constexpr int kBarDone = 14;
-    static constexpr int kNumBars = 15;
+    static constexpr int kBarStageFull = 15;  // dQ stage written (128 drain threads)
+    static constexpr int kBarStageFree = 16;  // dQ stage read by the bulk reduce (leader)
+    static constexpr int kNumBars = 17;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
 };
 
@@ -166,7 +172,7 @@ template <int D>
 __global__ void __launch_bounds__(448, 1)
 attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const __grid_constant__ BwdParams p) {
+                     const __grid_constant__ CUtensorMap tm_dqacc, const __grid_constant__ BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -194,7 +200,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int i = 0; i < C::kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i == C::kBarSdpFree || i == C::kBarPsFull || i == C::kBarPsFull + 1) cnt = 256;
-            if (i == C::kBarDqEmpty) cnt = 128;
+            if (i == C::kBarDqEmpty || i == C::kBarStageFull) cnt = 128;
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
@@ -375,50 +381,69 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarPsEmpty + pb), ((it >> 1) & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
             // 128-byte swizzled K-major rows: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
-            uint8_t *prow = sptr + C::kOffP + pb * C::kPSBytes + kr * 128;
-            uint8_t *drow = sptr + C::kOffDS + pb * C::kPSBytes + kr * 128;
+            const uint32_t prow = sbase + C::kOffP + pb * C::kPSBytes + kr * 128;
+            const uint32_t drow = sbase + C::kOffDS + pb * C::kPSBytes + kr * 128;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int chunk = (hf * 4 + u) ^ (kr & 7);
-                *reinterpret_cast<uint4 *>(prow + chunk * 16) =
-                    make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-                *reinterpret_cast<uint4 *>(drow + chunk * 16) =
-                    make_uint4(dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2], dsp[4 * u + 3]);
+                const uint32_t chunk = static_cast<uint32_t>((hf * 4 + u) ^ (kr & 7)) << 4;
+                st_shared_v4(prow + chunk, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
+                st_shared_v4(drow + chunk, dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2], dsp[4 * u + 3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(C::kBarPsFull + pb));
         }
     } else {
         // ------------------------------------------------------------ dQ drain + dK/dV epilogue
+        // Each dQ_i tile (fp32, M = 64) goes TMEM -> registers -> a 128-byte swizzled
+        // shared-memory stage -> one bulk tensor reduce-add per 32-column box into the
+        // fp32 accumulator (the L2 does the additions line by line).  Query rows past
+        // the sequence hold exact zeros (their P is 0), so adding them is harmless.
         const int q4 = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const bool leader = threadIdx.x == 256;
+        const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
+        const uint32_t stage = sbase + C::kOffDQ;
+        const int r = q4 * 16 + lane;  // M = 64 accumulator: row r sits in TMEM lane (r % 16) + 32 * (r / 16)
         bool ok = true;
         for (int it = 0; it < nq; ++it) {
             ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDqFull), it & 1, p.ctl, abort_flag));
+            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarStageFree), (it & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            // M = 64 accumulator layout: row r sits in TMEM lane (r % 16) + 32 * (r / 16)
-            const int qrow = (i0 + it) * 64 + q4 * 16 + lane;
-            const bool valid = lane < 16 && qrow < len;
-            float *dst = p.dq_acc + (lrow0 + static_cast<long long>(qrow) * lrs) * D;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + C::kColDQ + c0, r);
+            for (int x = 0; x < D / 32; ++x) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + C::kColDQ + x * 32, v);
                 tmem_wait_ld();
-                if (c0 + 32 >= D) {
+                if (x == D / 32 - 1) {
                     tc_fence_before();
                     mbar_arrive(bar(C::kBarDqEmpty));
                 }
-                if (valid) {
+                if (lane < 16) {
+                    const uint32_t rowa = stage + x * C::kDQBox + r * 128;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + c0 + 4 * v),
-                                  make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                              __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+                    for (int k = 0; k < 8; ++k)
+                        st_shared_v4(rowa + ((static_cast<uint32_t>(k ^ (r & 7))) << 4), v[4 * k], v[4 * k + 1],
+                                     v[4 * k + 2], v[4 * k + 3]);
                 }
             }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(C::kBarStageFull));
+            if (leader) {
+                ok = wait_phase(bar(C::kBarStageFull), it & 1, p.ctl, abort_flag);
+                if (ok) {
+                    const int q0 = (i0 + it) * 64;
+#pragma unroll
+                    for (int x = 0; x < D / 32; ++x) tma_reduce_add_3d(&tm_dqacc, stage + x * C::kDQBox, x * 32, row0 + q0, slab);
+                    bulk_commit();
+                    bulk_wait_read0();
+                }
+                mbar_arrive(bar(C::kBarStageFree));
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
         }
+        if (leader) bulk_wait0();  // the accumulator updates are complete before the CTA exits
         if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKdv), 0, p.ctl, abort_flag));
         if (ok) {
             tc_fence_after();
@@ -496,7 +521,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
         dim3 grid(a.g.H, a.g.B, p.n_kv);
-        attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+        attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do,
+                                                                             a.tm_dqacc, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -273,9 +273,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
 
             // ---- running max with lazy correction
-            float mx = s[0];
+            // four independent 3-input max chains (short dependency chains: one warp per
+            // scheduler runs this, so latency, not issue rate, is what matters)
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mq[u] = fmax3(mq[u], s[c + 2 * u], s[c + 2 * u + 1]);
+            }
+            const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
             const float m_cand = mx * c2;
             const bool need = m_cand > m_used + kRescaleThreshold;
             const bool warp_rescale = __any_sync(0xffffffffu, need);
@@ -288,7 +294,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
 
             // ---- probabilities (bf16) into TMEM over S, and the row sum
-            float sum = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
@@ -296,12 +302,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int c = 0; c < 32; ++c) {
                     const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * c], c2, -m_use));
                     const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * c + 1], c2, -m_use));
-                    sum += p0 + p1;
+                    ps[c & 3] += p0 + p1;
                     pk[c] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(tS + half * 32, pk);
             }
-            l += sum;
+            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             // Lazy correction of O_t, after the scores are dead (fewer live registers)
             // but before P_t is published: PV_t(j) is issued only after the arrive.
             if (warp_rescale && j > 0) {

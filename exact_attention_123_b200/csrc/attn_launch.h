@@ -20,6 +20,7 @@ struct FwdLaunch {
 
 struct BwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;  // K, V: 128-row boxes; Q, dO: 64-row boxes
+    CUtensorMap tm_dqacc;                 // fp32 dQ accumulator, box 32 columns x 64 rows
     Geom g;
     SyncCtl ctl;
     const void *o, *dout;
