@@ -20,6 +20,8 @@
 //        dP^T = V_j dO_i^T     (tcgen05, M=128, N=64)               -> TMEM
 //        P^T  = 2^(S^T scale log2e - lse2), dS^T = P^T o (dP^T - D) by 8 warps,
 //               written as bf16 into 128-byte-swizzled shared-memory tiles
+//        (Q_i, dO_i and their row terms sit in a 3-stage ring so the next tiles'
+//         loads are in flight a full iteration before they are needed)
 //        dV  += P^T  dO_i      (M=128, N=d, K=64)                   -> TMEM
 //        dK  += dS^T Q_i       (M=128, N=d, K=64)                   -> TMEM
 //        dQ_i = dS K_j         (M=64,  N=d, K=128)                  -> TMEM, then
@@ -123,7 +125,7 @@ struct BwdCfg {
     static constexpr int kQBox = 64 * 128;        // one 64-column box of a 64-row tile
     static constexpr int kBoxes = D / 64;
     static constexpr int kPSBytes = 128 * 128;    // P^T or dS^T: 128 keys x 64 queries bf16
-    static constexpr int kStages = 2;             // Q/dO/vector stages
+    static constexpr int kStages = 3;             // Q/dO/vector stages (load latency stays hidden)
     static constexpr int kThreads = 448;
     static constexpr int kTmemCols = 512;
     static constexpr int kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 128 + D, kColDK = 128 + 2 * D;
@@ -132,28 +134,33 @@ struct BwdCfg {
     static constexpr int kOffV = kKVBytes;
     static constexpr int kOffQ = 2 * kKVBytes;                         // + st * kQBytes
     static constexpr int kOffDO = kOffQ + kStages * kQBytes;           // + st * kQBytes
-    static constexpr int kOffP = kOffDO + kStages * kQBytes;           // + b * kPSBytes
-    static constexpr int kOffDS = kOffP + 2 * kPSBytes;                // + b * kPSBytes
-    static constexpr int kOffVec = kOffDS + 2 * kPSBytes;              // + st * 512: lse2[64], D[64]
-    static constexpr int kOffDQ = kOffVec + kStages * 512;             // fp32 dQ stage: d/32 boxes of 64x32
+    static constexpr int kOffP = kOffDO + kStages * kQBytes;           // P^T tile (single buffer)
+    static constexpr int kOffDS = kOffP + kPSBytes;                    // dS^T tile (single buffer)
+    static constexpr int kOffDQ = kOffDS + kPSBytes;                   // fp32 dQ stage: d/32 boxes of 64x32
     static constexpr int kDQBox = 64 * 128;
-    static constexpr int kOffBar = kOffDQ + (D / 32) * kDQBox;
+    static constexpr int kOffVec = kOffDQ + (D / 32) * kDQBox;         // + st * 512: lse2[64], D[64]
+    static constexpr int kOffBar = kOffVec + kStages * 512;
+    // every swizzled tile must start on a 1024-byte boundary
+    static_assert(kOffQ % 1024 == 0 && kOffDO % 1024 == 0 && kOffP % 1024 == 0 && kOffDS % 1024 == 0 &&
+                      kOffDQ % 1024 == 0 && kQBytes % 1024 == 0,
+                  "swizzled shared-memory tiles must be 1024-byte aligned");
     // barriers
     static constexpr int kBarKV = 0;
-    static constexpr int kBarQFull = 1;    // + st
-    static constexpr int kBarQEmpty = 3;   // + st
-    static constexpr int kBarSdpFull = 5;
-    static constexpr int kBarSdpFree = 6;
-    static constexpr int kBarPsFull = 7;   // + b
-    static constexpr int kBarPsEmpty = 9;  // + b
-    static constexpr int kBarDqFull = 11;
-    static constexpr int kBarDqEmpty = 12;
-    static constexpr int kBarKdv = 13;
-    static constexpr int kBarDone = 14;
-    static constexpr int kBarStageFull = 15;  // dQ stage written (128 drain threads)
-    static constexpr int kBarStageFree = 16;  // dQ stage read by the bulk reduce (leader)
-    static constexpr int kNumBars = 17;
+    static constexpr int kBarQFull = 1;                 // + st
+    static constexpr int kBarQEmpty = 1 + kStages;      // + st
+    static constexpr int kBarSdpFull = 1 + 2 * kStages;
+    static constexpr int kBarSdpFree = 2 + 2 * kStages;
+    static constexpr int kBarPsFull = 3 + 2 * kStages;  // P^T and dS^T written (256 threads)
+    static constexpr int kBarPsEmpty = 4 + 2 * kStages; // dV, dK, dQ finished reading them
+    static constexpr int kBarDqFull = 5 + 2 * kStages;
+    static constexpr int kBarDqEmpty = 6 + 2 * kStages;
+    static constexpr int kBarKdv = 7 + 2 * kStages;
+    static constexpr int kBarDone = 8 + 2 * kStages;
+    static constexpr int kBarStageFull = 9 + 2 * kStages;   // dQ stage written (128 drain threads)
+    static constexpr int kBarStageFree = 10 + 2 * kStages;  // dQ stage read by the bulk reduce (leader)
+    static constexpr int kNumBars = 11 + 2 * kStages;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
 
 struct BwdParams {
@@ -199,7 +206,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
             uint32_t cnt = 1;
-            if (i == C::kBarSdpFree || i == C::kBarPsFull || i == C::kBarPsFull + 1) cnt = 256;
+            if (i == C::kBarSdpFree || i == C::kBarPsFull) cnt = 256;
             if (i == C::kBarDqEmpty || i == C::kBarStageFull) cnt = 128;
             mbar_init(bar(i), cnt);
         }
@@ -230,9 +237,9 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
         for (int it = 0; it < nq; ++it) {
-            const int st = it & 1;
-            const bool ok = __all_sync(0xffffffffu,
-                                       wait_phase(bar(C::kBarQEmpty + st), ((it >> 1) & 1) ^ 1, p.ctl, abort_flag));
+            const int st = it % C::kStages;
+            const bool ok = __all_sync(
+                0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((it / C::kStages) & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
             const int q0 = (i0 + it) * 64;
             float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 512);
@@ -267,7 +274,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             constexpr uint32_t idKV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
             constexpr uint32_t idQ = idesc_bf16_f32(64, D, 1, 1);     // dQ
             auto issue_sdp = [&](int it) {
-                const int st = it & 1;
+                const int st = it % C::kStages;
                 const uint32_t qs = sbase + C::kOffQ + st * C::kQBytes;
                 const uint32_t ds = sbase + C::kOffDO + st * C::kQBytes;
 #pragma unroll
@@ -293,19 +300,20 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 issue_sdp(0);
             }
             for (int it = 0; ok && it < nq; ++it) {
-                const int st = it & 1, pb = it & 1;
+                const int st = it % C::kStages;
                 if (it + 1 < nq) {
-                    ok = wait_phase(bar(C::kBarQFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, p.ctl, abort_flag);
+                    const int nx = it + 1;
+                    ok = wait_phase(bar(C::kBarQFull + nx % C::kStages), (nx / C::kStages) & 1, p.ctl, abort_flag);
                     if (ok) ok = wait_phase(bar(C::kBarSdpFree), it & 1, p.ctl, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_sdp(it + 1);
                 }
-                ok = wait_phase(bar(C::kBarPsFull + pb), (it >> 1) & 1, p.ctl, abort_flag);
+                ok = wait_phase(bar(C::kBarPsFull), it & 1, p.ctl, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t ps = sbase + C::kOffP + pb * C::kPSBytes;
-                const uint32_t dss = sbase + C::kOffDS + pb * C::kPSBytes;
+                const uint32_t ps = sbase + C::kOffP;
+                const uint32_t dss = sbase + C::kOffDS;
                 const uint32_t qs = sbase + C::kOffQ + st * C::kQBytes;
                 const uint32_t dos = sbase + C::kOffDO + st * C::kQBytes;
                 // dV += P^T dO_i ; dK += dS^T Q_i   (K = 64 queries, 4 steps)
@@ -328,7 +336,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     mma_ss(tmem + C::kColDQ, sw128_desc(dss + kk * 2048, 8192, 1024),
                            sw128_desc(sbase + C::kOffK + kk * 2048, C::kKVBox, 1024), idQ, kk > 0);
                 tc_commit(bar(C::kBarDqFull));
-                tc_commit(bar(C::kBarPsEmpty + pb));
+                tc_commit(bar(C::kBarPsEmpty));
             }
             if (ok) tc_commit(bar(C::kBarKdv));
             tc_commit(bar(C::kBarDone));
@@ -344,7 +352,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(b, start) + key] != 0;
         const float c2 = p.scale_log2;
         for (int it = 0; it < nq; ++it) {
-            const int st = it & 1, pb = it & 1;
+            const int st = it % C::kStages;
             bool ok = wait_phase(bar(C::kBarSdpFull), it & 1, p.ctl, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -355,7 +363,8 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(C::kBarSdpFree));
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarQFull + st), (it >> 1) & 1, p.ctl, abort_flag));
+            ok = __all_sync(0xffffffffu,
+                            wait_phase(bar(C::kBarQFull + st), (it / C::kStages) & 1, p.ctl, abort_flag));
             if (!ok) break;
             const float *vec = reinterpret_cast<const float *>(sptr + C::kOffVec + st * 512);
             const int qb = (i0 + it) * 64 + hf * 32;  // first query column of this warp
@@ -378,11 +387,11 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 pp[c >> 1] = pack_bf16x2(pr[0], pr[1]);
                 dsp[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
             }
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarPsEmpty + pb), ((it >> 1) & 1) ^ 1, p.ctl, abort_flag));
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarPsEmpty), (it & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
             // 128-byte swizzled K-major rows: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
-            const uint32_t prow = sbase + C::kOffP + pb * C::kPSBytes + kr * 128;
-            const uint32_t drow = sbase + C::kOffDS + pb * C::kPSBytes + kr * 128;
+            const uint32_t prow = sbase + C::kOffP + kr * 128;
+            const uint32_t drow = sbase + C::kOffDS + kr * 128;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const uint32_t chunk = static_cast<uint32_t>((hf * 4 + u) ^ (kr & 7)) << 4;
@@ -390,7 +399,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 st_shared_v4(drow + chunk, dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2], dsp[4 * u + 3]);
             }
             fence_proxy_async_smem();
-            mbar_arrive(bar(C::kBarPsFull + pb));
+            mbar_arrive(bar(C::kBarPsFull));
         }
     } else {
         // ------------------------------------------------------------ dQ drain + dK/dV epilogue
@@ -481,8 +490,8 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp == 12 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
         drain_phase(bar(C::kBarKV), 0, p.ctl, abort_flag);
-        for (int it = max(0, n_issued - 2); it < n_issued; ++it)
-            drain_phase(bar(C::kBarQFull + (it & 1)), (it >> 1) & 1, p.ctl, abort_flag);
+        for (int it = max(0, n_issued - C::kStages); it < n_issued; ++it)
+            drain_phase(bar(C::kBarQFull + it % C::kStages), (it / C::kStages) & 1, p.ctl, abort_flag);
     }
     if (warp == 13) {
         tc_fence_after();

@@ -62,6 +62,8 @@ struct FwdCfg {
     static constexpr int kNumBars = 8 + 2 * kStages;
     static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
     static constexpr int kSmemBytes = 1024 + kSmemTiles + kNumBars * 8 + 16;
+    static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
 
 struct FwdParams {
