@@ -195,7 +195,7 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
 def attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, *, workspace, scale: Optional[float] = None,
                    causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
                    stream=None):
-    """Launch one backward phase (0 preprocess, 1 main, 2 dQ conversion)."""
+    """Launch one backward phase (0 preprocess, 1 dK/dV, 2 dQ)."""
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)

@@ -149,10 +149,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     return attn::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-size_t bwd_ws_bytes(long long rows_x_heads, int d) {
-    // dQ fp32 accumulator, then D and lse2 (fp32 each), each region 256-byte aligned
+size_t bwd_ws_bytes(long long rows_x_heads, int /*d*/) {
+    // D and lse2 (fp32 each, one per query row and head), each region 256-byte aligned
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    return up(static_cast<size_t>(rows_x_heads) * d * 4) + 2 * up(static_cast<size_t>(rows_x_heads) * 4);
+    return 2 * up(static_cast<size_t>(rows_x_heads) * 4);
 }
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
@@ -172,9 +172,8 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     if ((rc = device_state(&ds))) return rc;
     if (s.cu && s.total == 0) return ATTN_OK;
     attn::BwdLaunch a{};
-    // the backward sweeps 64-row query tiles against 128-row key tiles
-    if ((rc = map_for(&a.tm_q, q, s, 64)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
-        (rc = map_for(&a.tm_do, dout, s, 64)))
+    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
+        (rc = map_for(&a.tm_do, dout, s)))
         return rc;
     a.g = geom_of(s, key_keep);
     a.ctl = ctl_of(ds);
@@ -186,11 +185,8 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     a.dv = dv;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     char *w = static_cast<char *>(workspace);
-    a.dq_acc = reinterpret_cast<float *>(w);
-    // the accumulator has the layout of q (row pitch d), in fp32
-    if ((rc = map_for(&a.tm_dqacc, a.dq_acc, s, 64, true))) return rc;
-    a.dvec = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4));
-    a.lse2 = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * s.d * 4) + up(static_cast<size_t>(rows) * 4));
+    a.dvec = reinterpret_cast<float *>(w);
+    a.lse2 = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * 4));
     a.rows_total = rows;
     a.scale = scale;
     a.causal = is_causal ? 1 : 0;

@@ -9,37 +9,29 @@
 //   dQ = scale dS K,   dK = scale dS^T Q.
 // (D_i equals sum_k P_ik dP_ik because O_i = sum_k P_ik V_k.)
 //
-// Three launches on one stream:
-//   1. attn_bwd_pre_kernel   D_i, lse2_i = lse_i log2(e) (+inf for rows that saw no
-//                            key, so their recomputed P is exactly 0), and a zeroed
-//                            fp32 dQ accumulator.  HBM-bound, vectorised.
-//   2. attn_bwd_main_kernel  one CTA per 128-key tile of one (sequence, head); it
-//                            keeps K_j, V_j in shared memory and sweeps the 64-row
-//                            query tiles i (only i >= the diagonal when causal):
-//        S^T  = K_j Q_i^T      (tcgen05, M=128 keys, N=64 queries)  -> TMEM
-//        dP^T = V_j dO_i^T     (tcgen05, M=128, N=64)               -> TMEM
-//        P^T  = 2^(S^T scale log2e - lse2), dS^T = P^T o (dP^T - D) by 8 warps,
-//               written as bf16 into 128-byte-swizzled shared-memory tiles
-//        (Q_i, dO_i and their row terms sit in a 3-stage ring so the next tiles'
-//         loads are in flight a full iteration before they are needed)
-//        dV  += P^T  dO_i      (M=128, N=d, K=64)                   -> TMEM
-//        dK  += dS^T Q_i       (M=128, N=d, K=64)                   -> TMEM
-//        dQ_i = dS K_j         (M=64,  N=d, K=128)                  -> TMEM, then
-//               staged in shared memory by 4 warps and added into the fp32
-//               accumulator with bulk tensor reduce-adds (TMA)
-//      and finally writes dV and scale*dK in bf16.
-//   3. attn_bwd_dq_kernel    dQ = bf16(scale * accumulator).  HBM-bound.
-//
-// Tensor memory of the main kernel (columns): S^T [0,64), dP^T [64,128),
-// dQ [128,128+d), dV [128+d,128+2d), dK [128+2d,128+3d): no region is shared, so
-// the next tile's S^T / dP^T products are issued as soon as the softmax warps have
-// copied the current ones into registers, and overlap its softmax work.
-//
-// Warp roles (448 threads): warps 0-7 probabilities/dS (warp w: key rows
-// 32*(w%4).., query columns 32*(w/4)..), warps 8-11 dQ drain (thread 256 issues
-// the bulk reductions) and the dK/dV
-// epilogue, warp 12 loader (TMA for K, V, Q, dO; plain loads for lse2/D),
-// warp 13 TMEM allocator and MMA issuer.
+// Three launches on one stream, with no atomics (the result is deterministic):
+//   1. attn_bwd_pre_kernel   D_i and lse2_i = lse_i log2(e) (+inf for rows that saw
+//                            no key, so their recomputed P is exactly 0).
+//   2. attn_bwd_sm100_kernel, mode 0 (dK/dV): one CTA per 128-key tile sweeps the
+//      128-row query tiles
+//                            (from the diagonal when causal):
+//        S^T  = K_j Q_i^T   (SS, M=128 keys, N=128 queries)   -> TMEM
+//        dP^T = V_j dO_i^T  (SS)                              -> TMEM
+//        P^T  = 2^(S^T scale log2e - lse2)  written back over S^T as bf16,
+//        dS^T = P^T o (dP^T - D)            written back over dP^T as bf16
+//               (8 warps; each keeps its P in fp32 registers for dS)
+//        dV  += P^T dO_i    (TS: A = P^T from TMEM, M=128, N=d, K=128)
+//        dK  += dS^T Q_i    (TS: A = dS^T from TMEM)
+//      then writes dV and scale*dK.
+//   3. attn_bwd_sm100_kernel, mode 1 (dQ): one CTA per 128-row query tile sweeps
+//      the key tiles:
+//        S  = Q_i K_j^T, dP = dO_i V_j^T (SS, M=128 queries, N=128 keys) -> TMEM,
+//        S double-buffered so the next tile's product overlaps this tile's math;
+//        dS = P o (dP - D) written back over S as bf16 (8 warps);
+//        dQ += dS K_j      (TS: A = dS from TMEM, M=128, N=d, K=128)
+//      then writes scale*dQ.
+// Every product is a full 128 x 128 (x d) tensor-core tile; the extra S and dP
+// products of the dQ pass cost less than the reductions they replace.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -59,9 +51,8 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *__restrict__ o,
                                                           const __nv_bfloat16 *__restrict__ dout,
                                                           const float *__restrict__ lse, float *__restrict__ dvec,
-                                                          float *__restrict__ lse2, float *__restrict__ dq_acc,
-                                                          long long rows, const int32_t *cu_seqlens, int nseq,
-                                                          int H) {
+                                                          float *__restrict__ lse2, long long rows,
+                                                          const int32_t *cu_seqlens, int nseq, int H) {
     constexpr int TPR = D / 8;  // threads per row
     long long limit = rows;
     if (cu_seqlens) limit = min(rows, static_cast<long long>(cu_seqlens[nseq]) * H);
@@ -73,18 +64,14 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *
     if (active) {
         const uint4 a = *reinterpret_cast<const uint4 *>(o + row * D + part * 8);
         const uint4 g = *reinterpret_cast<const uint4 *>(dout + row * D + part * 8);
-        const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
-        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&g);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 x = __bfloat1622float2(a2[e]);
-            const float2 y = __bfloat1622float2(g2[e]);
+            const float2 x = unpack_bf16x2(aw[e]);
+            const float2 y = unpack_bf16x2(gw[e]);
             acc = fmaf(x.x, y.x, acc);
             acc = fmaf(x.y, y.y, acc);
         }
-        float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D + part * 8);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -95,93 +82,53 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *
     }
 }
 
-// ============================================================================ dQ finish
-template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float *__restrict__ dq_acc,
-                                                         __nv_bfloat16 *__restrict__ dq, long long rows, float scale,
-                                                         const int32_t *cu_seqlens, int nseq, int H) {
-    long long limit = rows;
-    if (cu_seqlens) limit = min(rows, static_cast<long long>(cu_seqlens[nseq]) * H);
-    const long long n8 = limit * D / 8;
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const float4 a = reinterpret_cast<const float4 *>(dq_acc)[2 * i];
-        const float4 b = reinterpret_cast<const float4 *>(dq_acc)[2 * i + 1];
-        uint4 r;
-        r.x = pack_bf16x2(a.x * scale, a.y * scale);
-        r.y = pack_bf16x2(a.z * scale, a.w * scale);
-        r.z = pack_bf16x2(b.x * scale, b.y * scale);
-        r.w = pack_bf16x2(b.z * scale, b.w * scale);
-        reinterpret_cast<uint4 *>(dq)[i] = r;
-    }
-}
-
-// ============================================================================ main kernel
-template <int D>
-struct BwdCfg {
-    static constexpr int kKVBytes = 128 * D * 2;  // K_j or V_j (128 rows)
-    static constexpr int kQBytes = 64 * D * 2;    // Q_i or dO_i (64 rows)
-    static constexpr int kKVBox = 128 * 128;      // one 64-column box of a 128-row tile
-    static constexpr int kQBox = 64 * 128;        // one 64-column box of a 64-row tile
-    static constexpr int kBoxes = D / 64;
-    static constexpr int kPSBytes = 128 * 128;    // P^T or dS^T: 128 keys x 64 queries bf16
-    static constexpr int kStages = 3;             // Q/dO/vector stages (load latency stays hidden)
-    static constexpr int kThreads = 448;
-    static constexpr int kTmemCols = 512;
-    static constexpr int kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 128 + D, kColDK = 128 + 2 * D;
-    // shared-memory offsets (from the 1024-aligned base)
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = kKVBytes;
-    static constexpr int kOffQ = 2 * kKVBytes;                         // + st * kQBytes
-    static constexpr int kOffDO = kOffQ + kStages * kQBytes;           // + st * kQBytes
-    static constexpr int kOffP = kOffDO + kStages * kQBytes;           // P^T tile (single buffer)
-    static constexpr int kOffDS = kOffP + kPSBytes;                    // dS^T tile (single buffer)
-    static constexpr int kOffDQ = kOffDS + kPSBytes;                   // fp32 dQ stage: d/32 boxes of 64x32
-    static constexpr int kDQBox = 64 * 128;
-    static constexpr int kOffVec = kOffDQ + (D / 32) * kDQBox;         // + st * 512: lse2[64], D[64]
-    static constexpr int kOffBar = kOffVec + kStages * 512;
-    // every swizzled tile must start on a 1024-byte boundary
-    static_assert(kOffQ % 1024 == 0 && kOffDO % 1024 == 0 && kOffP % 1024 == 0 && kOffDS % 1024 == 0 &&
-                      kOffDQ % 1024 == 0 && kQBytes % 1024 == 0,
-                  "swizzled shared-memory tiles must be 1024-byte aligned");
-    // barriers
-    static constexpr int kBarKV = 0;
-    static constexpr int kBarQFull = 1;                 // + st
-    static constexpr int kBarQEmpty = 1 + kStages;      // + st
-    static constexpr int kBarSdpFull = 1 + 2 * kStages;
-    static constexpr int kBarSdpFree = 2 + 2 * kStages;
-    static constexpr int kBarPsFull = 3 + 2 * kStages;  // P^T and dS^T written (256 threads)
-    static constexpr int kBarPsEmpty = 4 + 2 * kStages; // dV, dK, dQ finished reading them
-    static constexpr int kBarDqFull = 5 + 2 * kStages;
-    static constexpr int kBarDqEmpty = 6 + 2 * kStages;
-    static constexpr int kBarKdv = 7 + 2 * kStages;
-    static constexpr int kBarDone = 8 + 2 * kStages;
-    static constexpr int kBarStageFull = 9 + 2 * kStages;   // dQ stage written (128 drain threads)
-    static constexpr int kBarStageFree = 10 + 2 * kStages;  // dQ stage read by the bulk reduce (leader)
-    static constexpr int kNumBars = 11 + 2 * kStages;
-    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
-    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
-};
-
 struct BwdParams {
     Geom g;
     SyncCtl ctl;
-    __nv_bfloat16 *dk, *dv;
-    float *dq_acc;
+    __nv_bfloat16 *dq, *dk, *dv;
     const float *dvec, *lse2;
     float scale;
     float scale_log2;
     int causal;
-    int n_kv;  // 128-key tiles per slice (grid z)
+    int n_tiles;  // 128-row tiles per slice (grid z)
+};
+
+// Offset of K-step kk (16 columns) inside a 128-row, 128-byte-swizzled K-major tile.
+__device__ __forceinline__ uint32_t kstep_off(int kk) { return (kk >> 2) * 16384 + (kk & 3) * 32; }
+
+// ============================================================================ dK / dV
+template <int D>
+struct DkdvCfg {
+    static constexpr int kTile = 128 * D * 2;  // any 128-row bf16 tile (K, V, Q, dO)
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kStages = 2;
+    static constexpr int kThreads = 320;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static constexpr int kOffK = 0, kOffV = kTile;
+    static constexpr int kOffQ = 2 * kTile;                  // + st * kTile
+    static constexpr int kOffDO = kOffQ + kStages * kTile;   // + st * kTile
+    static constexpr int kOffVec = kOffDO + kStages * kTile; // + st * 1024: lse2[128], D[128]
+    static constexpr int kOffBar = kOffVec + kStages * 1024;
+    static constexpr int kBarKV = 0;
+    static constexpr int kBarQFull = 1;                  // + st
+    static constexpr int kBarQEmpty = 1 + kStages;       // + st
+    static constexpr int kBarSFull = 1 + 2 * kStages;
+    static constexpr int kBarDPFull = 2 + 2 * kStages;
+    static constexpr int kBarPFull = 3 + 2 * kStages;    // P^T written (256 threads)
+    static constexpr int kBarDSFull = 4 + 2 * kStages;   // dS^T written (256 threads)
+    static constexpr int kBarKdv = 5 + 2 * kStages;
+    static constexpr int kBarDone = 6 + 2 * kStages;
+    static constexpr int kNumBars = 7 + 2 * kStages;
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
+    static_assert(kTile % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
 
 template <int D>
-__global__ void __launch_bounds__(448, 1)
-attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                     const __grid_constant__ CUtensorMap tm_dqacc, const __grid_constant__ BwdParams p) {
-    using C = BwdCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
+__device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                          const CUtensorMap &tm_do, const BwdParams &p, uint8_t *smem_raw, int j) {
+    using C = DkdvCfg<D>;
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
     uint8_t *sptr = smem_raw + (sbase - raw_u32);
@@ -190,26 +137,22 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, b = blockIdx.y, j = blockIdx.z;  // small j (most query tiles) first
+    const int h = blockIdx.x, b = blockIdx.y;
     int start, len;
     p.g.slice(b, start, len);
     const int kv0 = j * 128;
     if (kv0 >= len) return;  // uniform, before any barrier or allocation
-    const int nq_all = (len + 63) / 64;
-    const int i0 = p.causal ? (kv0 / 64) : 0;
+    const int nq_all = (len + 127) / 128;
+    const int i0 = p.causal ? j : 0;
     const int nq = nq_all - i0;  // >= 1
 
-    if (warp == 13) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::kNumBars; ++i) {
-            uint32_t cnt = 1;
-            if (i == C::kBarSdpFree || i == C::kBarPsFull) cnt = 256;
-            if (i == C::kBarDqEmpty || i == C::kBarStageFull) cnt = 128;
-            mbar_init(bar(i), cnt);
-        }
+        for (int i = 0; i < C::kNumBars; ++i)
+            mbar_init(bar(i), (i == C::kBarPFull || i == C::kBarDSFull) ? 256u : 1u);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -221,7 +164,7 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const long long lrs = p.g.row_stride(1);
     int n_issued = 0;  // loader: query-tile loads 0 .. n_issued-1 were started
 
-    if (warp == 12) {
+    if (warp == 8) {
         // ------------------------------------------------------------ loader
         const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
         if (lane == 0) {
@@ -229,11 +172,11 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kKVBytes);
+            mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTile);
 #pragma unroll
             for (int x = 0; x < C::kBoxes; ++x) {
-                tma_load_3d(sbase + C::kOffK + x * C::kKVBox, &tm_k, bar(C::kBarKV), x * 64, row0 + kv0, slab);
-                tma_load_3d(sbase + C::kOffV + x * C::kKVBox, &tm_v, bar(C::kBarKV), x * 64, row0 + kv0, slab);
+                tma_load_3d(sbase + C::kOffK + x * 16384, &tm_k, bar(C::kBarKV), x * 64, row0 + kv0, slab);
+                tma_load_3d(sbase + C::kOffV + x * 16384, &tm_v, bar(C::kBarKV), x * 64, row0 + kv0, slab);
             }
         }
         for (int it = 0; it < nq; ++it) {
@@ -241,10 +184,10 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const bool ok = __all_sync(
                 0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((it / C::kStages) & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
-            const int q0 = (i0 + it) * 64;
-            float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 512);
+            const int q0 = (i0 + it) * 128;
+            float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 const int q = q0 + u * 32 + lane;
                 float l2 = INFINITY, dd = 0.f;  // rows past the sequence: P = 0
                 if (q < len) {
@@ -252,233 +195,195 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     dd = p.dvec[lrow0 + q * lrs];
                 }
                 vec[u * 32 + lane] = l2;
-                vec[64 + u * 32 + lane] = dd;
+                vec[128 + u * 32 + lane] = dd;
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kQBytes);
+                mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
 #pragma unroll
                 for (int x = 0; x < C::kBoxes; ++x) {
-                    tma_load_3d(sbase + C::kOffQ + st * C::kQBytes + x * C::kQBox, &tm_q, bar(C::kBarQFull + st),
-                                x * 64, row0 + q0, slab);
-                    tma_load_3d(sbase + C::kOffDO + st * C::kQBytes + x * C::kQBox, &tm_do, bar(C::kBarQFull + st),
+                    tma_load_3d(sbase + C::kOffQ + st * C::kTile + x * 16384, &tm_q, bar(C::kBarQFull + st), x * 64,
+                                row0 + q0, slab);
+                    tma_load_3d(sbase + C::kOffDO + st * C::kTile + x * 16384, &tm_do, bar(C::kBarQFull + st),
                                 x * 64, row0 + q0, slab);
                 }
             }
             n_issued = it + 1;
         }
-    } else if (warp == 13) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idSP = idesc_bf16_f32(128, 64, 0, 0);  // S^T, dP^T
+            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
             constexpr uint32_t idKV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
-            constexpr uint32_t idQ = idesc_bf16_f32(64, D, 1, 1);     // dQ
-            auto issue_sdp = [&](int it) {
-                const int st = it % C::kStages;
-                const uint32_t qs = sbase + C::kOffQ + st * C::kQBytes;
-                const uint32_t ds = sbase + C::kOffDO + st * C::kQBytes;
+            // P^T / dS^T sit in TMEM with queries 0-63 at columns 0-31 and queries
+            // 64-127 at columns 64-95 of the S^T / dP^T regions (each math warp writes
+            // only inside the columns it read).
+            auto acol = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
+            auto issue_s = [&](int it) {
+                const uint32_t qs = sbase + C::kOffQ + (it % C::kStages) * C::kTile;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t okv = (kk >> 2) * C::kKVBox + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * C::kQBox + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColS, sw128_desc(sbase + C::kOffK + okv, 16, 1024), sw128_desc(qs + oq, 16, 1024),
-                           idSP, kk > 0);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::kColS, sw128_desc(sbase + C::kOffK + kstep_off(kk), 16, 1024),
+                           sw128_desc(qs + kstep_off(kk), 16, 1024), idS, kk > 0);
+                tc_commit(bar(C::kBarSFull));
+            };
+            auto issue_dp = [&](int it) {
+                const uint32_t ds = sbase + C::kOffDO + (it % C::kStages) * C::kTile;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t okv = (kk >> 2) * C::kKVBox + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * C::kQBox + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffV + okv, 16, 1024),
-                           sw128_desc(ds + oq, 16, 1024), idSP, kk > 0);
-                }
-                tc_commit(bar(C::kBarSdpFull));
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffV + kstep_off(kk), 16, 1024),
+                           sw128_desc(ds + kstep_off(kk), 16, 1024), idS, kk > 0);
+                tc_commit(bar(C::kBarDPFull));
             };
             bool ok = wait_phase(bar(C::kBarKV), 0, p.ctl, abort_flag);
             if (ok) ok = wait_phase(bar(C::kBarQFull + 0), 0, p.ctl, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_sdp(0);
+                issue_s(0);
+                issue_dp(0);
             }
             for (int it = 0; ok && it < nq; ++it) {
                 const int st = it % C::kStages;
-                if (it + 1 < nq) {
-                    const int nx = it + 1;
-                    ok = wait_phase(bar(C::kBarQFull + nx % C::kStages), (nx / C::kStages) & 1, p.ctl, abort_flag);
-                    if (ok) ok = wait_phase(bar(C::kBarSdpFree), it & 1, p.ctl, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_sdp(it + 1);
-                }
-                ok = wait_phase(bar(C::kBarPsFull), it & 1, p.ctl, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t ps = sbase + C::kOffP;
-                const uint32_t dss = sbase + C::kOffDS;
-                const uint32_t qs = sbase + C::kOffQ + st * C::kQBytes;
-                const uint32_t dos = sbase + C::kOffDO + st * C::kQBytes;
-                // dV += P^T dO_i ; dK += dS^T Q_i   (K = 64 queries, 4 steps)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem + C::kColDV, sw128_desc(ps + kk * 32, 16, 1024),
-                           sw128_desc(dos + kk * 2048, C::kQBox, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tmem + C::kColDK, sw128_desc(dss + kk * 32, 16, 1024),
-                           sw128_desc(qs + kk * 2048, C::kQBox, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(C::kBarQEmpty + st));
-                // dQ_i = dS K_j   (M = 64 queries, K = 128 keys, 8 steps); the drain
-                // warps must have emptied the previous dQ tile first.
-                ok = wait_phase(bar(C::kBarDqEmpty), (it & 1) ^ 1, p.ctl, abort_flag);
+                const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
+                const uint32_t dos = sbase + C::kOffDO + st * C::kTile;
+                const bool more = it + 1 < nq;
+                // dV += P^T dO_i   (K = 128 queries: 8 steps)
+                ok = wait_phase(bar(C::kBarPFull), it & 1, p.ctl, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::kColDQ, sw128_desc(dss + kk * 2048, 8192, 1024),
-                           sw128_desc(sbase + C::kOffK + kk * 2048, C::kKVBox, 1024), idQ, kk > 0);
-                tc_commit(bar(C::kBarDqFull));
-                tc_commit(bar(C::kBarPsEmpty));
+                    mma_ts(tmem + C::kColDV, tmem + C::kColS + acol(kk), sw128_desc(dos + kk * 2048, 16384, 1024),
+                           idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                // S^T_{i+1} may overwrite P^T_i now: the math warps keep P in registers
+                // and dV_i, issued first, completes first.
+                if (more) {
+                    ok = wait_phase(bar(C::kBarQFull + (it + 1) % C::kStages), ((it + 1) / C::kStages) & 1, p.ctl,
+                                    abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(it + 1);
+                }
+                // dK += dS^T Q_i
+                ok = wait_phase(bar(C::kBarDSFull), it & 1, p.ctl, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::kColDK, tmem + C::kColDP + acol(kk), sw128_desc(qs + kk * 2048, 16384, 1024),
+                           idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(C::kBarQEmpty + st));
+                if (more) issue_dp(it + 1);
             }
             if (ok) tc_commit(bar(C::kBarKdv));
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ P^T and dS^T
+    } else {
+        // ------------------------------------------------------------ P^T and dS^T (warps 0-7)
+        // warp w: key rows 32*(w%4).., query columns 64*(w/4) .. +63 of each query tile.
         const int q4 = warp & 3, hf = warp >> 2;
         const int kr = q4 * 32 + lane;  // key row within the tile
         const int key = kv0 + kr;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::kColS + hf * 64;
+        const uint32_t tDP = tmem + lane_off + C::kColDP + hf * 64;
         bool kvalid = key < len;
         if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(b, start) + key] != 0;
         const float c2 = p.scale_log2;
-        for (int it = 0; it < nq; ++it) {
-            const int st = it % C::kStages;
-            bool ok = wait_phase(bar(C::kBarSdpFull), it & 1, p.ctl, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t sr[32], dpr[32];
-            tmem_ld32(tmem + lane_off + C::kColS + hf * 32, sr);
-            tmem_ld32(tmem + lane_off + C::kColDP + hf * 32, dpr);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarSdpFree));
-            ok = __all_sync(0xffffffffu,
-                            wait_phase(bar(C::kBarQFull + st), (it / C::kStages) & 1, p.ctl, abort_flag));
-            if (!ok) break;
-            const float *vec = reinterpret_cast<const float *>(sptr + C::kOffVec + st * 512);
-            const int qb = (i0 + it) * 64 + hf * 32;  // first query column of this warp
-            int lim = p.causal ? key - qb : 0;         // columns c < lim have query < key
-            if (!kvalid) lim = 32;
-            uint32_t pp[16], dsp[16];
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                float pr[2], dsv[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int cc = c + e;
-                    const float l2 = vec[hf * 32 + cc];
-                    const float dd = vec[64 + hf * 32 + cc];
-                    float pv = ex2_approx(fmaf(__uint_as_float(sr[cc]), c2, -l2));
-                    if (cc < lim) pv = 0.f;
-                    pr[e] = pv;
-                    dsv[e] = pv * (__uint_as_float(dpr[cc]) - dd);
-                }
-                pp[c >> 1] = pack_bf16x2(pr[0], pr[1]);
-                dsp[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-            }
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarPsEmpty), (it & 1) ^ 1, p.ctl, abort_flag));
-            if (!ok) break;
-            // 128-byte swizzled K-major rows: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
-            const uint32_t prow = sbase + C::kOffP + kr * 128;
-            const uint32_t drow = sbase + C::kOffDS + kr * 128;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t chunk = static_cast<uint32_t>((hf * 4 + u) ^ (kr & 7)) << 4;
-                st_shared_v4(prow + chunk, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-                st_shared_v4(drow + chunk, dsp[4 * u], dsp[4 * u + 1], dsp[4 * u + 2], dsp[4 * u + 3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(C::kBarPsFull));
-        }
-    } else {
-        // ------------------------------------------------------------ dQ drain + dK/dV epilogue
-        // Each dQ_i tile (fp32, M = 64) goes TMEM -> registers -> a 128-byte swizzled
-        // shared-memory stage -> one bulk tensor reduce-add per 32-column box into the
-        // fp32 accumulator (the L2 does the additions line by line).  Query rows past
-        // the sequence hold exact zeros (their P is 0), so adding them is harmless.
-        const int q4 = warp & 3;
-        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-        const bool leader = threadIdx.x == 256;
-        const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
-        const uint32_t stage = sbase + C::kOffDQ;
-        const int r = q4 * 16 + lane;  // M = 64 accumulator: row r sits in TMEM lane (r % 16) + 32 * (r / 16)
         bool ok = true;
         for (int it = 0; it < nq; ++it) {
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDqFull), it & 1, p.ctl, abort_flag));
-            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarStageFree), (it & 1) ^ 1, p.ctl, abort_flag));
+            const int st = it % C::kStages;
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull), it & 1, p.ctl, abort_flag));
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                wait_phase(bar(C::kBarQFull + st), (it / C::kStages) & 1, p.ctl, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float4 *vec = reinterpret_cast<const float4 *>(sptr + C::kOffVec + st * 1024) + hf * 16;
+            uint32_t sr[2][32];
+            tmem_ld32(tS, sr[0]);
+            tmem_ld32(tS + 32, sr[1]);
+            tmem_wait_ld();
+            // P^T = 2^(S^T c - lse2), 0 where the query precedes the key (causal),
+            // for keys outside the sequence or padded, and for rows past the end.
+            const int qb = (i0 + it) * 128 + hf * 64;  // first query column of this warp
+            int lim = p.causal ? key - qb : 0;          // columns c < lim are masked
+            if (!kvalid) lim = 64;
+            float pf[64];
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 l2 = vec[c4];
+                const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = c4 * 4 + e;
+                    pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2v[e]));
+                }
+            }
+            if (lim > 0) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c < lim) pf[c] = 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pf[x * 32 + 2 * c], pf[x * 32 + 2 * c + 1]);
+                tmem_st16(tS + x * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarPFull));
+            // dS^T = P^T o (dP^T - D), P taken from registers (fp32)
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), it & 1, p.ctl, abort_flag));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int x = 0; x < D / 32; ++x) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_off + C::kColDQ + x * 32, v);
+            for (int x = 0; x < 2; ++x) {
+                uint32_t dr[32];
+                tmem_ld32(tDP + x * 32, dr);
                 tmem_wait_ld();
-                if (x == D / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(bar(C::kBarDqEmpty));
-                }
-                if (lane < 16) {
-                    const uint32_t rowa = stage + x * C::kDQBox + r * 128;
+                uint32_t pk[16];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        st_shared_v4(rowa + ((static_cast<uint32_t>(k ^ (r & 7))) << 4), v[4 * k], v[4 * k + 1],
-                                     v[4 * k + 2], v[4 * k + 3]);
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 dd = vec[32 + x * 8 + c4];
+                    const int c = x * 32 + c4 * 4;
+                    pk[2 * c4] = pack_bf16x2(pf[c] * (__uint_as_float(dr[c4 * 4]) - dd.x),
+                                             pf[c + 1] * (__uint_as_float(dr[c4 * 4 + 1]) - dd.y));
+                    pk[2 * c4 + 1] = pack_bf16x2(pf[c + 2] * (__uint_as_float(dr[c4 * 4 + 2]) - dd.z),
+                                                 pf[c + 3] * (__uint_as_float(dr[c4 * 4 + 3]) - dd.w));
                 }
+                tmem_st16(tDP + x * 16, pk);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(C::kBarStageFull));
-            if (leader) {
-                ok = wait_phase(bar(C::kBarStageFull), it & 1, p.ctl, abort_flag);
-                if (ok) {
-                    const int q0 = (i0 + it) * 64;
-#pragma unroll
-                    for (int x = 0; x < D / 32; ++x) tma_reduce_add_3d(&tm_dqacc, stage + x * C::kDQBox, x * 32, row0 + q0, slab);
-                    bulk_commit();
-                    bulk_wait_read0();
-                }
-                mbar_arrive(bar(C::kBarStageFree));
-            }
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarDSFull));
         }
-        if (leader) bulk_wait0();  // the accumulator updates are complete before the CTA exits
+        // ---- epilogue: warps 0-3 write dV, warps 4-7 write scale * dK
         if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKdv), 0, p.ctl, abort_flag));
         if (ok) {
             tc_fence_after();
-            const int key = kv0 + q4 * 32 + lane;
+            const bool is_dv = hf == 0;
             const bool valid = key < len;
             const long long off = p.g.base(b, h, start, D) + static_cast<long long>(key) * p.g.row_stride(D);
+            __nv_bfloat16 *out = (is_dv ? p.dv : p.dk) + off;
+            const float mul = is_dv ? 1.f : p.scale;
+            const uint32_t col = is_dv ? C::kColDV : C::kColDK;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16 *out = (which == 0 ? p.dv : p.dk) + off;
-                const float mul = which == 0 ? 1.f : p.scale;
-                const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + col + c0, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + col + c0, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
-                    if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    }
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
         }
@@ -487,62 +392,359 @@ attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncwarp();
     tc_fence_before();
     __syncthreads();
-    if (warp == 12 && lane == 0 && *abort_flag) {
+    if (warp == 8 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
         drain_phase(bar(C::kBarKV), 0, p.ctl, abort_flag);
         for (int it = max(0, n_issued - C::kStages); it < n_issued; ++it)
             drain_phase(bar(C::kBarQFull + it % C::kStages), (it / C::kStages) & 1, p.ctl, abort_flag);
     }
-    if (warp == 13) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
+// ============================================================================ dQ
+template <int D>
+struct DqCfg {
+    static constexpr int kTile = 128 * D * 2;
+    static constexpr int kBoxes = D / 64;
+    // K_j is read by S_j and by dQ_j (the last product of step j), V_j only by dP_j,
+    // so K gets the deeper ring: the next tiles' loads are in flight a full step ahead.
+    static constexpr int kKStages = (D == 128) ? 3 : 6;
+    static constexpr int kVStages = (D == 128) ? 2 : 4;
+    static constexpr int kThreads = 320;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColS0 = 0, kColS1 = 128, kColDP = 256, kColDQ = 384;
+    static constexpr int kOffQ = 0, kOffDO = kTile;
+    static constexpr int kOffK = 2 * kTile;                     // + s * kTile
+    static constexpr int kOffV = kOffK + kKStages * kTile;      // + s * kTile
+    static constexpr int kOffBar = kOffV + kVStages * kTile;
+    static constexpr int kBarQ = 0;
+    static constexpr int kBarKFull = 1;                          // + slot
+    static constexpr int kBarKEmpty = kBarKFull + kKStages;      // + slot
+    static constexpr int kBarVFull = kBarKEmpty + kKStages;      // + slot
+    static constexpr int kBarVEmpty = kBarVFull + kVStages;      // + slot
+    static constexpr int kBarSFull = kBarVEmpty + kVStages;      // + buffer
+    static constexpr int kBarDPFull = kBarSFull + 2;
+    static constexpr int kBarDPFree = kBarDPFull + 1;            // 256 threads copied dP out
+    static constexpr int kBarDSFull = kBarDPFree + 1;            // 256 threads wrote dS
+    static constexpr int kBarDq = kBarDSFull + 1;
+    static constexpr int kBarDone = kBarDq + 1;
+    static constexpr int kNumBars = kBarDone + 1;
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
+    static_assert(kTile % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
+    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
+    static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
+};
+
+template <int D>
+__device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                        const CUtensorMap &tm_do, const BwdParams &p, uint8_t *smem_raw, int qt) {
+    using C = DqCfg<D>;
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+    uint8_t *sptr = smem_raw + (sbase - raw_u32);
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
+    auto kslot = [&](int jt) -> uint32_t { return sbase + C::kOffK + static_cast<uint32_t>(jt % C::kKStages) * C::kTile; };
+    auto vslot = [&](int jt) -> uint32_t { return sbase + C::kOffV + static_cast<uint32_t>(jt % C::kVStages) * C::kTile; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    int start, len;
+    p.g.slice(b, start, len);
+    const int q0 = qt * 128;
+    if (q0 >= len) return;
+    const int nkv_all = (len + 127) / 128;
+    const int nkv = p.causal ? min(nkv_all, qt + 1) : nkv_all;
+
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kNumBars; ++i)
+            mbar_init(bar(i), (i == C::kBarDPFree || i == C::kBarDSFull) ? 256u : 1u);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    int n_issued = 0;  // loader: K/V tiles 0 .. n_issued-1 were started (K_j before V_j)
+    bool v_issued_last = true;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ loader
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
+            mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTile);
+#pragma unroll
+            for (int x = 0; x < C::kBoxes; ++x) {
+                tma_load_3d(sbase + C::kOffQ + x * 16384, &tm_q, bar(C::kBarQ), x * 64, row0 + q0, slab);
+                tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQ), x * 64, row0 + q0, slab);
+            }
+            for (int jt = 0; jt < nkv; ++jt) {
+                const int ks = jt % C::kKStages, vs = jt % C::kVStages;
+                if (!wait_phase(bar(C::kBarKEmpty + ks), ((jt / C::kKStages) & 1) ^ 1, p.ctl, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(C::kBarKFull + ks), C::kTile);
+#pragma unroll
+                for (int x = 0; x < C::kBoxes; ++x)
+                    tma_load_3d(kslot(jt) + x * 16384, &tm_k, bar(C::kBarKFull + ks), x * 64, row0 + 128 * jt, slab);
+                n_issued = jt + 1;
+                v_issued_last = false;
+                if (!wait_phase(bar(C::kBarVEmpty + vs), ((jt / C::kVStages) & 1) ^ 1, p.ctl, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
+#pragma unroll
+                for (int x = 0; x < C::kBoxes; ++x)
+                    tma_load_3d(vslot(jt) + x * 16384, &tm_v, bar(C::kBarVFull + vs), x * 64, row0 + 128 * jt, slab);
+                v_issued_last = true;
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idQ = idesc_bf16_f32(128, D, 0, 1);
+            auto issue_s = [&](int jt) {
+                const uint32_t ks = kslot(jt);
+                const uint32_t col = (jt & 1) ? C::kColS1 : C::kColS0;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + col, sw128_desc(sbase + C::kOffQ + kstep_off(kk), 16, 1024),
+                           sw128_desc(ks + kstep_off(kk), 16, 1024), idS, kk > 0);
+                tc_commit(bar(C::kBarSFull + (jt & 1)));
+            };
+            auto issue_dp = [&](int jt) {
+                const uint32_t vs = vslot(jt);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffDO + kstep_off(kk), 16, 1024),
+                           sw128_desc(vs + kstep_off(kk), 16, 1024), idS, kk > 0);
+                tc_commit(bar(C::kBarDPFull));
+                tc_commit(bar(C::kBarVEmpty + jt % C::kVStages));  // V_j is free once dP_j is done
+            };
+            auto wait_k = [&](int jt) {
+                return wait_phase(bar(C::kBarKFull + jt % C::kKStages), (jt / C::kKStages) & 1, p.ctl, abort_flag);
+            };
+            auto wait_v = [&](int jt) {
+                return wait_phase(bar(C::kBarVFull + jt % C::kVStages), (jt / C::kVStages) & 1, p.ctl, abort_flag);
+            };
+            bool ok = wait_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+            if (ok) ok = wait_k(0);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+                ok = wait_v(0);
+            }
+            if (ok) {
+                tc_fence_after();
+                issue_dp(0);
+            }
+            for (int jt = 0; ok && jt < nkv; ++jt) {
+                if (jt + 1 < nkv) {
+                    // S_{j+1} into the other buffer (its previous dS was read by dQ_{j-1},
+                    // issued earlier: in-order completion makes the overwrite safe)
+                    ok = wait_k(jt + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(jt + 1);
+                    // dP_{j+1} once the softmax warps have copied dP_j out
+                    ok = wait_phase(bar(C::kBarDPFree), jt & 1, p.ctl, abort_flag);
+                    if (ok) ok = wait_v(jt + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_dp(jt + 1);
+                }
+                // dQ += dS_j K_j  (A = dS from TMEM: keys 0-63 at columns 0-31, keys 64-127 at 64-95)
+                ok = wait_phase(bar(C::kBarDSFull), jt & 1, p.ctl, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t scol = (jt & 1) ? C::kColS1 : C::kColS0;
+                const uint32_t ks = kslot(jt);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t acol = scol + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+                    mma_ts(tmem + C::kColDQ, tmem + acol, sw128_desc(ks + kk * 2048, 16384, 1024), idQ,
+                           (jt > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar(C::kBarKEmpty + jt % C::kKStages));  // K_j is free once dQ_j is done
+            }
+            if (ok) tc_commit(bar(C::kBarDq));
+            tc_commit(bar(C::kBarDone));
+            drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
+        }
+    } else {
+        // ------------------------------------------------------------ P and dS (8 warps)
+        // warp w: query rows 32*(w%4).., keys 64*(w/4) .. +63 of each key tile.
+        const int q4 = warp & 3, hf = warp >> 2;
+        const int qrow = q0 + q4 * 32 + lane;  // query row within the slice
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const long long lidx = p.g.base(b, h, start, 1) + static_cast<long long>(qrow) * p.g.row_stride(1);
+        const float l2 = (qrow < len) ? p.lse2[lidx] : INFINITY;  // rows past the sequence: P = 0
+        const float dd = (qrow < len) ? p.dvec[lidx] : 0.f;
+        const float c2 = p.scale_log2;
+        const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(b, start) : nullptr;
+        bool ok = true;
+        for (int jt = 0; jt < nkv; ++jt) {
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull + (jt & 1)), (jt >> 1) & 1, p.ctl, abort_flag));
+            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), jt & 1, p.ctl, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t scol = (jt & 1) ? C::kColS1 : C::kColS0;
+            uint32_t sr[2][32], dr[2][32];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                tmem_ld32(tmem + lane_off + scol + hf * 64 + x * 32, sr[x]);
+                tmem_ld32(tmem + lane_off + C::kColDP + hf * 64 + x * 32, dr[x]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarDPFree));
+            // masking: keys outside the sequence, above the diagonal, or padded
+            const int kb = jt * 128 + hf * 64;  // first key of this warp's columns
+            int limit = len - kb;
+            if (p.causal) limit = min(limit, qrow - kb + 1);
+            uint32_t kmask[2] = {0xffffffffu, 0xffffffffu};
+            if (keep != nullptr) {
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int c = x * 32 + lane;
+                    kmask[x] = __ballot_sync(0xffffffffu, (c < len - kb) && keep[kb + c] != 0);
+                }
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                float pf[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pf[c] = ex2_approx(fmaf(__uint_as_float(sr[x][c]), c2, -l2));
+                // masks only where this warp's 32 keys need them
+                const int lim_x = limit - 32 * x;  // columns c >= lim_x are masked
+                if (lim_x < 32) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (c >= lim_x) pf[c] = 0.f;
+                }
+                if (keep != nullptr) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (!((kmask[x] >> c) & 1u)) pf[c] = 0.f;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2)
+                    pk[c >> 1] = pack_bf16x2(pf[c] * (__uint_as_float(dr[x][c]) - dd),
+                                             pf[c + 1] * (__uint_as_float(dr[x][c + 1]) - dd));
+                tmem_st16(tmem + lane_off + scol + hf * 64 + x * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarDSFull));
+        }
+        // ---- epilogue: scale * dQ in bf16 (warp w writes columns (w/4)*d/2 ..)
+        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDq), 0, p.ctl, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            const bool valid = qrow < len;
+            __nv_bfloat16 *out = p.dq + p.g.base(b, h, start, D) + static_cast<long long>(qrow) * p.g.row_stride(D);
+#pragma unroll
+            for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + C::kColDQ + c0, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * p.scale, __uint_as_float(r[2 * c + 1]) * p.scale);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8 && lane == 0 && *abort_flag) {
+        // After an abort, every copy the loader started must land before the CTA exits.
+        drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+        for (int jt = max(0, n_issued - C::kKStages); jt < n_issued; ++jt)
+            drain_phase(bar(C::kBarKFull + jt % C::kKStages), (jt / C::kKStages) & 1, p.ctl, abort_flag);
+        const int nv = v_issued_last ? n_issued : n_issued - 1;
+        for (int jt = max(0, nv - C::kVStages); jt < nv; ++jt)
+            drain_phase(bar(C::kBarVFull + jt % C::kVStages), (jt / C::kVStages) & 1, p.ctl, abort_flag);
+    }
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ============================================================================ dK/dV and dQ kernel
+// mode 0: dK/dV CTAs; mode 1: dQ CTAs.  Along grid z the heaviest causal tiles of
+// each kind come first.
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+attn_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ BwdParams p, int mode) {
+    extern __shared__ uint8_t smem_raw[];
+    const int rank = static_cast<int>(blockIdx.z);  // 0 = heaviest tile of its kind
+    if (mode == 0)
+        dkdv_body<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw, rank);  // key tile j: small j has the most query tiles
+    else
+        dq_body<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw, p.n_tiles - 1 - rank);  // query tile: large has the most keys
+}
+
+// ============================================================================ launch
 template <int D>
 static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
-    using C = BwdCfg<D>;
     const int nseq = a.g.B;
     const int *cu = a.g.varlen ? a.g.cu_seqlens : nullptr;
+    BwdParams p{};
+    p.g = a.g;
+    p.ctl = a.ctl;
+    p.dq = static_cast<__nv_bfloat16 *>(a.dq);
+    p.dk = static_cast<__nv_bfloat16 *>(a.dk);
+    p.dv = static_cast<__nv_bfloat16 *>(a.dv);
+    p.dvec = a.dvec;
+    p.lse2 = a.lse2;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * kLog2e;
+    p.causal = a.causal;
+    p.n_tiles = (a.g.N + 127) / 128;
     if (a.phases & 1) {
         const long long threads = a.rows_total * (D / 8);
         const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-        attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(a.o), static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.dvec,
-            a.lse2, a.dq_acc, a.rows_total, cu, nseq, a.g.H);
+        attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(a.o),
+                                                           static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.dvec,
+                                                           a.lse2, a.rows_total, cu, nseq, a.g.H);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    // dK/dV then dQ, as two launches: one grid holding both kinds of CTA measured
+    // slower than the two back to back.
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         max(DkdvCfg<D>::kSmemBytes, DqCfg<D>::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    const dim3 g(a.g.H, a.g.B, p.n_tiles);
     if (a.phases & 2) {
-        BwdParams p{};
-        p.g = a.g;
-        p.ctl = a.ctl;
-        p.dk = static_cast<__nv_bfloat16 *>(a.dk);
-        p.dv = static_cast<__nv_bfloat16 *>(a.dv);
-        p.dq_acc = a.dq_acc;
-        p.dvec = a.dvec;
-        p.lse2 = a.lse2;
-        p.scale = a.scale;
-        p.scale_log2 = a.scale * kLog2e;
-        p.causal = a.causal;
-        p.n_kv = (a.g.N + 127) / 128;
-        cudaError_t e = cudaFuncSetAttribute(attn_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        dim3 grid(a.g.H, a.g.B, p.n_kv);
-        attn_bwd_main_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do,
-                                                                             a.tm_dqacc, p);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        attn_bwd_sm100_kernel<D><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p, 0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.phases & 4) {
-        const long long n8 = a.rows_total * D / 8;
-        long long blocks = (n8 + 255) / 256;
-        if (blocks > 148LL * 64) blocks = 148LL * 64;
-        if (blocks < 1) blocks = 1;
-        attn_bwd_dq_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            a.dq_acc, static_cast<__nv_bfloat16 *>(a.dq), a.rows_total, a.scale, cu, nseq, a.g.H);
-        return cudaGetLastError();
+        attn_bwd_sm100_kernel<D><<<g, 320, DqCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p, 1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -19,20 +19,18 @@ struct FwdLaunch {
 };
 
 struct BwdLaunch {
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;  // K, V: 128-row boxes; Q, dO: 64-row boxes
-    CUtensorMap tm_dqacc;                 // fp32 dQ accumulator, box 32 columns x 64 rows
+    CUtensorMap tm_q, tm_k, tm_v, tm_do;  // same map shape as the forward (128-row boxes)
     Geom g;
     SyncCtl ctl;
     const void *o, *dout;
     const float *lse;
     void *dq, *dk, *dv;
-    float *dq_acc;     // fp32 [rows, H, d] or [B, H, N, d] accumulator (workspace)
     float *dvec;       // fp32 D_i = rowsum(dO o O), lse layout (workspace)
     float *lse2;       // fp32 lse * log2(e), +inf for empty rows, lse layout (workspace)
     long long rows_total;  // token rows (packed) or B*H*N (dense) of the lse layout
     float scale;
     int causal;
-    int phases;        // bit 0: preprocess, bit 1: main kernel, bit 2: dQ conversion
+    int phases;        // bit 0: preprocess, bit 1: dK/dV kernel, bit 2: dQ kernel
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);

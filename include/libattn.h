@@ -112,8 +112,9 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
  *   dq, dk, dv : outputs (bf16, layout of q).
  *   workspace  : caller-owned device memory of at least
  *                attn_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
- *                its contents are scratch (fp32 dQ accumulator and per-row
- *                terms) and need no initialisation.
+ *                its contents are scratch (two fp32 terms per query row and
+ *                head) and need no initialisation.
+ * The result is deterministic: no atomics are used.
  * Returns an attn_status_t code.
  */
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -149,10 +150,12 @@ ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const 
 /*
  * One of the backward's three kernels (attn_bwd / attn_bwd_varlen launch all three
  * in this order); lets a caller time or schedule them separately.
- *   phase 0 : per-row terms D_i = rowsum(dO o O) and lse2 = lse*log2(e), and a
- *             zeroed fp32 dQ accumulator, all in `workspace`
- *   phase 1 : main kernel: dK, dV (written) and dQ (accumulated in `workspace`)
- *   phase 2 : dQ = scale * accumulator, written as bf16
+ *   phase 0 : per-row terms D_i = rowsum(dO o O) and lse2 = lse*log2(e), in
+ *             `workspace`
+ *   phase 1 : dK and dV (one pass per 128-key tile over the query tiles)
+ *   phase 2 : dQ (one pass per 128-row query tile over the key tiles)
+ * Phases 1 and 2 both read only the inputs and phase 0's terms, so after phase 0
+ * they may run in either order (or concurrently on two streams).
  * Phases must run in order on the same workspace and stream.  Other arguments as
  * attn_bwd_varlen; for the dense layout pass cu_seqlens = NULL, num_seqs = B,
  * max_seqlen = N and total_tokens = 0.
