@@ -6,7 +6,8 @@ current stream.  There is no CPU or library fallback: if ``libattn.so`` is
 missing, importing the entry points raises.
 
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
-``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_workspace_bytes``,
+``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
+``attn_bwd_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
 ``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
 """
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
+    L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp]
+    L.attn_bwd_noalloc.restype = i
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
     L.attn_strerror.restype = ctypes.c_char_p
@@ -208,6 +211,27 @@ def attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, *, workspace, sc
                               _ptr(dk), _ptr(dv), nseq, total, N, H, d, float(scale), int(causal), _ptr(cu_seqlens),
                               _ptr(key_keep), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "attn_bwd_phase")
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[float] = None,
+                     causal: bool = True, key_keep=None, stream=None):
+    """Dense-layout backward that uses the library's own scratch array instead of a
+    caller workspace, for callers that cannot allocate device memory (see the C
+    declaration for the size limit and the sharing rules).  Returns (dq, dk, dv)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, H, N, d, float(scale), int(causal), None, _ptr(key_keep),
+                                _stream(stream))
+    _check(rc, "attn_bwd_noalloc")
+    return dq, dk, dv
 
 
 def attn_status(stream=None) -> int:

@@ -166,6 +166,37 @@ ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void 
                             int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
+#define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * attn_bwd without a workspace argument, for callers that cannot allocate device
+ * memory themselves: code running with a fixed memory budget or inside another
+ * framework's allocator that forbids raw device allocations, or code that must
+ * not allocate once it has started (no counterpart in the attention pages: this
+ * is a deployment convenience, not part of the method).
+ *
+ * The backward's scratch (two fp32 terms per query row and head) lives instead in
+ * a fixed array of ATTN_NOALLOC_SCRATCH_BYTES inside the library, one copy per
+ * GPU that loads the library, kept until the process exits.  Nothing is
+ * allocated per call.  Arguments and layouts are those of attn_bwd (with
+ * cu_seqlens != NULL the packed buffers must span B*N token rows).
+ *   - The sizes may need at most ATTN_NOALLOC_SCRATCH_BYTES of scratch, i.e.
+ *     attn_bwd_workspace_bytes(B, H, N, d) <= ATTN_NOALLOC_SCRATCH_BYTES
+ *     (B*H*N <= 1,048,576); larger sizes return ATTN_ERR_WORKSPACE without
+ *     launching anything.
+ *   - The first call on a device looks up that device's copy of the array (with
+ *     the device current); make that first call before any stream capture.
+ *   - Every call shares the array, which keeps the last call's contents.  Nothing
+ *     in it needs to start at zero (each call writes every term it reads), but
+ *     two calls whose kernels overlap on the GPU (different streams, no ordering
+ *     between them) race on it.
+ */
+ATTN_API int attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              int B, int H, int N, int d, float scale, int is_causal,
+                              const int32_t *cu_seqlens, const uint8_t *key_keep, void *stream);
+
 /*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait
