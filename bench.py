@@ -320,8 +320,8 @@ def run_ours(args):
     # the headline value; the recomputed S and dP of the dQ pass are not.)
     dkdv_tf = 2.0 * flops_fwd() / (dkdv_ms * 1e-3) / 1e12
     dq_tf = 1.5 * flops_fwd() / (dq_ms * 1e-3) / 1e12
-    per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf), "attn_bwd_sm100_kernel(dK/dV)": (dkdv_ms, dkdv_tf),
-                  "attn_bwd_sm100_kernel(dQ)": (dq_ms, dq_tf)}
+    per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf), "attn_bwd_dkdv_sm100_kernel": (dkdv_ms, dkdv_tf),
+                  "attn_bwd_dq_sm100_kernel": (dq_ms, dq_tf)}
     dominant = max(per_kernel, key=lambda kname: per_kernel[kname][0])
     dom_tf = per_kernel[dominant][1]
 

@@ -29,6 +29,7 @@ std::atomic<int> g_skip_load{-1};
 struct DeviceState {
     std::once_flag once;
     int supported = 0;  // 1 if sm_100
+    int num_sms = 0;
     int *status = nullptr;
     cudaError_t err = cudaSuccess;
 };
@@ -57,6 +58,7 @@ int device_state(DeviceState **out) {
         s.err = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
         if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         s.supported = (major == 10 && minor == 0);
+        if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (s.err == cudaSuccess && s.supported) s.err = cudaGetSymbolAddress(reinterpret_cast<void **>(&s.status), g_attn_status);
     });
     if (s.err != cudaSuccess) return ATTN_ERR_CUDA;
@@ -191,6 +193,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     a.scale = scale;
     a.causal = is_causal ? 1 : 0;
     a.phases = phases;
+    a.num_sms = ds->num_sms > 0 ? ds->num_sms : 1;
     return attn::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -12,9 +12,8 @@
 // Three launches on one stream, with no atomics (the result is deterministic):
 //   1. attn_bwd_pre_kernel   D_i and lse2_i = lse_i log2(e) (+inf for rows that saw
 //                            no key, so their recomputed P is exactly 0).
-//   2. attn_bwd_sm100_kernel, mode 0 (dK/dV): one CTA per 128-key tile sweeps the
-//      128-row query tiles
-//                            (from the diagonal when causal):
+//   2. attn_bwd_dkdv_sm100_kernel: work unit = one 128-key tile of one (b, h), which
+//      sweeps the 128-row query tiles (from the diagonal when causal):
 //        S^T  = K_j Q_i^T   (SS, M=128 keys, N=128 queries)   -> TMEM
 //        dP^T = V_j dO_i^T  (SS)                              -> TMEM
 //        P^T  = 2^(S^T scale log2e - lse2)  written back over S^T as bf16,
@@ -23,13 +22,17 @@
 //        dV  += P^T dO_i    (TS: A = P^T from TMEM, M=128, N=d, K=128)
 //        dK  += dS^T Q_i    (TS: A = dS^T from TMEM)
 //      then writes dV and scale*dK.
-//   3. attn_bwd_sm100_kernel, mode 1 (dQ): one CTA per 128-row query tile sweeps
-//      the key tiles:
+//   3. attn_bwd_dq_sm100_kernel: work unit = one 128-row query tile of one (b, h),
+//      which sweeps the key tiles:
 //        S  = Q_i K_j^T, dP = dO_i V_j^T (SS, M=128 queries, N=128 keys) -> TMEM,
 //        S double-buffered so the next tile's product overlaps this tile's math;
 //        dS = P o (dP - D) written back over S as bf16 (8 warps);
 //        dQ += dS K_j      (TS: A = dS from TMEM, M=128, N=d, K=128)
 //      then writes scale*dQ.
+// Both main kernels are persistent (one CTA per SM, units dealt heaviest first in a
+// snake order).  Every barrier keeps counting phases across units, so a CTA loads
+// the next unit's tiles and issues its first products while the math warps are
+// still writing the previous unit's result.
 // Every product is a full 128 x 128 (x d) tensor-core tile; the extra S and dP
 // products of the dQ pass cost less than the reductions they replace.
 #include <cuda_bf16.h>
@@ -90,11 +93,19 @@ struct BwdParams {
     float scale;
     float scale_log2;
     int causal;
-    int n_tiles;  // 128-row tiles per slice (grid z)
+    int n_tiles;  // 128-row tiles per slice
 };
 
 // Offset of K-step kk (16 columns) inside a 128-row, 128-byte-swizzled K-major tile.
 __device__ __forceinline__ uint32_t kstep_off(int kk) { return (kk >> 2) * 16384 + (kk & 3) * 32; }
+
+// ============================================================================ persistent schedule
+// Both backward passes run one persistent CTA per SM.  Work units are ranked
+// heaviest first (for causal masking: key tile 0 / the last query tile have the
+// most partner tiles); CTA c of G takes ranks c, 2G-1-c, 2G+c, 4G-1-c, ... (a
+// snake order, which balances the per-CTA totals of a decreasing sequence).  Every
+// role of a CTA walks the same list, so they agree on the tiles without talking.
+__device__ __forceinline__ int snake_rank(int k, int c, int G) { return k * G + ((k & 1) ? (G - 1 - c) : c); }
 
 // ============================================================================ dK / dV
 template <int D>
@@ -110,24 +121,27 @@ struct DkdvCfg {
     static constexpr int kOffDO = kOffQ + kStages * kTile;   // + st * kTile
     static constexpr int kOffVec = kOffDO + kStages * kTile; // + st * 1024: lse2[128], D[128]
     static constexpr int kOffBar = kOffVec + kStages * 1024;
-    static constexpr int kBarKV = 0;
-    static constexpr int kBarQFull = 1;                  // + st
-    static constexpr int kBarQEmpty = 1 + kStages;       // + st
-    static constexpr int kBarSFull = 1 + 2 * kStages;
-    static constexpr int kBarDPFull = 2 + 2 * kStages;
-    static constexpr int kBarPFull = 3 + 2 * kStages;    // P^T written (256 threads)
-    static constexpr int kBarDSFull = 4 + 2 * kStages;   // dS^T written (256 threads)
-    static constexpr int kBarKdv = 5 + 2 * kStages;
-    static constexpr int kBarDone = 6 + 2 * kStages;
-    static constexpr int kNumBars = 7 + 2 * kStages;
+    static constexpr int kBarKVFull = 0;
+    static constexpr int kBarKVEmpty = 1;                // K_j, V_j free: the tile's last S^T/dP^T are done
+    static constexpr int kBarQFull = 2;                  // + st
+    static constexpr int kBarQEmpty = 2 + kStages;       // + st
+    static constexpr int kBarSFull = 2 + 2 * kStages;
+    static constexpr int kBarDPFull = 3 + 2 * kStages;
+    static constexpr int kBarPFull = 4 + 2 * kStages;    // P^T written (256 threads)
+    static constexpr int kBarDSFull = 5 + 2 * kStages;   // dS^T written (256 threads)
+    static constexpr int kBarKdv = 6 + 2 * kStages;      // dV, dK accumulators complete
+    static constexpr int kBarAccFree = 7 + 2 * kStages;  // dV, dK copied out of TMEM (256 threads)
+    static constexpr int kBarDone = 8 + 2 * kStages;
+    static constexpr int kNumBars = 9 + 2 * kStages;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
     static_assert(kTile % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
 
 template <int D>
-__device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                                          const CUtensorMap &tm_do, const BwdParams &p, uint8_t *smem_raw, int j) {
+__device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                                const CUtensorMap &tm_v, const CUtensorMap &tm_do,
+                                                const BwdParams &p, uint8_t *smem_raw) {
     using C = DkdvCfg<D>;
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
@@ -137,14 +151,25 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    int start, len;
-    p.g.slice(b, start, len);
-    const int kv0 = j * 128;
-    if (kv0 >= len) return;  // uniform, before any barrier or allocation
-    const int nq_all = (len + 127) / 128;
-    const int i0 = p.causal ? j : 0;
-    const int nq = nq_all - i0;  // >= 1
+    const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+    const int BH = p.g.B * p.g.H;
+    const int T = BH * p.n_tiles;
+    // work unit of rank r: key tile j (heaviest = 0), slice (b, h); false if empty
+    struct Tile {
+        int b, h, j, start, len, kv0, i0, nq;
+    };
+    auto tile_at = [&](int r, Tile &t) -> bool {
+        t.j = r / BH;
+        const int bh = r - t.j * BH;
+        t.b = bh / p.g.H;
+        t.h = bh - t.b * p.g.H;
+        p.g.slice(t.b, t.start, t.len);
+        t.kv0 = t.j * 128;
+        if (t.kv0 >= t.len) return false;
+        t.i0 = p.causal ? t.j : 0;
+        t.nq = (t.len + 127) / 128 - t.i0;
+        return true;
+    };
 
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -152,7 +177,7 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i)
-            mbar_init(bar(i), (i == C::kBarPFull || i == C::kBarDSFull) ? 256u : 1u);
+            mbar_init(bar(i), (i == C::kBarPFull || i == C::kBarDSFull || i == C::kBarAccFree) ? 256u : 1u);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -160,55 +185,67 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const long long lrow0 = p.g.base(b, h, start, 1);
-    const long long lrs = p.g.row_stride(1);
-    int n_issued = 0;  // loader: query-tile loads 0 .. n_issued-1 were started
+    int n_q = 0, n_kv = 0;  // loader: query-tile and K/V loads started (for the abort drain)
 
     if (warp == 8) {
         // ------------------------------------------------------------ loader
-        const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTile);
-#pragma unroll
-            for (int x = 0; x < C::kBoxes; ++x) {
-                tma_load_3d(sbase + C::kOffK + x * 16384, &tm_k, bar(C::kBarKV), x * 64, row0 + kv0, slab);
-                tma_load_3d(sbase + C::kOffV + x * 16384, &tm_v, bar(C::kBarKV), x * 64, row0 + kv0, slab);
-            }
         }
-        for (int it = 0; it < nq; ++it) {
-            const int st = it % C::kStages;
-            const bool ok = __all_sync(
-                0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((it / C::kStages) & 1) ^ 1, p.ctl, abort_flag));
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            const int r = snake_rank(k, cta, G);
+            if (r >= T) break;
+            Tile t;
+            if (!tile_at(r, t)) continue;
+            const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
+            const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
+            // K_j, V_j once the previous tile's last S^T / dP^T have read theirs
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKVEmpty), (n_kv & 1) ^ 1, p.ctl, abort_flag));
             if (!ok) break;
-            const int q0 = (i0 + it) * 128;
-            float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int q = q0 + u * 32 + lane;
-                float l2 = INFINITY, dd = 0.f;  // rows past the sequence: P = 0
-                if (q < len) {
-                    l2 = p.lse2[lrow0 + q * lrs];
-                    dd = p.dvec[lrow0 + q * lrs];
-                }
-                vec[u * 32 + lane] = l2;
-                vec[128 + u * 32 + lane] = dd;
-            }
-            __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
+                mbar_arrive_expect_tx(bar(C::kBarKVFull), 2 * C::kTile);
 #pragma unroll
                 for (int x = 0; x < C::kBoxes; ++x) {
-                    tma_load_3d(sbase + C::kOffQ + st * C::kTile + x * 16384, &tm_q, bar(C::kBarQFull + st), x * 64,
-                                row0 + q0, slab);
-                    tma_load_3d(sbase + C::kOffDO + st * C::kTile + x * 16384, &tm_do, bar(C::kBarQFull + st),
-                                x * 64, row0 + q0, slab);
+                    tma_load_3d(sbase + C::kOffK + x * 16384, &tm_k, bar(C::kBarKVFull), x * 64, row0 + t.kv0, slab);
+                    tma_load_3d(sbase + C::kOffV + x * 16384, &tm_v, bar(C::kBarKVFull), x * 64, row0 + t.kv0, slab);
                 }
             }
-            n_issued = it + 1;
+            ++n_kv;
+            for (int it = 0; it < t.nq; ++it) {
+                const int gi = n_q, st = gi % C::kStages;
+                ok = __all_sync(0xffffffffu,
+                                wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1, p.ctl, abort_flag));
+                if (!ok) break;
+                const int q0 = (t.i0 + it) * 128;
+                float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int q = q0 + u * 32 + lane;
+                    float l2 = INFINITY, dd = 0.f;  // rows past the sequence: P = 0
+                    if (q < t.len) {
+                        l2 = p.lse2[lrow0 + q * lrs];
+                        dd = p.dvec[lrow0 + q * lrs];
+                    }
+                    vec[u * 32 + lane] = l2;
+                    vec[128 + u * 32 + lane] = dd;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
+#pragma unroll
+                    for (int x = 0; x < C::kBoxes; ++x) {
+                        tma_load_3d(sbase + C::kOffQ + st * C::kTile + x * 16384, &tm_q, bar(C::kBarQFull + st),
+                                    x * 64, row0 + q0, slab);
+                        tma_load_3d(sbase + C::kOffDO + st * C::kTile + x * 16384, &tm_do, bar(C::kBarQFull + st),
+                                    x * 64, row0 + q0, slab);
+                    }
+                }
+                ++n_q;
+            }
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
@@ -219,63 +256,84 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
             // 64-127 at columns 64-95 of the S^T / dP^T regions (each math warp writes
             // only inside the columns it read).
             auto acol = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
-            auto issue_s = [&](int it) {
-                const uint32_t qs = sbase + C::kOffQ + (it % C::kStages) * C::kTile;
+            auto issue_s = [&](int gi) {
+                const uint32_t qs = sbase + C::kOffQ + (gi % C::kStages) * C::kTile;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + C::kColS, sw128_desc(sbase + C::kOffK + kstep_off(kk), 16, 1024),
                            sw128_desc(qs + kstep_off(kk), 16, 1024), idS, kk > 0);
                 tc_commit(bar(C::kBarSFull));
             };
-            auto issue_dp = [&](int it) {
-                const uint32_t ds = sbase + C::kOffDO + (it % C::kStages) * C::kTile;
+            auto issue_dp = [&](int gi) {
+                const uint32_t ds = sbase + C::kOffDO + (gi % C::kStages) * C::kTile;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffV + kstep_off(kk), 16, 1024),
                            sw128_desc(ds + kstep_off(kk), 16, 1024), idS, kk > 0);
                 tc_commit(bar(C::kBarDPFull));
             };
-            bool ok = wait_phase(bar(C::kBarKV), 0, p.ctl, abort_flag);
-            if (ok) ok = wait_phase(bar(C::kBarQFull + 0), 0, p.ctl, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0);
-                issue_dp(0);
-            }
-            for (int it = 0; ok && it < nq; ++it) {
-                const int st = it % C::kStages;
-                const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
-                const uint32_t dos = sbase + C::kOffDO + st * C::kTile;
-                const bool more = it + 1 < nq;
-                // dV += P^T dO_i   (K = 128 queries: 8 steps)
-                ok = wait_phase(bar(C::kBarPFull), it & 1, p.ctl, abort_flag);
+            auto wait_q = [&](int gi) {
+                return wait_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+            };
+            bool ok = true;
+            int gbase = 0, n_t = 0;
+            for (int k = 0; ok; ++k) {
+                const int r = snake_rank(k, cta, G);
+                if (r >= T) break;
+                Tile t;
+                if (!tile_at(r, t)) continue;
+                ok = wait_phase(bar(C::kBarKVFull), n_t & 1, p.ctl, abort_flag);
+                if (ok) ok = wait_q(gbase);
                 if (!ok) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::kColDV, tmem + C::kColS + acol(kk), sw128_desc(dos + kk * 2048, 16384, 1024),
-                           idKV, (it > 0 || kk > 0) ? 1u : 0u);
-                // S^T_{i+1} may overwrite P^T_i now: the math warps keep P in registers
-                // and dV_i, issued first, completes first.
-                if (more) {
-                    ok = wait_phase(bar(C::kBarQFull + (it + 1) % C::kStages), ((it + 1) / C::kStages) & 1, p.ctl,
-                                    abort_flag);
+                // S^T / dP^T regions are free: the previous tile's last dV / dK, which
+                // read P^T / dS^T from them, were issued earlier (in-order completion)
+                // and its math warps had finished reading before those were issued.
+                issue_s(gbase);
+                issue_dp(gbase);
+                if (t.nq == 1) tc_commit(bar(C::kBarKVEmpty));
+                for (int it = 0; ok && it < t.nq; ++it) {
+                    const int gi = gbase + it, st = gi % C::kStages;
+                    const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
+                    const uint32_t dos = sbase + C::kOffDO + st * C::kTile;
+                    const bool more = it + 1 < t.nq;
+                    // dV += P^T dO_i   (K = 128 queries: 8 steps)
+                    ok = wait_phase(bar(C::kBarPFull), gi & 1, p.ctl, abort_flag);
+                    if (ok && it == 0 && n_t > 0)  // the previous tile's dV / dK have been copied out
+                        ok = wait_phase(bar(C::kBarAccFree), (n_t - 1) & 1, p.ctl, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(it + 1);
-                }
-                // dK += dS^T Q_i
-                ok = wait_phase(bar(C::kBarDSFull), it & 1, p.ctl, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::kColDK, tmem + C::kColDP + acol(kk), sw128_desc(qs + kk * 2048, 16384, 1024),
-                           idKV, (it > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(C::kBarQEmpty + st));
-                if (more) issue_dp(it + 1);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::kColDV, tmem + C::kColS + acol(kk), sw128_desc(dos + kk * 2048, 16384, 1024),
+                               idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                    // S^T_{i+1} may overwrite P^T_i now: the math warps keep P in registers
+                    // and dV_i, issued first, completes first.
+                    if (more) {
+                        ok = wait_q(gi + 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(gi + 1);
+                    }
+                    // dK += dS^T Q_i
+                    ok = wait_phase(bar(C::kBarDSFull), gi & 1, p.ctl, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::kColDK, tmem + C::kColDP + acol(kk), sw128_desc(qs + kk * 2048, 16384, 1024),
+                               idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(C::kBarQEmpty + st));
+                    if (more) {
+                        issue_dp(gi + 1);
+                        if (it + 2 == t.nq) tc_commit(bar(C::kBarKVEmpty));  // last S^T / dP^T of the tile
+                    }
+                }
+                if (!ok) break;
+                tc_commit(bar(C::kBarKdv));
+                gbase += t.nq;
+                ++n_t;
             }
-            if (ok) tc_commit(bar(C::kBarKdv));
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
         }
@@ -284,108 +342,122 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
         // warp w: key rows 32*(w%4).., query columns 64*(w/4) .. +63 of each query tile.
         const int q4 = warp & 3, hf = warp >> 2;
         const int kr = q4 * 32 + lane;  // key row within the tile
-        const int key = kv0 + kr;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
         const uint32_t tS = tmem + lane_off + C::kColS + hf * 64;
         const uint32_t tDP = tmem + lane_off + C::kColDP + hf * 64;
-        bool kvalid = key < len;
-        if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(b, start) + key] != 0;
         const float c2 = p.scale_log2;
         bool ok = true;
-        for (int it = 0; it < nq; ++it) {
-            const int st = it % C::kStages;
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull), it & 1, p.ctl, abort_flag));
-            if (ok)
-                ok = __all_sync(0xffffffffu,
-                                wait_phase(bar(C::kBarQFull + st), (it / C::kStages) & 1, p.ctl, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const float4 *vec = reinterpret_cast<const float4 *>(sptr + C::kOffVec + st * 1024) + hf * 16;
-            uint32_t sr[2][32];
-            tmem_ld32(tS, sr[0]);
-            tmem_ld32(tS + 32, sr[1]);
-            tmem_wait_ld();
-            // P^T = 2^(S^T c - lse2), 0 where the query precedes the key (causal),
-            // for keys outside the sequence or padded, and for rows past the end.
-            const int qb = (i0 + it) * 128 + hf * 64;  // first query column of this warp
-            int lim = p.causal ? key - qb : 0;          // columns c < lim are masked
-            if (!kvalid) lim = 64;
-            float pf[64];
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 l2 = vec[c4];
-                const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = c4 * 4 + e;
-                    pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2v[e]));
-                }
-            }
-            if (lim > 0) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c < lim) pf[c] = 0.f;
-            }
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pf[x * 32 + 2 * c], pf[x * 32 + 2 * c + 1]);
-                tmem_st16(tS + x * 16, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarPFull));
-            // dS^T = P^T o (dP^T - D), P taken from registers (fp32)
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), it & 1, p.ctl, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                uint32_t dr[32];
-                tmem_ld32(tDP + x * 32, dr);
+        int gbase = 0, n_t = 0;
+        for (int k = 0; ok; ++k) {
+            const int r = snake_rank(k, cta, G);
+            if (r >= T) break;
+            Tile t;
+            if (!tile_at(r, t)) continue;
+            const int key = t.kv0 + kr;
+            bool kvalid = key < t.len;
+            if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(t.b, t.start) + key] != 0;
+            for (int it = 0; it < t.nq; ++it) {
+                const int gi = gbase + it, st = gi % C::kStages;
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull), gi & 1, p.ctl, abort_flag));
+                if (ok)
+                    ok = __all_sync(0xffffffffu,
+                                    wait_phase(bar(C::kBarQFull + st), (gi / C::kStages) & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                const float4 *vec = reinterpret_cast<const float4 *>(sptr + C::kOffVec + st * 1024) + hf * 16;
+                uint32_t sr[2][32];
+                tmem_ld32(tS, sr[0]);
+                tmem_ld32(tS + 32, sr[1]);
                 tmem_wait_ld();
-                uint32_t pk[16];
+                // P^T = 2^(S^T c - lse2), 0 where the query precedes the key (causal),
+                // for keys outside the sequence or padded, and for rows past the end.
+                const int qb = (t.i0 + it) * 128 + hf * 64;  // first query column of this warp
+                int lim = p.causal ? key - qb : 0;            // columns c < lim are masked
+                if (!kvalid) lim = 64;
+                float pf[64];
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const float4 dd = vec[32 + x * 8 + c4];
-                    const int c = x * 32 + c4 * 4;
-                    pk[2 * c4] = pack_bf16x2(pf[c] * (__uint_as_float(dr[c4 * 4]) - dd.x),
-                                             pf[c + 1] * (__uint_as_float(dr[c4 * 4 + 1]) - dd.y));
-                    pk[2 * c4 + 1] = pack_bf16x2(pf[c + 2] * (__uint_as_float(dr[c4 * 4 + 2]) - dd.z),
-                                                 pf[c + 3] * (__uint_as_float(dr[c4 * 4 + 3]) - dd.w));
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 l2 = vec[c4];
+                    const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = c4 * 4 + e;
+                        pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2v[e]));
+                    }
                 }
-                tmem_st16(tDP + x * 16, pk);
+                if (lim > 0) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < lim) pf[c] = 0.f;
+                }
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pf[x * 32 + 2 * c], pf[x * 32 + 2 * c + 1]);
+                    tmem_st16(tS + x * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull));
+                // dS^T = P^T o (dP^T - D), P taken from registers (fp32)
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), gi & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    uint32_t dr[32];
+                    tmem_ld32(tDP + x * 32, dr);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 dd = vec[32 + x * 8 + c4];
+                        const int c = x * 32 + c4 * 4;
+                        pk[2 * c4] = pack_bf16x2(pf[c] * (__uint_as_float(dr[c4 * 4]) - dd.x),
+                                                 pf[c + 1] * (__uint_as_float(dr[c4 * 4 + 1]) - dd.y));
+                        pk[2 * c4 + 1] = pack_bf16x2(pf[c + 2] * (__uint_as_float(dr[c4 * 4 + 2]) - dd.z),
+                                                     pf[c + 3] * (__uint_as_float(dr[c4 * 4 + 3]) - dd.w));
+                    }
+                    tmem_st16(tDP + x * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarDSFull));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarDSFull));
-        }
-        // ---- epilogue: warps 0-3 write dV, warps 4-7 write scale * dK
-        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKdv), 0, p.ctl, abort_flag));
-        if (ok) {
+            if (!ok) break;
+            // ---- epilogue: warps 0-3 write dV, warps 4-7 write scale * dK; TMEM is
+            // released (acc free) as soon as the values are in registers
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKdv), n_t & 1, p.ctl, abort_flag));
+            if (!ok) break;
             tc_fence_after();
             const bool is_dv = hf == 0;
-            const bool valid = key < len;
-            const long long off = p.g.base(b, h, start, D) + static_cast<long long>(key) * p.g.row_stride(D);
+            const bool valid = key < t.len;
+            const long long off = p.g.base(t.b, t.h, t.start, D) + static_cast<long long>(key) * p.g.row_stride(D);
             __nv_bfloat16 *out = (is_dv ? p.dv : p.dk) + off;
             const float mul = is_dv ? 1.f : p.scale;
             const uint32_t col = is_dv ? C::kColDV : C::kColDK;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + col + c0, r);
+                uint32_t rr[32];
+                tmem_ld32(tmem + lane_off + col + c0, rr);
                 tmem_wait_ld();
+                if (c0 + 32 == D) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarAccFree));
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
+                    pk[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
+            gbase += t.nq;
+            ++n_t;
         }
     }
 
@@ -394,9 +466,9 @@ __device__ __forceinline__ void dkdv_body(const CUtensorMap &tm_q, const CUtenso
     __syncthreads();
     if (warp == 8 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        drain_phase(bar(C::kBarKV), 0, p.ctl, abort_flag);
-        for (int it = max(0, n_issued - C::kStages); it < n_issued; ++it)
-            drain_phase(bar(C::kBarQFull + it % C::kStages), (it / C::kStages) & 1, p.ctl, abort_flag);
+        if (n_kv > 0) drain_phase(bar(C::kBarKVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
+            drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
     }
     if (warp == 9) {
         tc_fence_after();
@@ -420,17 +492,21 @@ struct DqCfg {
     static constexpr int kOffK = 2 * kTile;                     // + s * kTile
     static constexpr int kOffV = kOffK + kKStages * kTile;      // + s * kTile
     static constexpr int kOffBar = kOffV + kVStages * kTile;
-    static constexpr int kBarQ = 0;
-    static constexpr int kBarKFull = 1;                          // + slot
+    static constexpr int kBarQFull = 0;                          // Q_i, dO_i of the tile loaded
+    static constexpr int kBarQEmpty = 1;                         // the tile's last S / dP are done
+    static constexpr int kBarKFull = 2;                          // + slot
     static constexpr int kBarKEmpty = kBarKFull + kKStages;      // + slot
     static constexpr int kBarVFull = kBarKEmpty + kKStages;      // + slot
     static constexpr int kBarVEmpty = kBarVFull + kVStages;      // + slot
     static constexpr int kBarSFull = kBarVEmpty + kVStages;      // + buffer
     static constexpr int kBarDPFull = kBarSFull + 2;
     static constexpr int kBarDPFree = kBarDPFull + 1;            // 256 threads copied dP out
-    static constexpr int kBarDSFull = kBarDPFree + 1;            // 256 threads wrote dS
-    static constexpr int kBarDq = kBarDSFull + 1;
-    static constexpr int kBarDone = kBarDq + 1;
+    // 256 threads wrote dS, + buffer: per buffer, so that the math warps (which may
+    // finish step j+1 before the issuer looks at step j) never run two phases ahead
+    static constexpr int kBarDSFull = kBarDPFree + 1;
+    static constexpr int kBarDq = kBarDSFull + 2;                // dQ accumulator complete
+    static constexpr int kBarAccFree = kBarDq + 1;               // dQ copied out of TMEM (256 threads)
+    static constexpr int kBarDone = kBarAccFree + 1;
     static constexpr int kNumBars = kBarDone + 1;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
     static_assert(kTile % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
@@ -439,26 +515,40 @@ struct DqCfg {
 };
 
 template <int D>
-__device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                                        const CUtensorMap &tm_do, const BwdParams &p, uint8_t *smem_raw, int qt) {
+__device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                              const CUtensorMap &tm_v, const CUtensorMap &tm_do,
+                                              const BwdParams &p, uint8_t *smem_raw) {
     using C = DqCfg<D>;
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
     uint8_t *sptr = smem_raw + (sbase - raw_u32);
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
-    auto kslot = [&](int jt) -> uint32_t { return sbase + C::kOffK + static_cast<uint32_t>(jt % C::kKStages) * C::kTile; };
-    auto vslot = [&](int jt) -> uint32_t { return sbase + C::kOffV + static_cast<uint32_t>(jt % C::kVStages) * C::kTile; };
+    auto kslot = [&](int gj) -> uint32_t { return sbase + C::kOffK + static_cast<uint32_t>(gj % C::kKStages) * C::kTile; };
+    auto vslot = [&](int gj) -> uint32_t { return sbase + C::kOffV + static_cast<uint32_t>(gj % C::kVStages) * C::kTile; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    int start, len;
-    p.g.slice(b, start, len);
-    const int q0 = qt * 128;
-    if (q0 >= len) return;
-    const int nkv_all = (len + 127) / 128;
-    const int nkv = p.causal ? min(nkv_all, qt + 1) : nkv_all;
+    const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+    const int BH = p.g.B * p.g.H;
+    const int T = BH * p.n_tiles;
+    // work unit of rank r: query tile qt (heaviest = the last), slice (b, h); false if empty
+    struct Tile {
+        int b, h, qt, start, len, q0, nkv;
+    };
+    auto tile_at = [&](int r, Tile &t) -> bool {
+        const int k = r / BH;
+        const int bh = r - k * BH;
+        t.qt = p.n_tiles - 1 - k;
+        t.b = bh / p.g.H;
+        t.h = bh - t.b * p.g.H;
+        p.g.slice(t.b, t.start, t.len);
+        t.q0 = t.qt * 128;
+        if (t.q0 >= t.len) return false;
+        const int nkv_all = (t.len + 127) / 128;
+        t.nkv = p.causal ? min(nkv_all, t.qt + 1) : nkv_all;
+        return true;
+    };
 
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -466,7 +556,8 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i)
-            mbar_init(bar(i), (i == C::kBarDPFree || i == C::kBarDSFull) ? 256u : 1u);
+            mbar_init(bar(i), (i == C::kBarDPFree || i == C::kBarDSFull || i == C::kBarDSFull + 1 ||
+                               i == C::kBarAccFree) ? 256u : 1u);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -474,8 +565,7 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    int n_issued = 0;  // loader: K/V tiles 0 .. n_issued-1 were started (K_j before V_j)
-    bool v_issued_last = true;
+    int n_k = 0, n_v = 0, n_qt = 0;  // loader: K/V tiles and Q/dO pairs started (for the abort drain)
 
     if (warp == 8) {
         // ------------------------------------------------------------ loader
@@ -484,28 +574,46 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
-            mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTile);
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int r = snake_rank(k, cta, G);
+                if (r >= T) break;
+                Tile t;
+                if (!tile_at(r, t)) continue;
+                const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
+                // Q_i, dO_i once the previous tile's last S / dP have read theirs
+                if (!wait_phase(bar(C::kBarQEmpty), (n_qt & 1) ^ 1, p.ctl, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(C::kBarQFull), 2 * C::kTile);
 #pragma unroll
-            for (int x = 0; x < C::kBoxes; ++x) {
-                tma_load_3d(sbase + C::kOffQ + x * 16384, &tm_q, bar(C::kBarQ), x * 64, row0 + q0, slab);
-                tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQ), x * 64, row0 + q0, slab);
-            }
-            for (int jt = 0; jt < nkv; ++jt) {
-                const int ks = jt % C::kKStages, vs = jt % C::kVStages;
-                if (!wait_phase(bar(C::kBarKEmpty + ks), ((jt / C::kKStages) & 1) ^ 1, p.ctl, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(C::kBarKFull + ks), C::kTile);
+                for (int x = 0; x < C::kBoxes; ++x) {
+                    tma_load_3d(sbase + C::kOffQ + x * 16384, &tm_q, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
+                    tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
+                }
+                ++n_qt;
+                for (int jt = 0; jt < t.nkv; ++jt) {
+                    const int gk = n_k, ks = gk % C::kKStages;
+                    if (!wait_phase(bar(C::kBarKEmpty + ks), ((gk / C::kKStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(C::kBarKFull + ks), C::kTile);
 #pragma unroll
-                for (int x = 0; x < C::kBoxes; ++x)
-                    tma_load_3d(kslot(jt) + x * 16384, &tm_k, bar(C::kBarKFull + ks), x * 64, row0 + 128 * jt, slab);
-                n_issued = jt + 1;
-                v_issued_last = false;
-                if (!wait_phase(bar(C::kBarVEmpty + vs), ((jt / C::kVStages) & 1) ^ 1, p.ctl, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
+                    for (int x = 0; x < C::kBoxes; ++x)
+                        tma_load_3d(kslot(gk) + x * 16384, &tm_k, bar(C::kBarKFull + ks), x * 64, row0 + 128 * jt,
+                                    slab);
+                    ++n_k;
+                    const int gv = n_v, vs = gv % C::kVStages;
+                    if (!wait_phase(bar(C::kBarVEmpty + vs), ((gv / C::kVStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
 #pragma unroll
-                for (int x = 0; x < C::kBoxes; ++x)
-                    tma_load_3d(vslot(jt) + x * 16384, &tm_v, bar(C::kBarVFull + vs), x * 64, row0 + 128 * jt, slab);
-                v_issued_last = true;
+                    for (int x = 0; x < C::kBoxes; ++x)
+                        tma_load_3d(vslot(gv) + x * 16384, &tm_v, bar(C::kBarVFull + vs), x * 64, row0 + 128 * jt,
+                                    slab);
+                    ++n_v;
+                }
             }
         }
     } else if (warp == 9) {
@@ -513,71 +621,86 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idQ = idesc_bf16_f32(128, D, 0, 1);
-            auto issue_s = [&](int jt) {
-                const uint32_t ks = kslot(jt);
-                const uint32_t col = (jt & 1) ? C::kColS1 : C::kColS0;
+            auto issue_s = [&](int gj) {
+                const uint32_t ks = kslot(gj);
+                const uint32_t col = (gj & 1) ? C::kColS1 : C::kColS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + col, sw128_desc(sbase + C::kOffQ + kstep_off(kk), 16, 1024),
                            sw128_desc(ks + kstep_off(kk), 16, 1024), idS, kk > 0);
-                tc_commit(bar(C::kBarSFull + (jt & 1)));
+                tc_commit(bar(C::kBarSFull + (gj & 1)));
             };
-            auto issue_dp = [&](int jt) {
-                const uint32_t vs = vslot(jt);
+            auto issue_dp = [&](int gj) {
+                const uint32_t vs = vslot(gj);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffDO + kstep_off(kk), 16, 1024),
                            sw128_desc(vs + kstep_off(kk), 16, 1024), idS, kk > 0);
                 tc_commit(bar(C::kBarDPFull));
-                tc_commit(bar(C::kBarVEmpty + jt % C::kVStages));  // V_j is free once dP_j is done
+                tc_commit(bar(C::kBarVEmpty + gj % C::kVStages));  // V_j is free once dP_j is done
             };
-            auto wait_k = [&](int jt) {
-                return wait_phase(bar(C::kBarKFull + jt % C::kKStages), (jt / C::kKStages) & 1, p.ctl, abort_flag);
+            auto wait_k = [&](int gj) {
+                return wait_phase(bar(C::kBarKFull + gj % C::kKStages), (gj / C::kKStages) & 1, p.ctl, abort_flag);
             };
-            auto wait_v = [&](int jt) {
-                return wait_phase(bar(C::kBarVFull + jt % C::kVStages), (jt / C::kVStages) & 1, p.ctl, abort_flag);
+            auto wait_v = [&](int gj) {
+                return wait_phase(bar(C::kBarVFull + gj % C::kVStages), (gj / C::kVStages) & 1, p.ctl, abort_flag);
             };
-            bool ok = wait_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
-            if (ok) ok = wait_k(0);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0);
-                ok = wait_v(0);
-            }
-            if (ok) {
-                tc_fence_after();
-                issue_dp(0);
-            }
-            for (int jt = 0; ok && jt < nkv; ++jt) {
-                if (jt + 1 < nkv) {
-                    // S_{j+1} into the other buffer (its previous dS was read by dQ_{j-1},
-                    // issued earlier: in-order completion makes the overwrite safe)
-                    ok = wait_k(jt + 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_s(jt + 1);
-                    // dP_{j+1} once the softmax warps have copied dP_j out
-                    ok = wait_phase(bar(C::kBarDPFree), jt & 1, p.ctl, abort_flag);
-                    if (ok) ok = wait_v(jt + 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_dp(jt + 1);
-                }
-                // dQ += dS_j K_j  (A = dS from TMEM: keys 0-63 at columns 0-31, keys 64-127 at 64-95)
-                ok = wait_phase(bar(C::kBarDSFull), jt & 1, p.ctl, abort_flag);
+            bool ok = true;
+            int gbase = 0, n_t = 0;
+            for (int k = 0; ok; ++k) {
+                const int r = snake_rank(k, cta, G);
+                if (r >= T) break;
+                Tile t;
+                if (!tile_at(r, t)) continue;
+                ok = wait_phase(bar(C::kBarQFull), n_t & 1, p.ctl, abort_flag);
+                if (ok) ok = wait_k(gbase);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t scol = (jt & 1) ? C::kColS1 : C::kColS0;
-                const uint32_t ks = kslot(jt);
+                // S buffer gbase & 1 last held dS of step gbase-2, read by a dQ product
+                // issued earlier; the dP region was copied out (dP free) before the
+                // previous tile's last dQ was issued.
+                issue_s(gbase);
+                if (n_t > 0) ok = wait_phase(bar(C::kBarDPFree), (gbase - 1) & 1, p.ctl, abort_flag);
+                if (ok) ok = wait_v(gbase);
+                if (!ok) break;
+                tc_fence_after();
+                issue_dp(gbase);
+                if (t.nkv == 1) tc_commit(bar(C::kBarQEmpty));
+                for (int jt = 0; ok && jt < t.nkv; ++jt) {
+                    const int gj = gbase + jt;
+                    if (jt + 1 < t.nkv) {
+                        ok = wait_k(gj + 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(gj + 1);
+                        ok = wait_phase(bar(C::kBarDPFree), gj & 1, p.ctl, abort_flag);
+                        if (ok) ok = wait_v(gj + 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_dp(gj + 1);
+                        if (jt + 2 == t.nkv) tc_commit(bar(C::kBarQEmpty));  // last S / dP of the tile
+                    }
+                    // dQ += dS_j K_j  (A = dS from TMEM: keys 0-63 at columns 0-31, keys 64-127 at 64-95)
+                    ok = wait_phase(bar(C::kBarDSFull + (gj & 1)), (gj >> 1) & 1, p.ctl, abort_flag);
+                    if (ok && jt == 0 && n_t > 0)  // the previous tile's dQ has been copied out
+                        ok = wait_phase(bar(C::kBarAccFree), (n_t - 1) & 1, p.ctl, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t scol = (gj & 1) ? C::kColS1 : C::kColS0;
+                    const uint32_t ks = kslot(gj);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t acol = scol + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-                    mma_ts(tmem + C::kColDQ, tmem + acol, sw128_desc(ks + kk * 2048, 16384, 1024), idQ,
-                           (jt > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t acol = scol + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+                        mma_ts(tmem + C::kColDQ, tmem + acol, sw128_desc(ks + kk * 2048, 16384, 1024), idQ,
+                               (jt > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(bar(C::kBarKEmpty + gj % C::kKStages));  // K_j is free once dQ_j is done
                 }
-                tc_commit(bar(C::kBarKEmpty + jt % C::kKStages));  // K_j is free once dQ_j is done
+                if (!ok) break;
+                tc_commit(bar(C::kBarDq));
+                gbase += t.nkv;
+                ++n_t;
             }
-            if (ok) tc_commit(bar(C::kBarDq));
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
         }
@@ -585,90 +708,104 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
         // ------------------------------------------------------------ P and dS (8 warps)
         // warp w: query rows 32*(w%4).., keys 64*(w/4) .. +63 of each key tile.
         const int q4 = warp & 3, hf = warp >> 2;
-        const int qrow = q0 + q4 * 32 + lane;  // query row within the slice
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-        const long long lidx = p.g.base(b, h, start, 1) + static_cast<long long>(qrow) * p.g.row_stride(1);
-        const float l2 = (qrow < len) ? p.lse2[lidx] : INFINITY;  // rows past the sequence: P = 0
-        const float dd = (qrow < len) ? p.dvec[lidx] : 0.f;
         const float c2 = p.scale_log2;
-        const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(b, start) : nullptr;
         bool ok = true;
-        for (int jt = 0; jt < nkv; ++jt) {
-            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull + (jt & 1)), (jt >> 1) & 1, p.ctl, abort_flag));
-            if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), jt & 1, p.ctl, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t scol = (jt & 1) ? C::kColS1 : C::kColS0;
-            uint32_t sr[2][32], dr[2][32];
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                tmem_ld32(tmem + lane_off + scol + hf * 64 + x * 32, sr[x]);
-                tmem_ld32(tmem + lane_off + C::kColDP + hf * 64 + x * 32, dr[x]);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarDPFree));
-            // masking: keys outside the sequence, above the diagonal, or padded
-            const int kb = jt * 128 + hf * 64;  // first key of this warp's columns
-            int limit = len - kb;
-            if (p.causal) limit = min(limit, qrow - kb + 1);
-            uint32_t kmask[2] = {0xffffffffu, 0xffffffffu};
-            if (keep != nullptr) {
+        int gbase = 0, n_t = 0;
+        for (int k = 0; ok; ++k) {
+            const int r = snake_rank(k, cta, G);
+            if (r >= T) break;
+            Tile t;
+            if (!tile_at(r, t)) continue;
+            const int qrow = t.q0 + q4 * 32 + lane;  // query row within the slice
+            const long long lidx = p.g.base(t.b, t.h, t.start, 1) + static_cast<long long>(qrow) * p.g.row_stride(1);
+            const float l2 = (qrow < t.len) ? p.lse2[lidx] : INFINITY;  // rows past the sequence: P = 0
+            const float dd = (qrow < t.len) ? p.dvec[lidx] : 0.f;
+            const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(t.b, t.start) : nullptr;
+            for (int jt = 0; jt < t.nkv; ++jt) {
+                const int gj = gbase + jt;
+                ok = __all_sync(0xffffffffu,
+                                wait_phase(bar(C::kBarSFull + (gj & 1)), (gj >> 1) & 1, p.ctl, abort_flag));
+                if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), gj & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t scol = (gj & 1) ? C::kColS1 : C::kColS0;
+                uint32_t sr[2][32], dr[2][32];
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    const int c = x * 32 + lane;
-                    kmask[x] = __ballot_sync(0xffffffffu, (c < len - kb) && keep[kb + c] != 0);
+                    tmem_ld32(tmem + lane_off + scol + hf * 64 + x * 32, sr[x]);
+                    tmem_ld32(tmem + lane_off + C::kColDP + hf * 64 + x * 32, dr[x]);
                 }
-            }
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                float pf[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) pf[c] = ex2_approx(fmaf(__uint_as_float(sr[x][c]), c2, -l2));
-                // masks only where this warp's 32 keys need them
-                const int lim_x = limit - 32 * x;  // columns c >= lim_x are masked
-                if (lim_x < 32) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c >= lim_x) pf[c] = 0.f;
-                }
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarDPFree));
+                // masking: keys outside the sequence, above the diagonal, or padded
+                const int kb = jt * 128 + hf * 64;  // first key of this warp's columns
+                int limit = t.len - kb;
+                if (p.causal) limit = min(limit, qrow - kb + 1);
+                uint32_t kmask[2] = {0xffffffffu, 0xffffffffu};
                 if (keep != nullptr) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (!((kmask[x] >> c) & 1u)) pf[c] = 0.f;
+                    for (int x = 0; x < 2; ++x) {
+                        const int c = x * 32 + lane;
+                        kmask[x] = __ballot_sync(0xffffffffu, (c < t.len - kb) && keep[kb + c] != 0);
+                    }
                 }
-                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    pk[c >> 1] = pack_bf16x2(pf[c] * (__uint_as_float(dr[x][c]) - dd),
-                                             pf[c + 1] * (__uint_as_float(dr[x][c + 1]) - dd));
-                tmem_st16(tmem + lane_off + scol + hf * 64 + x * 16, pk);
+                for (int x = 0; x < 2; ++x) {
+                    float pf[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pf[c] = ex2_approx(fmaf(__uint_as_float(sr[x][c]), c2, -l2));
+                    const int lim_x = limit - 32 * x;  // columns c >= lim_x are masked
+                    if (lim_x < 32) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (c >= lim_x) pf[c] = 0.f;
+                    }
+                    if (keep != nullptr) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (!((kmask[x] >> c) & 1u)) pf[c] = 0.f;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2)
+                        pk[c >> 1] = pack_bf16x2(pf[c] * (__uint_as_float(dr[x][c]) - dd),
+                                                 pf[c + 1] * (__uint_as_float(dr[x][c + 1]) - dd));
+                    tmem_st16(tmem + lane_off + scol + hf * 64 + x * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarDSFull + (gj & 1)));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::kBarDSFull));
-        }
-        // ---- epilogue: scale * dQ in bf16 (warp w writes columns (w/4)*d/2 ..)
-        if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDq), 0, p.ctl, abort_flag));
-        if (ok) {
+            if (!ok) break;
+            // ---- epilogue: scale * dQ in bf16 (warp w writes columns (w/4)*d/2 ..)
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDq), n_t & 1, p.ctl, abort_flag));
+            if (!ok) break;
             tc_fence_after();
-            const bool valid = qrow < len;
-            __nv_bfloat16 *out = p.dq + p.g.base(b, h, start, D) + static_cast<long long>(qrow) * p.g.row_stride(D);
+            const bool valid = qrow < t.len;
+            __nv_bfloat16 *out = p.dq + p.g.base(t.b, t.h, t.start, D) + static_cast<long long>(qrow) * p.g.row_stride(D);
 #pragma unroll
             for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + C::kColDQ + c0, r);
+                uint32_t rr[32];
+                tmem_ld32(tmem + lane_off + C::kColDQ + c0, rr);
                 tmem_wait_ld();
+                if (c0 + 32 == (hf + 1) * (D / 2)) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarAccFree));
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * p.scale, __uint_as_float(r[2 * c + 1]) * p.scale);
+                    pk[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * p.scale, __uint_as_float(rr[2 * c + 1]) * p.scale);
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
+            gbase += t.nkv;
+            ++n_t;
         }
     }
 
@@ -677,12 +814,11 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
     __syncthreads();
     if (warp == 8 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
-        for (int jt = max(0, n_issued - C::kKStages); jt < n_issued; ++jt)
-            drain_phase(bar(C::kBarKFull + jt % C::kKStages), (jt / C::kKStages) & 1, p.ctl, abort_flag);
-        const int nv = v_issued_last ? n_issued : n_issued - 1;
-        for (int jt = max(0, nv - C::kVStages); jt < nv; ++jt)
-            drain_phase(bar(C::kBarVFull + jt % C::kVStages), (jt / C::kVStages) & 1, p.ctl, abort_flag);
+        if (n_qt > 0) drain_phase(bar(C::kBarQFull), (n_qt - 1) & 1, p.ctl, abort_flag);
+        for (int g = max(0, n_k - C::kKStages); g < n_k; ++g)
+            drain_phase(bar(C::kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, p.ctl, abort_flag);
+        for (int g = max(0, n_v - C::kVStages); g < n_v; ++g)
+            drain_phase(bar(C::kBarVFull + g % C::kVStages), (g / C::kVStages) & 1, p.ctl, abort_flag);
     }
     if (warp == 9) {
         tc_fence_after();
@@ -690,20 +826,24 @@ __device__ __forceinline__ void dq_body(const CUtensorMap &tm_q, const CUtensorM
     }
 }
 
-// ============================================================================ dK/dV and dQ kernel
-// mode 0: dK/dV CTAs; mode 1: dQ CTAs.  Along grid z the heaviest causal tiles of
-// each kind come first.
+// ============================================================================ kernels
+// Persistent: one CTA per SM walks its share of the work units.
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-attn_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                      const __grid_constant__ BwdParams p, int mode) {
+attn_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                           const __grid_constant__ BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
-    const int rank = static_cast<int>(blockIdx.z);  // 0 = heaviest tile of its kind
-    if (mode == 0)
-        dkdv_body<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw, rank);  // key tile j: small j has the most query tiles
-    else
-        dq_body<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw, p.n_tiles - 1 - rank);  // query tile: large has the most keys
+    dkdv_persistent<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    dq_persistent<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
 }
 
 // ============================================================================ launch
@@ -734,16 +874,21 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
     }
     // dK/dV then dQ, as two launches: one grid holding both kinds of CTA measured
     // slower than the two back to back.
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         max(DkdvCfg<D>::kSmemBytes, DqCfg<D>::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    const dim3 g(a.g.H, a.g.B, p.n_tiles);
+    const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_tiles;
+    const dim3 g(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
+    cudaError_t e;
     if (a.phases & 2) {
-        attn_bwd_sm100_kernel<D><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p, 0);
+        e = cudaFuncSetAttribute(attn_bwd_dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DkdvCfg<D>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attn_bwd_dkdv_sm100_kernel<D><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.phases & 4) {
-        attn_bwd_sm100_kernel<D><<<g, 320, DqCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p, 1);
+        e = cudaFuncSetAttribute(attn_bwd_dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DqCfg<D>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attn_bwd_dq_sm100_kernel<D><<<g, 320, DqCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -31,6 +31,7 @@ struct BwdLaunch {
     float scale;
     int causal;
     int phases;        // bit 0: preprocess, bit 1: dK/dV kernel, bit 2: dQ kernel
+    int num_sms;       // persistent grid size
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);
