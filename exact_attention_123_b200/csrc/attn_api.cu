@@ -148,6 +148,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     a.lse = lse;
     a.scale = scale;
     a.causal = is_causal ? 1 : 0;
+    a.num_sms = ds->num_sms > 0 ? ds->num_sms : 1;
     return attn::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

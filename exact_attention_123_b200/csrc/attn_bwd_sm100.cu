@@ -120,7 +120,8 @@ struct DkdvCfg {
     static constexpr int kOffQ = 2 * kTile;                  // + st * kTile
     static constexpr int kOffDO = kOffQ + kStages * kTile;   // + st * kTile
     static constexpr int kOffVec = kOffDO + kStages * kTile; // + st * 1024: lse2[128], D[128]
-    static constexpr int kOffBar = kOffVec + kStages * 1024;
+    static constexpr int kOffStage = kOffVec + kStages * 1024;  // 8 math warps x 2 KB output staging
+    static constexpr int kOffBar = kOffStage + 8 * 2048;
     static constexpr int kBarKVFull = 0;
     static constexpr int kBarKVEmpty = 1;                // K_j, V_j free: the tile's last S^T/dP^T are done
     static constexpr int kBarQFull = 2;                  // + st
@@ -432,11 +433,12 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
             if (!ok) break;
             tc_fence_after();
             const bool is_dv = hf == 0;
-            const bool valid = key < t.len;
-            const long long off = p.g.base(t.b, t.h, t.start, D) + static_cast<long long>(key) * p.g.row_stride(D);
-            __nv_bfloat16 *out = (is_dv ? p.dv : p.dk) + off;
+            const int key_w0 = t.kv0 + q4 * 32;  // this warp's first key row
+            __nv_bfloat16 *out0 = (is_dv ? p.dv : p.dk) + p.g.base(t.b, t.h, t.start, D) +
+                                  static_cast<long long>(key_w0) * p.g.row_stride(D);
             const float mul = is_dv ? 1.f : p.scale;
             const uint32_t col = is_dv ? C::kColDV : C::kColDK;
+            const uint32_t stage = sbase + C::kOffStage + warp * 2048;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t rr[32];
@@ -450,11 +452,7 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     pk[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
-                if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                }
+                warp_store_rows32(stage, pk, out0 + c0, p.g.row_stride(D), t.len - key_w0, lane);
             }
             gbase += t.nq;
             ++n_t;
@@ -785,7 +783,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
             tc_fence_after();
             const bool valid = qrow < t.len;
             __nv_bfloat16 *out = p.dq + p.g.base(t.b, t.h, t.start, D) + static_cast<long long>(qrow) * p.g.row_stride(D);
-#pragma unroll
+#pragma unroll 1  // (unrolled, the key loop above runs out of registers)
             for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
                 uint32_t rr[32];
                 tmem_ld32(tmem + lane_off + C::kColDQ + c0, rr);

@@ -3,6 +3,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "sm100_ptx.cuh"
@@ -93,6 +94,30 @@ __device__ __forceinline__ bool drain_phase(uint32_t bar, uint32_t parity, const
             return false;
         }
     }
+}
+
+// One warp writes a 32-row x 32-column bf16 block to global memory.  On entry lane
+// r holds row r as 16 packed words (the tensor-memory layout: one row per lane).
+// Stored directly, every warp store would touch 32 rows, 16 bytes each; instead
+// the block passes through a 2 KB shared-memory staging area so that each store
+// instruction writes 8 rows x 64 contiguous bytes.  Chunk c (16 bytes) of row r
+// sits at r*64 + ((c ^ (r >> 1)) & 3)*16, which keeps both the row-per-lane writes
+// and the 4-lanes-per-row reads free of bank conflicts.  Rows r >= nvalid are not
+// written.  dst0 points at column 0 of row 0; ld is the row stride in elements.
+__device__ __forceinline__ void warp_store_rows32(uint32_t stage, const uint32_t (&pk)[16], __nv_bfloat16 *dst0,
+                                                  long long ld, int nvalid, int lane) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        st_shared_v4(stage + lane * 64 + (((c ^ (lane >> 1)) & 3) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                     pk[4 * c + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = i * 8 + (lane >> 2), c = lane & 3;
+        const uint4 v = ld_shared_v4(stage + r * 64 + (((c ^ (r >> 1)) & 3) << 4));
+        if (r < nvalid) *reinterpret_cast<uint4 *>(dst0 + r * ld + c * 8) = v;
+    }
+    __syncwarp();  // the staging area is free again
 }
 
 }  // namespace attn

@@ -1,7 +1,7 @@
 // attn_fwd_sm100.cu -- fused exact-attention forward for B200 (sm_100a).
 //
-// One CTA owns 256 query rows of one (sequence, head) slice, as two 128-row
-// tiles Q0 and Q1, and sweeps the key/value tiles of 128 keys with the online
+// A work unit is 256 query rows of one (sequence, head) slice, as two 128-row
+// tiles Q0 and Q1, which sweeps the key/value tiles of 128 keys with the online
 // softmax recurrence ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", 第三步 §1;
 // codechina FlashAttention article §3.2): per query row a running max m, a running
 // sum l and an un-normalised output accumulator, rescaled when m moves, divided by
@@ -26,6 +26,12 @@
 // on S0(j+1) and vice versa.  Because tcgen05 operations issued by one thread
 // complete in order, the commit that publishes S_t(j+1) also proves PV_t(j) is
 // done, which is what makes reading/rescaling O_t and overwriting P_t safe.
+//
+// The kernel is persistent: one CTA per SM walks its units, ranked heaviest
+// first (causal: the last query rows see the most keys) and dealt to the CTAs in
+// a snake order.  Every barrier counts phases across units and the key/value ring
+// runs on, so the next unit's Q tiles load as soon as the current unit's last
+// S products are done and its first S products overlap the current epilogue.
 //
 // Exponentials are base 2: p = 2^(s * scale * log2(e) - m).  The running max is
 // only moved when a row's new max exceeds the one in use by more than 8 (log2
@@ -59,9 +65,11 @@ struct FwdCfg {
     static constexpr int kBarP = 3 + 2 * kStages;            // + tile
     static constexpr int kBarO = 5 + 2 * kStages;            // + tile
     static constexpr int kBarDone = 7 + 2 * kStages;
-    static constexpr int kNumBars = 8 + 2 * kStages;
+    static constexpr int kBarQEmpty = 8 + 2 * kStages;       // the unit's last S products are done
+    static constexpr int kNumBars = 9 + 2 * kStages;
     static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
-    static constexpr int kSmemBytes = 1024 + kSmemTiles + kNumBars * 8 + 16;
+    static constexpr int kOffBar = kSmemTiles;
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
@@ -73,8 +81,35 @@ struct FwdParams {
     float *lse;
     float scale_log2;  // scale * log2(e)
     int causal;
-    int n_pairs;       // 256-row query blocks per slice (grid z)
+    int n_pairs;       // 256-row query blocks per slice
 };
+
+// Unit r of the persistent schedule: k = r / (B*H) counts down the 256-row blocks
+// from the last one, so ranks are ordered heaviest first for causal masking.
+// CTA c of G takes ranks c, 2G-1-c, 2G+c, 4G-1-c, ... (snake order).
+struct FwdUnit {
+    int b, h, start, len, m0;
+    int nkv0, nkv1;  // key tiles seen by Q0 and Q1 (0: the tile lies past the sequence)
+    __device__ __forceinline__ int nkv(int t) const { return t ? nkv1 : nkv0; }
+    __device__ __forceinline__ int nkv_max() const { return max(nkv0, nkv1); }
+};
+
+__device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int G, FwdUnit &u) {
+    const int BH = p.g.B * p.g.H;
+    const int r = k * G + ((k & 1) ? (G - 1 - cta) : cta);
+    const int kk = r / BH;
+    const int bh = r - kk * BH;
+    u.b = bh / p.g.H;
+    u.h = bh - u.b * p.g.H;
+    p.g.slice(u.b, u.start, u.len);
+    u.m0 = (p.n_pairs - 1 - kk) * 256;
+    if (u.m0 >= u.len) return false;
+    const int nkv_all = (u.len + 127) / 128;
+    const int r1 = u.m0 + 128;
+    u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
+    u.nkv1 = (r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
+    return true;
+}
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -88,28 +123,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
     uint8_t *sptr = smem_raw + (sbase - raw_u32);
-    const uint32_t bars = sbase + C::kSmemTiles;
+    const uint32_t bars = sbase + C::kOffBar;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     auto slot = [&](int s) -> uint32_t { return sbase + static_cast<uint32_t>(2 + s) * C::kTileBytes; };
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kSmemTiles + C::kNumBars * 8);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.z);  // heaviest causal blocks first
-    int start, len;
-    p.g.slice(b, start, len);
-    const int m0 = pair * 256;
-    if (m0 >= len) return;  // uniform for the CTA, before any barrier or allocation
-
-    const int nkv_all = (len + 127) / 128;
-    int nkv[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int r0 = m0 + 128 * t;
-        nkv[t] = (r0 >= len) ? 0 : (p.causal ? min(nkv_all, r0 / 128 + 1) : nkv_all);
-    }
-    const int nkv_max = max(nkv[0], nkv[1]);
+    const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+    const int n_ranks = p.g.B * p.g.H * p.n_pairs;
+    // walks this CTA's units in order; every role uses the same walk
+#define FOR_EACH_UNIT(u)                                                        \
+    for (int k_ = 0; k_ * G < n_ranks; ++k_)                                     \
+        if (FwdUnit u; (k_ * G + ((k_ & 1) ? (G - 1 - cta) : cta)) < n_ranks && \
+                       fwd_unit(p, k_, cta, G, u))
 
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -129,6 +156,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     int n_issued = 0;  // producer: ring loads 0 .. n_issued-1 were started (except a skipped one)
+    int n_qload = 0;   // producer: Q pairs whose load was started
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
@@ -136,30 +164,38 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int row0 = p.g.tma_row0(start), slab = p.g.tma_slab(b, h);
-            mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTileBytes);
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int x = 0; x < C::kBoxes; ++x)
-                    tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
-                                row0 + m0 + 128 * t, slab);
             bool ok = true;
-            for (int j = 0; j < nkv_max && ok; ++j) {
+            int idx = 0;  // ring position, continuing across units
+            FOR_EACH_UNIT(u) {
+                if (!ok) break;
+                const int row0 = p.g.tma_row0(u.start), slab = p.g.tma_slab(u.b, u.h);
+                // Q0/Q1 once the previous unit's last S products have read theirs
+                if (!wait_phase(bar(C::kBarQEmpty), (n_qload & 1) ^ 1, p.ctl, abort_flag)) break;
+                mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTileBytes);
 #pragma unroll
-                for (int kv = 0; kv < 2; ++kv) {
-                    const int idx = 2 * j + kv, s = idx % C::kStages;
-                    if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
-                    mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
+                for (int t = 0; t < 2; ++t)
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x)
-                        tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
-                                    row0 + 128 * j, slab);
-                    n_issued = idx + 1;
+                        tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
+                                    row0 + u.m0 + 128 * t, slab);
+                ++n_qload;
+                const int nkv_max = u.nkv_max();
+                for (int j = 0; j < nkv_max && ok; ++j) {
+#pragma unroll
+                    for (int kv = 0; kv < 2; ++kv, ++idx) {
+                        const int s = idx % C::kStages;
+                        if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
+                        mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
+                                        row0 + 128 * j, slab);
+                        n_issued = idx + 1;
+                    }
                 }
             }
         }
@@ -170,9 +206,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
-            auto issue_S = [&](int t, int j) {
+            auto issue_S = [&](int t, int base, int j) {
                 const uint32_t qs = sbase + t * C::kTileBytes;
-                const uint32_t ks = slot((2 * j) % C::kStages);
+                const uint32_t ks = slot((base + 2 * j) % C::kStages);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -181,49 +217,67 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 tc_commit(bar(C::kBarS + t));
             };
-            auto issue_PV = [&](int t, int j) {
-                const uint32_t vs = slot((2 * j + 1) % C::kStages);
+            auto issue_PV = [&](int t, int base, int j) {
+                const uint32_t vs = slot((base + 2 * j + 1) % C::kStages);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sw128_desc(vs + kk * 2048, 16384, 1024), idPV,
                            (j > 0 || kk > 0) ? 1u : 0u);
             };
-            bool ok = wait_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
-            if (ok) ok = wait_phase(bar(C::kBarFull + 0), 0, p.ctl, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                for (int t = 0; t < 2; ++t)
-                    if (nkv[t] > 0) issue_S(t, 0);
-                tc_commit(bar(C::kBarEmpty + 0));
-            }
-            for (int j = 0; ok && j < nkv_max; ++j) {
-                const int vidx = 2 * j + 1, kidx = 2 * j + 2;
-                ok = wait_phase(bar(C::kBarFull + vidx % C::kStages), (vidx / C::kStages) & 1, p.ctl, abort_flag);
+            bool ok = true;
+            int base = 0;          // ring position of the unit's K_0
+            int n_u = 0;           // units started
+            int gs[2] = {0, 0};    // S_t products issued (all units): phase counters
+            int go[2] = {0, 0};    // units in which tile t was active
+            FOR_EACH_UNIT(u) {
                 if (!ok) break;
-                bool k_next = false;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (j < nkv[t]) {
-                        ok = wait_phase(bar(C::kBarP + t), j & 1, p.ctl, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_PV(t, j);
-                        if (j == nkv[t] - 1) tc_commit(bar(C::kBarO + t));
-                    }
-                    if (j + 1 < nkv[t]) {
-                        if (!k_next) {
-                            ok = wait_phase(bar(C::kBarFull + kidx % C::kStages), (kidx / C::kStages) & 1, p.ctl,
-                                            abort_flag);
+                const int nkv_max = u.nkv_max();
+                ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
+                if (ok) ok = wait_phase(bar(C::kBarFull + base % C::kStages), (base / C::kStages) & 1, p.ctl, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // S_t(0) may overwrite S_t / P_t: PV_t of the previous unit was issued
+                // earlier (in-order completion) after its softmax had read S_t.
+                for (int t = 0; t < 2; ++t)
+                    if (u.nkv(t) > 0) issue_S(t, base, 0);
+                tc_commit(bar(C::kBarEmpty + base % C::kStages));
+                if (nkv_max == 1) tc_commit(bar(C::kBarQEmpty));
+                for (int j = 0; ok && j < nkv_max; ++j) {
+                    const int vidx = base + 2 * j + 1, kidx = base + 2 * j + 2;
+                    ok = wait_phase(bar(C::kBarFull + vidx % C::kStages), (vidx / C::kStages) & 1, p.ctl, abort_flag);
+                    if (!ok) break;
+                    bool k_next = false;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j < u.nkv(t)) {
+                            ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
                             if (!ok) break;
+                            ++gs[t];
                             tc_fence_after();
-                            k_next = true;
+                            issue_PV(t, base, j);
+                            if (j == u.nkv(t) - 1) tc_commit(bar(C::kBarO + t));
                         }
-                        issue_S(t, j + 1);
+                        if (j + 1 < u.nkv(t)) {
+                            if (!k_next) {
+                                ok = wait_phase(bar(C::kBarFull + kidx % C::kStages), (kidx / C::kStages) & 1, p.ctl,
+                                                abort_flag);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_next = true;
+                            }
+                            issue_S(t, base, j + 1);
+                        }
                     }
+                    if (!ok) break;
+                    tc_commit(bar(C::kBarEmpty + vidx % C::kStages));
+                    if (k_next) tc_commit(bar(C::kBarEmpty + kidx % C::kStages));
+                    if (j + 2 == nkv_max) tc_commit(bar(C::kBarQEmpty));  // the unit's last S products
                 }
                 if (!ok) break;
-                tc_commit(bar(C::kBarEmpty + vidx % C::kStages));
-                if (k_next) tc_commit(bar(C::kBarEmpty + kidx % C::kStages));
+                base += 2 * nkv_max;
+                ++n_u;
+                for (int t = 0; t < 2; ++t) go[t] += (u.nkv(t) > 0);
             }
+            (void)go;
             // Every MMA issued above must have finished before TMEM / smem go away.
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
@@ -231,16 +285,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else {
         // ------------------------------------------------------------ softmax warps
         const int t = warp >> 2, q4 = warp & 3;
-        const int row = m0 + 128 * t + q4 * 32 + lane;  // query row within the slice
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
         const uint32_t tS = tmem + lane_off + (t ? C::kColS1 : C::kColS0);
         const uint32_t tO = tmem + lane_off + (t ? C::kColO1 : C::kColO0);
         const float c2 = p.scale_log2;
-        const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(b, start) : nullptr;
-        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nkv[t]; ++j) {
-            ok = wait_phase(bar(C::kBarS + t), j & 1, p.ctl, abort_flag);
+        int gs = 0;  // S_t phases consumed (all units)
+        int go = 0;  // units in which this tile was active
+        FOR_EACH_UNIT(u) {
+        if (!ok) break;
+        const int len = u.len;
+        const int row = u.m0 + 128 * t + q4 * 32 + lane;  // query row within the slice
+        const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(u.b, u.start) : nullptr;
+        float m_used = -INFINITY, l = 0.f;
+        for (int j = 0; j < u.nkv(t); ++j, ++gs) {
+            ok = wait_phase(bar(C::kBarS + t), gs & 1, p.ctl, abort_flag);
             if (!ok) break;
             tc_fence_after();
             uint32_t sr[4][32];
@@ -328,15 +387,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mbar_arrive(bar(C::kBarP + t));
         }
 
-        // ---- epilogue: O / l in bf16, lse in natural log
-        if (ok && nkv[t] > 0) ok = wait_phase(bar(C::kBarO + t), 0, p.ctl, abort_flag);
-        if (ok && nkv[t] > 0) {
+        // ---- epilogue: O / l in bf16, lse in natural log.  The next unit's PV_t(0),
+        // which overwrites O_t, is issued only after this thread's next P_t arrive.
+        if (ok && u.nkv(t) > 0) ok = wait_phase(bar(C::kBarO + t), go & 1, p.ctl, abort_flag);
+        if (ok && u.nkv(t) > 0) {
+            ++go;
             tc_fence_after();
             const bool valid = row < len;
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-            __nv_bfloat16 *orow = p.o + p.g.base(b, h, start, D) + static_cast<long long>(row) * p.g.row_stride(D);
-#pragma unroll
+            FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
+            fwd_unit(p, k_, cta, G, e);
+            __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
+#pragma unroll 1  // (unrolled, the 128-wide key loop above runs out of registers)
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t orr[32];
                 tmem_ld32(tO + q * 32, orr);
@@ -352,9 +415,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
-            if (valid) p.lse[p.g.base(b, h, start, 1) + static_cast<long long>(row) * p.g.row_stride(1)] = lse_v;
+            if (valid) p.lse[p.g.base(e.b, e.h, e.start, 1) + static_cast<long long>(row) * p.g.row_stride(1)] = lse_v;
+        }
         }
     }
+#undef FOR_EACH_UNIT
 
     __syncwarp();  // reconverge the single-lane roles before the CTA barrier
     tc_fence_before();
@@ -367,7 +432,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (last == p.ctl.inject_skip_load) last -= C::kStages;
             if (last >= 0) drain_phase(bar(C::kBarFull + s), (last / C::kStages) & 1, p.ctl, abort_flag);
         }
-        drain_phase(bar(C::kBarQ), 0, p.ctl, abort_flag);
+        if (n_qload > 0) drain_phase(bar(C::kBarQ), (n_qload - 1) & 1, p.ctl, abort_flag);
     }
     if (warp == 9) {
         tc_fence_after();
@@ -389,7 +454,8 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.g.H, a.g.B, p.n_pairs);
+    const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
+    const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
     attn_fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
     return cudaGetLastError();
 }

@@ -16,6 +16,7 @@ struct FwdLaunch {
     float *lse;
     float scale;
     int causal;
+    int num_sms;  // persistent grid size
 };
 
 struct BwdLaunch {
