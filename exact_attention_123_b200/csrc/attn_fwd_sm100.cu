@@ -54,7 +54,14 @@ struct FwdCfg {
     static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
     static constexpr int kBoxes = D / 64;           // 128-byte-swizzle boxes per tile
     static constexpr int kStages = (D == 128) ? 4 : 8;
-    static constexpr int kThreads = 320;
+    // 3 warpgroups: two softmax groups, and one with the TMA producer, the MMA issuer
+    // and two idle warps (registers move by whole warpgroups).  Launched at 168
+    // registers per thread (the most 384 threads allow), the control group gives
+    // registers back and the softmax groups take them: 2*128*200 + 128*104 = 384*168.
+    static constexpr int kThreads = 384;
+    static constexpr int kLaunchRegs = 168, kRegsSoftmax = 200, kRegsControl = 104;
+    static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
+                  "register reallocation exceeds the launch pool");
     static constexpr int kTmemCols = 512;
     static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
     // barrier indices
@@ -115,7 +122,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D>;
@@ -157,7 +164,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t tmem = *tmem_holder;
     int n_issued = 0;  // producer: ring loads 0 .. n_issued-1 were started (except a skipped one)
     int n_qload = 0;   // producer: Q pairs whose load was started
-
+    if (warp >= 8) {
+    setmaxnreg_dec<C::kRegsControl>();
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -282,7 +290,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
         }
+    }
     } else {
+        setmaxnreg_inc<C::kRegsSoftmax>();
         // ------------------------------------------------------------ softmax warps
         const int t = warp >> 2, q4 = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
@@ -354,21 +364,31 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
 
-            // ---- probabilities (bf16) into TMEM over S, and the row sum
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- probabilities (bf16) into TMEM over S, and the row sum.  Column pairs
+            // go through the packed f32x2 pipe: one instruction scales and shifts both
+            // scores, one adds both probabilities to a pair of running sums.
+            const uint64_t c2x2 = f2_pack(c2, c2), negm2 = f2_pack(-m_use, -m_use);
+            uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * c], c2, -m_use));
-                    const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * c + 1], c2, -m_use));
-                    ps[c & 3] += p0 + p1;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[half * 64 + 2 * c], s[half * 64 + 2 * c + 1]), c2x2, negm2), x0, x1);
+                    const float p0 = ex2_approx(x0);
+                    const float p1 = ex2_approx(x1);
+                    ps2[c & 1] = f2_add(ps2[c & 1], f2_pack(p0, p1));
                     pk[c] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(tS + half * 32, pk);
             }
-            l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(ps2[0], a0, a1);
+                f2_unpack(ps2[1], b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             // Lazy correction of O_t, after the scores are dead (fewer live registers)
             // but before P_t is published: PV_t(j) is issued only after the arrive.
             if (warp_rescale && j > 0) {
@@ -454,6 +474,15 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // The in-kernel register reallocation assumes the launch register count it was
+    // sized for; with fewer, an increase could never be satisfied, so refuse.
+    static const cudaError_t regs_ok = [] {
+        cudaFuncAttributes fa{};
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D>);
+        if (r != cudaSuccess) return r;
+        return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
+    }();
+    if (regs_ok != cudaSuccess) return regs_ok;
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
     const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
     attn_fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
