@@ -29,12 +29,12 @@ def lib():
         ip = ctypes.POINTER(ctypes.c_int)
         up = ctypes.POINTER(ctypes.c_ubyte)
         L.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_int, ctypes.c_double, ctypes.c_int, ip, up, ip,
-                                      ctypes.c_int, ctypes.c_int]
+                                      ctypes.c_int, ctypes.c_double, ctypes.c_int, ip, up, up, ctypes.c_int,
+                                      ip, ctypes.c_int, ctypes.c_int]
         L.oracle_attn_fwd.restype = ctypes.c_int
         L.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                      ip, up, ip, ctypes.c_int, ctypes.c_int]
+                                      ip, up, up, ctypes.c_int, ip, ctypes.c_int, ctypes.c_int]
         L.oracle_attn_bwd.restype = ctypes.c_int
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
@@ -84,8 +84,12 @@ def default_threads() -> int:
     return max(1, os.cpu_count() or 1)
 
 
-def fwd(q, k, v, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nthreads=None, N=None):
+def fwd(q, k, v, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nthreads=None, N=None,
+        block_mask=None, block=128):
     """Forward pass.  q,k,v: dense [B,H,N,d] or packed [total,H,d] (with cu_seqlens).
+
+    block_mask (dense layout only): [H, ceil(N/block), ceil(N/block)] uint8 tile mask;
+    a zero leaves the whole (query tile, key tile) pair out.
 
     Returns (o, lse) as float64 arrays with the input's layout ([B,H,N] / [total,H] for lse).
     Rows of slices not listed in ``slices`` (b*H+h indices) are left as NaN.
@@ -103,9 +107,11 @@ def fwd(q, k, v, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nth
         lse = np.full((q.shape[0], H), np.nan)
     o = np.full(q.shape, np.nan)
     sl = _i32(slices)
+    bm = _u8(block_mask)
     rc = lib().oracle_attn_fwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
                                _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double), B, H, Nn, d,
                                float(scale), int(bool(causal)), _ptr(cu, ctypes.c_int), _ptr(kk, ctypes.c_ubyte),
+                               _ptr(bm, ctypes.c_ubyte), int(block),
                                _ptr(sl, ctypes.c_int), 0 if sl is None else len(sl),
                                int(nthreads or default_threads()))
     if rc != 0:
@@ -113,7 +119,8 @@ def fwd(q, k, v, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nth
     return o, lse
 
 
-def bwd(q, k, v, dout, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nthreads=None, N=None):
+def bwd(q, k, v, dout, scale, causal, cu_seqlens=None, key_keep=None, slices=None, nthreads=None, N=None,
+        block_mask=None, block=128):
     """Backward pass from the softmax Jacobian.  Returns (dq, dk, dv) float64."""
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     cu = _i32(cu_seqlens)
@@ -128,10 +135,12 @@ def bwd(q, k, v, dout, scale, causal, cu_seqlens=None, key_keep=None, slices=Non
     dk = np.full(q.shape, np.nan)
     dv = np.full(q.shape, np.nan)
     sl = _i32(slices)
+    bm = _u8(block_mask)
     rc = lib().oracle_attn_bwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
                                _ptr(dout, ctypes.c_double), _ptr(dq, ctypes.c_double),
                                _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), B, H, Nn, d,
                                float(scale), int(bool(causal)), _ptr(cu, ctypes.c_int), _ptr(kk, ctypes.c_ubyte),
+                               _ptr(bm, ctypes.c_ubyte), int(block),
                                _ptr(sl, ctypes.c_int), 0 if sl is None else len(sl),
                                int(nthreads or default_threads()))
     if rc != 0:

@@ -10,6 +10,7 @@
  *
  *   S_ij = scale * sum_c Q_ic K_jc                      full n x n matrix
  *   S_ij = -inf  unless (not causal or j <= i) and key_keep[j] != 0
+ *                 and block_mask[h][i / block][j / block] != 0
  *   m_i  = max_j S_ij
  *   if m_i == -inf :  O_i = 0,  lse_i = -inf,  P_i. = 0   (fully masked row)
  *   else           :  P_ij = exp(S_ij - m_i) / sum_k exp(S_ik - m_i)
@@ -31,13 +32,20 @@
  *   dQ = scale * dS K,   dK = scale * dS^T Q.
  * The backward recomputes its own float64 P; it never uses a GPU result.
  *
+ * The tile mask is the block-sparse variant named in "4.5 注意力优化实战：从
+ * PyTorch到CUDA的完整流程", §7.1 (Block-Sparse FlashAttention: compute only the
+ * important pairs, combining a sparsity pattern with the tiling): a pair of a
+ * block-row query tile and a block-column key tile either takes part or is left
+ * out as a whole; left-out pairs behave exactly like masked scores.
+ *
  * Layouts (element offsets, double precision arrays):
  *   dense   (cu_seqlens == NULL): Q,K,V,O,dO,dQ,dK,dV are [B,H,N,d]; lse is [B,H,N];
- *           key_keep (optional) is [B,N].
+ *           key_keep (optional) is [B,N]; block_mask (optional) is [H, nb, nb] with
+ *           nb = ceil(N / block), shared by all batch entries.
  *   packed  (cu_seqlens != NULL): tensors are token-major [total,H,d]; lse is
  *           [total,H]; key_keep (optional) is [total]; cu_seqlens has B+1
  *           entries and sequence b owns tokens cu_seqlens[b] .. cu_seqlens[b+1]-1.
- *           Causal indices are local to each sequence.
+ *           Causal indices are local to each sequence.  No block_mask.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -78,16 +86,20 @@ static int make_slice(int b, int h, int B, int H, int N, int d, const int *cu, s
     return 0;
 }
 
-/* Fill S (n x n, row-major) with masked scaled scores for one slice. */
+/* Fill S (n x n, row-major) with masked scaled scores for one slice.  tiles is
+ * this head's [nb x nb] tile mask (or NULL). */
 static void scores(const double *q, const double *k, const slice_t *s, int d, double scale,
-                   int causal, const unsigned char *keep, double *S, int nthreads)
+                   int causal, const unsigned char *keep, const unsigned char *tiles, int block,
+                   double *S, int nthreads)
 {
     const int n = s->n;
+    const int nb = (tiles != NULL) ? (n + block - 1) / block : 0;
 #pragma omp parallel for schedule(dynamic, 8) num_threads(nthreads)
     for (int i = 0; i < n; ++i) {
         const double *qi = q + s->base + (long)i * s->rstride;
         for (int j = 0; j < n; ++j) {
-            int allowed = (!causal || j <= i) && (keep == NULL || keep[s->kbase + j] != 0);
+            int allowed = (!causal || j <= i) && (keep == NULL || keep[s->kbase + j] != 0) &&
+                          (tiles == NULL || tiles[(long)(i / block) * nb + j / block] != 0);
             if (!allowed) {
                 S[(long)i * n + j] = -INFINITY;
                 continue;
@@ -154,9 +166,11 @@ static int run_slices(int B, int H, const int *slices, int n_slices, int **out, 
 int oracle_attn_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
                     int B, int H, int N, int d, double scale, int is_causal,
                     const int *cu_seqlens, const unsigned char *key_keep,
+                    const unsigned char *block_mask, int block,
                     const int *slices, int n_slices, int nthreads)
 {
     if (!q || !k || !v || !o || B <= 0 || H <= 0 || N < 0 || d <= 0) return -1;
+    if (block_mask && (cu_seqlens || block <= 0)) return -1;
     if (nthreads <= 0) nthreads = 1;
     int *sel = NULL, cnt = 0;
     if (run_slices(B, H, slices, n_slices, &sel, &cnt)) return -1;
@@ -169,7 +183,9 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v, double *o
         if (n == 0) continue;
         double *S = (double *)malloc(sizeof(double) * (size_t)n * (size_t)n);
         if (!S) { rc = -1; break; }
-        scores(q, k, &s, d, scale, is_causal, key_keep, S, nthreads);
+        const long nb = block_mask ? (N + block - 1) / block : 0;
+        scores(q, k, &s, d, scale, is_causal, key_keep, block_mask ? block_mask + (long)h * nb * nb : NULL,
+               block, S, nthreads);
         softmax_rows(S, &s, lse, nthreads);
 #pragma omp parallel for schedule(static) num_threads(nthreads)
         for (int i = 0; i < n; ++i) {
@@ -197,10 +213,12 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
                     double *dq, double *dk, double *dv,
                     int B, int H, int N, int d, double scale, int is_causal,
                     const int *cu_seqlens, const unsigned char *key_keep,
+                    const unsigned char *block_mask, int block,
                     const int *slices, int n_slices, int nthreads)
 {
     if (!q || !k || !v || !dout || !dq || !dk || !dv || B <= 0 || H <= 0 || N < 0 || d <= 0)
         return -1;
+    if (block_mask && (cu_seqlens || block <= 0)) return -1;
     if (nthreads <= 0) nthreads = 1;
     int *sel = NULL, cnt = 0;
     if (run_slices(B, H, slices, n_slices, &sel, &cnt)) return -1;
@@ -214,7 +232,9 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
         double *P = (double *)malloc(sizeof(double) * (size_t)n * (size_t)n);
         double *dS = (double *)malloc(sizeof(double) * (size_t)n * (size_t)n);
         if (!P || !dS) { free(P); free(dS); rc = -1; break; }
-        scores(q, k, &s, d, scale, is_causal, key_keep, P, nthreads);
+        const long nb = block_mask ? (N + block - 1) / block : 0;
+        scores(q, k, &s, d, scale, is_causal, key_keep, block_mask ? block_mask + (long)h * nb * nb : NULL,
+               block, P, nthreads);
         softmax_rows(P, &s, NULL, nthreads);
 
         /* dP_ij = dO_i . V_j ; dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik) */

@@ -33,13 +33,15 @@ def _num(s):
     return float(Fraction(s))
 
 
-def brute_fwd(q, k, v, scale, causal, keep=None):
-    """Triple-loop forward on one head (lists of lists), naive exp(s)/sum exp(s)."""
+def brute_fwd(q, k, v, scale, causal, keep=None, allow=None):
+    """Triple-loop forward on one head (lists of lists), naive exp(s)/sum exp(s).
+    allow(i, j), if given, is an extra pair predicate (a tile mask)."""
     n, d = len(q), len(q[0])
     o = [[0.0] * d for _ in range(n)]
     lse = [0.0] * n
     for i in range(n):
-        vis = [j for j in range(n) if (not causal or j <= i) and (keep is None or keep[j])]
+        vis = [j for j in range(n) if (not causal or j <= i) and (keep is None or keep[j])
+               and (allow is None or allow(i, j))]
         if not vis:
             lse[i] = -math.inf
             continue
@@ -53,14 +55,15 @@ def brute_fwd(q, k, v, scale, causal, keep=None):
     return o, lse
 
 
-def brute_bwd(q, k, v, do, scale, causal, keep=None):
+def brute_bwd(q, k, v, do, scale, causal, keep=None, allow=None):
     """Backward by the chain rule through each row's softmax, written with loops."""
     n, d = len(q), len(q[0])
     dq = [[0.0] * d for _ in range(n)]
     dk = [[0.0] * d for _ in range(n)]
     dv = [[0.0] * d for _ in range(n)]
     for i in range(n):
-        vis = [j for j in range(n) if (not causal or j <= i) and (keep is None or keep[j])]
+        vis = [j for j in range(n) if (not causal or j <= i) and (keep is None or keep[j])
+               and (allow is None or allow(i, j))]
         if not vis:
             continue
         s = {j: scale * sum(q[i][c] * k[j][c] for c in range(d)) for j in vis}
@@ -379,3 +382,126 @@ def test_slice_selection_leaves_others_untouched():
     assert np.all(np.isnan(o[0])) and np.all(np.isnan(o[1, 0]))
     full, _ = oracle.fwd(inp.q, inp.k, inp.v, 0.5, True)
     np.testing.assert_array_equal(o[1, 1], full[1, 1])
+
+
+# ---------------------------------------------------------------- block-sparse tile mask
+# "4.5 注意力优化实战：从PyTorch到CUDA的完整流程", §7.1 (Block-Sparse FlashAttention):
+# a (query tile, key tile) pair either takes part as a whole or is left out.
+
+def _tile_mask(H, nb, seed, density=0.6):
+    return (np.random.default_rng(seed).random((H, nb, nb)) < density).astype(np.uint8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_brute_force(causal):
+    B, H, N, d, blk = 1, 2, 11, 5, 3          # 4 x 4 tiles, the last one ragged
+    q, k, v, do = (rnd((B, H, N, d), s) for s in (41, 42, 43, 44))
+    nb = -(-N // blk)
+    bm = _tile_mask(H, nb, 45)
+    bm[0, 1, :] = 0                           # head 0: query rows 3-5 see no key at all
+    scale = 0.53
+    o, lse = oracle.fwd(q, k, v, scale, causal, block_mask=bm, block=blk)
+    dq, dk, dv = oracle.bwd(q, k, v, do, scale, causal, block_mask=bm, block=blk)
+    for h in range(H):
+        allow = lambda i, j, h=h: bool(bm[h, i // blk, j // blk])
+        bo, bl = brute_fwd(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), scale, causal, None, allow)
+        np.testing.assert_allclose(o[0, h], bo, rtol=0, atol=1e-12)
+        for got, want in zip(lse[0, h], bl):
+            assert (got == want == -math.inf) or abs(got - want) < 1e-12
+        gq, gk, gv = brute_bwd(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), do[0, h].tolist(),
+                               scale, causal, None, allow)
+        np.testing.assert_allclose(dq[0, h], gq, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dk[0, h], gk, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dv[0, h], gv, rtol=0, atol=1e-12)
+    # the emptied query tile: O = 0, lse = -inf, no gradient flows through it
+    assert np.all(o[0, 0, 3:6] == 0) and np.all(lse[0, 0, 3:6] == -math.inf)
+    assert np.all(dq[0, 0, 3:6] == 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_of_key_columns_equals_key_keep(causal):
+    # leaving out key tile 2 for every query tile is the per-key mask of its keys
+    B, H, N, d, blk = 2, 3, 20, 4, 4
+    q, k, v, do = (rnd((B, H, N, d), s) for s in (51, 52, 53, 54))
+    nb = N // blk
+    bm = np.ones((H, nb, nb), np.uint8)
+    bm[:, :, 2] = 0
+    keep = np.ones((B, N), np.uint8)
+    keep[:, 8:12] = 0
+    a = oracle.fwd(q, k, v, 0.4, causal, block_mask=bm, block=blk)
+    b = oracle.fwd(q, k, v, 0.4, causal, key_keep=keep)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    ga = oracle.bwd(q, k, v, do, 0.4, causal, block_mask=bm, block=blk)
+    gb = oracle.bwd(q, k, v, do, 0.4, causal, key_keep=keep)
+    for x, y in zip(ga, gb):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_block_mask_single_tile_is_attention_on_that_tile():
+    # query tile i with only key tile j left in is plain attention of those rows on
+    # those keys (computed without any mask, on the cut-out tiles)
+    B, H, N, d, blk = 1, 2, 12, 3, 4
+    q, k, v = (rnd((B, H, N, d), s) for s in (61, 62, 63))
+    bm = np.zeros((H, 3, 3), np.uint8)
+    pick = {0: 2, 1: 0, 2: 1}                 # query tile -> its only key tile (same for both heads)
+    for i, j in pick.items():
+        bm[:, i, j] = 1
+    o, lse = oracle.fwd(q, k, v, 0.7, False, block_mask=bm, block=blk)
+    for i, j in pick.items():
+        qs = q[:, :, i * blk:(i + 1) * blk]
+        ks, vs = k[:, :, j * blk:(j + 1) * blk], v[:, :, j * blk:(j + 1) * blk]
+        o2, l2 = oracle.fwd(qs, ks, vs, 0.7, False)
+        np.testing.assert_allclose(o[:, :, i * blk:(i + 1) * blk], o2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, i * blk:(i + 1) * blk], l2, rtol=0, atol=1e-13)
+
+
+def test_block_mask_lower_triangle_with_causal_is_causal():
+    B, H, N, d, blk = 1, 2, 10, 4, 3
+    q, k, v, do = (rnd((B, H, N, d), s) for s in (71, 72, 73, 74))
+    nb = -(-N // blk)
+    tri = np.tril(np.ones((nb, nb), np.uint8))[None].repeat(H, 0)
+    ones = np.ones((H, nb, nb), np.uint8)
+    for bm in (tri, ones):
+        a = oracle.fwd(q, k, v, 0.5, True, block_mask=bm, block=blk)
+        b = oracle.fwd(q, k, v, 0.5, True)
+        for x, y in zip(a, b):
+            np.testing.assert_array_equal(x, y)
+        ga = oracle.bwd(q, k, v, do, 0.5, True, block_mask=bm, block=blk)
+        gb = oracle.bwd(q, k, v, do, 0.5, True)
+        for x, y in zip(ga, gb):
+            np.testing.assert_array_equal(x, y)
+
+
+def test_block_mask_finite_differences():
+    B, H, N, d, blk = 1, 1, 8, 3, 2
+    q, k, v, G = (rnd((B, H, N, d), s) for s in (81, 82, 83, 84))
+    bm = _tile_mask(H, N // blk, 85)
+    bm[0, 2, :] = 0
+    bm[0, 0, 0] = 1
+    scale = 0.8
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.fwd(qq, kk, vv, scale, True, block_mask=bm, block=blk)
+        return float(np.sum(o * G))
+
+    dq, dk, dv = oracle.bwd(q, k, v, G, scale, True, block_mask=bm, block=blk)
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.max(np.abs(num - grad)) / max(1e-12, np.max(np.abs(grad)))
+        assert err < 1e-6, (name, err)
+
+
+def test_block_mask_rejected_with_packed_layout():
+    q = np.zeros((8, 1, 4))
+    with pytest.raises(ValueError):
+        oracle.fwd(q, q, q, 1.0, False, cu_seqlens=[0, 3, 8], block_mask=np.ones((1, 1, 1), np.uint8), block=128)
