@@ -109,6 +109,22 @@ def padding_key_mask(lengths, seed: int, pad_frac: float = 0.02, extra_frac: flo
     return torch.cat(parts)
 
 
+def tile_mask(H: int, N: int, seed: int, density: float = 0.5, tile: int = 128,
+              empty_rows=(), empty_cols=()) -> torch.Tensor:
+    """uint8 ``[H, nb, nb]`` block-sparse tile mask, nb = ceil(N / tile): each
+    (query tile, key tile) pair kept with probability ``density``.  ``empty_rows`` /
+    ``empty_cols`` list (h, tile) pairs whose whole mask row / column is cleared
+    (a query tile that sees no key / a key tile that no query reaches)."""
+    nb = -(-N // tile)
+    g = torch.Generator("cpu").manual_seed(seed)
+    m = (torch.rand((H, nb, nb), generator=g) < density).to(torch.uint8)
+    for h, i in empty_rows:
+        m[h, i, :] = 0
+    for h, j in empty_cols:
+        m[h, :, j] = 0
+    return m
+
+
 @dataclass
 class Inputs:
     q: torch.Tensor

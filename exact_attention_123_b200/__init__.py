@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp]
+    L.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
+    L.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, sz, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
@@ -68,7 +70,8 @@ def lib() -> ctypes.CDLL:
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
     for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen", "attn_bwd_phase",
-                 "attn_status", "attn_set_wait_limit_ms", "attn_debug_skip_load"):
+                 "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_status", "attn_set_wait_limit_ms",
+                 "attn_debug_skip_load"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -192,6 +195,49 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
                             B, H, N, d, float(scale), int(causal), None, _ptr(key_keep), _ptr(workspace),
                             workspace.numel(), _stream(stream))
         _check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_fwd_blocksparse(q, k, v, block_mask, o=None, lse=None, *, scale: Optional[float] = None,
+                         causal: bool = False, stream=None):
+    """Block-sparse forward (dense [B,H,N,d] layout).  block_mask: uint8 device tensor
+    [H, ceil(N/128), ceil(N/128)]; a zero leaves that (query tile, key tile) pair out.
+    Returns (o, lse)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, n)
+    _need(block_mask, torch.uint8, "block_mask")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    rc = lib().attn_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                    int(causal), _ptr(block_mask), _stream(stream))
+    _check(rc, "attn_fwd_blocksparse")
+    return o, lse
+
+
+def attn_bwd_blocksparse(q, k, v, o, lse, do, block_mask, dq=None, dk=None, dv=None, *,
+                         scale: Optional[float] = None, causal: bool = False,
+                         workspace: Optional[torch.Tensor] = None, stream=None):
+    """Block-sparse backward (dense layout, same block_mask as the forward).
+    Returns (dq, dk, dv)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    _need(block_mask, torch.uint8, "block_mask")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(q)
+    rc = lib().attn_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), B, H, N, d, float(scale), int(causal), _ptr(block_mask),
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "attn_bwd_blocksparse")
     return dq, dk, dv
 
 

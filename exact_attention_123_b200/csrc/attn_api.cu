@@ -110,8 +110,10 @@ int check_common(const Shape &s, float scale) {
     return ATTN_OK;
 }
 
-attn::Geom geom_of(const Shape &s, const uint8_t *key_keep) {
+attn::Geom geom_of(const Shape &s, const uint8_t *key_keep, const uint8_t *block_mask = nullptr) {
     attn::Geom g{};
+    g.block_mask = block_mask;
+    g.nbt = (s.N + 127) / 128;
     g.B = s.B;
     g.H = s.H;
     g.N = s.N;
@@ -131,7 +133,7 @@ attn::SyncCtl ctl_of(DeviceState *ds) {
 }
 
 int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, const Shape &s, float scale,
-             int is_causal, const uint8_t *key_keep, void *stream) {
+             int is_causal, const uint8_t *key_keep, void *stream, const uint8_t *block_mask = nullptr) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -142,7 +144,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     if (s.cu && s.total == 0) return ATTN_OK;  // nothing to do
     attn::FwdLaunch a{};
     if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s))) return rc;
-    a.g = geom_of(s, key_keep);
+    a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);
     a.o = o;
     a.lse = lse;
@@ -160,7 +162,8 @@ size_t bwd_ws_bytes(long long rows_x_heads, int /*d*/) {
 
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
              void *dq, void *dk, void *dv, const Shape &s, float scale, int is_causal, const uint8_t *key_keep,
-             void *workspace, size_t workspace_bytes, void *stream, int phases = 7) {
+             void *workspace, size_t workspace_bytes, void *stream, int phases = 7,
+             const uint8_t *block_mask = nullptr) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -178,7 +181,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
         (rc = map_for(&a.tm_do, dout, s)))
         return rc;
-    a.g = geom_of(s, key_keep);
+    a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);
     a.o = o;
     a.dout = dout;
@@ -220,6 +223,25 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
     if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
     Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
     return fwd_impl(q, k, v, o, lse, s, scale, is_causal, key_keep, stream);
+}
+
+int attn_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
+                         int d, float scale, int is_causal, const uint8_t *block_mask, void *stream) {
+    if (!block_mask) return ATTN_ERR_INVALID_ARG;
+    if (N > 64 * 128) return ATTN_ERR_UNSUPPORTED;  // the kernels hold a row of the mask in 64 bits
+    Shape s{B, H, N, d, 0, nullptr};
+    return fwd_impl(q, k, v, o, lse, s, scale, is_causal, nullptr, stream, block_mask);
+}
+
+int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                         const void *dout, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                         int is_causal, const uint8_t *block_mask, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    if (!block_mask) return ATTN_ERR_INVALID_ARG;
+    if (N > 64 * 128) return ATTN_ERR_UNSUPPORTED;
+    Shape s{B, H, N, d, 0, nullptr};
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, nullptr, workspace, workspace_bytes,
+                    stream, 7, block_mask);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -139,7 +139,7 @@ struct DkdvCfg {
     static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
 };
 
-template <int D>
+template <int D, bool SP>
 __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                                 const CUtensorMap &tm_v, const CUtensorMap &tm_do,
                                                 const BwdParams &p, uint8_t *smem_raw) {
@@ -155,9 +155,12 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
     const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
     const int BH = p.g.B * p.g.H;
     const int T = BH * p.n_tiles;
-    // work unit of rank r: key tile j (heaviest = 0), slice (b, h); false if empty
+    // work unit of rank r: key tile j (heaviest = 0), slice (b, h); false if empty.
+    // qs: the query tiles that attend key tile j (all from i0 on without a tile
+    // mask); nq of them, walked in increasing order.
     struct Tile {
         int b, h, j, start, len, kv0, i0, nq;
+        TileSet qs;
     };
     auto tile_at = [&](int r, Tile &t) -> bool {
         t.j = r / BH;
@@ -168,7 +171,8 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
         t.kv0 = t.j * 128;
         if (t.kv0 >= t.len) return false;
         t.i0 = p.causal ? t.j : 0;
-        t.nq = (t.len + 127) / 128 - t.i0;
+        t.qs = col_tiles<SP>(p.g, t.h, t.j, t.i0, (t.len + 127) / 128);
+        t.nq = t.qs.count();
         return true;
     };
 
@@ -201,7 +205,7 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
             const int r = snake_rank(k, cta, G);
             if (r >= T) break;
             Tile t;
-            if (!tile_at(r, t)) continue;
+            if (!tile_at(r, t) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
             const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
             const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
             // K_j, V_j once the previous tile's last S^T / dP^T have read theirs
@@ -216,12 +220,12 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
                 }
             }
             ++n_kv;
-            for (int it = 0; it < t.nq; ++it) {
+            for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
                 const int gi = n_q, st = gi % C::kStages;
                 ok = __all_sync(0xffffffffu,
                                 wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1, p.ctl, abort_flag));
                 if (!ok) break;
-                const int q0 = (t.i0 + it) * 128;
+                const int q0 = i * 128;
                 float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -282,7 +286,7 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
                 const int r = snake_rank(k, cta, G);
                 if (r >= T) break;
                 Tile t;
-                if (!tile_at(r, t)) continue;
+                if (!tile_at(r, t) || t.nq == 0) continue;
                 ok = wait_phase(bar(C::kBarKVFull), n_t & 1, p.ctl, abort_flag);
                 if (ok) ok = wait_q(gbase);
                 if (!ok) break;
@@ -355,9 +359,20 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
             Tile t;
             if (!tile_at(r, t)) continue;
             const int key = t.kv0 + kr;
+            if (t.nq == 0) {
+                // The tile mask leaves key tile j no query tile: dV = dK = 0 for its keys
+                // (warps 0-3 write dV, 4-7 dK), and nothing was computed.
+                if (key < t.len) {
+                    uint4 *dst = reinterpret_cast<uint4 *>((hf == 0 ? p.dv : p.dk) + p.g.base(t.b, t.h, t.start, D) +
+                                                           static_cast<long long>(key) * p.g.row_stride(D));
+#pragma unroll 1
+                    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
             bool kvalid = key < t.len;
             if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(t.b, t.start) + key] != 0;
-            for (int it = 0; it < t.nq; ++it) {
+            for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
                 const int gi = gbase + it, st = gi % C::kStages;
                 ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull), gi & 1, p.ctl, abort_flag));
                 if (ok)
@@ -372,7 +387,7 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
                 tmem_wait_ld();
                 // P^T = 2^(S^T c - lse2), 0 where the query precedes the key (causal),
                 // for keys outside the sequence or padded, and for rows past the end.
-                const int qb = (t.i0 + it) * 128 + hf * 64;  // first query column of this warp
+                const int qb = i * 128 + hf * 64;  // first query column of this warp
                 int lim = p.causal ? key - qb : 0;            // columns c < lim are masked
                 if (!kvalid) lim = 64;
                 float pf[64];
@@ -512,7 +527,7 @@ struct DqCfg {
     static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
 };
 
-template <int D>
+template <int D, bool SP>
 __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                               const CUtensorMap &tm_v, const CUtensorMap &tm_do,
                                               const BwdParams &p, uint8_t *smem_raw) {
@@ -530,9 +545,12 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
     const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
     const int BH = p.g.B * p.g.H;
     const int T = BH * p.n_tiles;
-    // work unit of rank r: query tile qt (heaviest = the last), slice (b, h); false if empty
+    // work unit of rank r: query tile qt (heaviest = the last), slice (b, h); false if empty.
+    // ks: the key tiles query tile qt attends (all of [0, reach) without a tile mask);
+    // nkv of them, walked in increasing order.
     struct Tile {
         int b, h, qt, start, len, q0, nkv;
+        TileSet ks;
     };
     auto tile_at = [&](int r, Tile &t) -> bool {
         const int k = r / BH;
@@ -544,7 +562,8 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
         t.q0 = t.qt * 128;
         if (t.q0 >= t.len) return false;
         const int nkv_all = (t.len + 127) / 128;
-        t.nkv = p.causal ? min(nkv_all, t.qt + 1) : nkv_all;
+        t.ks = row_tiles<SP>(p.g, t.h, t.qt, p.causal ? min(nkv_all, t.qt + 1) : nkv_all);
+        t.nkv = t.ks.count();
         return true;
     };
 
@@ -577,7 +596,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                 const int r = snake_rank(k, cta, G);
                 if (r >= T) break;
                 Tile t;
-                if (!tile_at(r, t)) continue;
+                if (!tile_at(r, t) || t.nkv == 0) continue;  // (nkv == 0: the math warps write zeros)
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
                 // Q_i, dO_i once the previous tile's last S / dP have read theirs
                 if (!wait_phase(bar(C::kBarQEmpty), (n_qt & 1) ^ 1, p.ctl, abort_flag)) break;
@@ -588,7 +607,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                     tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
                 }
                 ++n_qt;
-                for (int jt = 0; jt < t.nkv; ++jt) {
+                for (int jt = 0, j = t.ks.next(0); jt < t.nkv; ++jt, j = t.ks.next(j + 1)) {
                     const int gk = n_k, ks = gk % C::kKStages;
                     if (!wait_phase(bar(C::kBarKEmpty + ks), ((gk / C::kKStages) & 1) ^ 1, p.ctl, abort_flag)) {
                         ok = false;
@@ -597,7 +616,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                     mbar_arrive_expect_tx(bar(C::kBarKFull + ks), C::kTile);
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x)
-                        tma_load_3d(kslot(gk) + x * 16384, &tm_k, bar(C::kBarKFull + ks), x * 64, row0 + 128 * jt,
+                        tma_load_3d(kslot(gk) + x * 16384, &tm_k, bar(C::kBarKFull + ks), x * 64, row0 + 128 * j,
                                     slab);
                     ++n_k;
                     const int gv = n_v, vs = gv % C::kVStages;
@@ -608,7 +627,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                     mbar_arrive_expect_tx(bar(C::kBarVFull + vs), C::kTile);
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x)
-                        tma_load_3d(vslot(gv) + x * 16384, &tm_v, bar(C::kBarVFull + vs), x * 64, row0 + 128 * jt,
+                        tma_load_3d(vslot(gv) + x * 16384, &tm_v, bar(C::kBarVFull + vs), x * 64, row0 + 128 * j,
                                     slab);
                     ++n_v;
                 }
@@ -649,7 +668,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                 const int r = snake_rank(k, cta, G);
                 if (r >= T) break;
                 Tile t;
-                if (!tile_at(r, t)) continue;
+                if (!tile_at(r, t) || t.nkv == 0) continue;
                 ok = wait_phase(bar(C::kBarQFull), n_t & 1, p.ctl, abort_flag);
                 if (ok) ok = wait_k(gbase);
                 if (!ok) break;
@@ -716,11 +735,22 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
             Tile t;
             if (!tile_at(r, t)) continue;
             const int qrow = t.q0 + q4 * 32 + lane;  // query row within the slice
+            if (t.nkv == 0) {
+                // The tile mask leaves query tile qt no key tile: dQ = 0 for its rows
+                // (warp w writes columns (w/4)*d/2 ..), and nothing was computed.
+                if (qrow < t.len) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.dq + p.g.base(t.b, t.h, t.start, D) +
+                                                           static_cast<long long>(qrow) * p.g.row_stride(D) + hf * (D / 2));
+#pragma unroll 1
+                    for (int v = 0; v < D / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
             const long long lidx = p.g.base(t.b, t.h, t.start, 1) + static_cast<long long>(qrow) * p.g.row_stride(1);
             const float l2 = (qrow < t.len) ? p.lse2[lidx] : INFINITY;  // rows past the sequence: P = 0
             const float dd = (qrow < t.len) ? p.dvec[lidx] : 0.f;
             const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(t.b, t.start) : nullptr;
-            for (int jt = 0; jt < t.nkv; ++jt) {
+            for (int jt = 0, j = t.ks.next(0); jt < t.nkv; ++jt, j = t.ks.next(j + 1)) {
                 const int gj = gbase + jt;
                 ok = __all_sync(0xffffffffu,
                                 wait_phase(bar(C::kBarSFull + (gj & 1)), (gj >> 1) & 1, p.ctl, abort_flag));
@@ -738,7 +768,7 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                 tc_fence_before();
                 mbar_arrive(bar(C::kBarDPFree));
                 // masking: keys outside the sequence, above the diagonal, or padded
-                const int kb = jt * 128 + hf * 64;  // first key of this warp's columns
+                const int kb = j * 128 + hf * 64;  // first key of this warp's columns
                 int limit = t.len - kb;
                 if (p.causal) limit = min(limit, qrow - kb + 1);
                 uint32_t kmask[2] = {0xffffffffu, 0xffffffffu};
@@ -826,26 +856,26 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
 
 // ============================================================================ kernels
 // Persistent: one CTA per SM walks its share of the work units.
-template <int D>
+template <int D, bool SP>
 __global__ void __launch_bounds__(320, 1)
 attn_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                            const __grid_constant__ BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
-    dkdv_persistent<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
+    dkdv_persistent<D, SP>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
 }
 
-template <int D>
+template <int D, bool SP>
 __global__ void __launch_bounds__(320, 1)
 attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
-    dq_persistent<D>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
+    dq_persistent<D, SP>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
 }
 
 // ============================================================================ launch
-template <int D>
+template <int D, bool SP>
 static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
     const int nseq = a.g.B;
     const int *cu = a.g.varlen ? a.g.cu_seqlens : nullptr;
@@ -876,25 +906,26 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
     const dim3 g(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
     cudaError_t e;
     if (a.phases & 2) {
-        e = cudaFuncSetAttribute(attn_bwd_dkdv_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(attn_bwd_dkdv_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  DkdvCfg<D>::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attn_bwd_dkdv_sm100_kernel<D><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+        attn_bwd_dkdv_sm100_kernel<D, SP><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.phases & 4) {
-        e = cudaFuncSetAttribute(attn_bwd_dq_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(attn_bwd_dq_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  DqCfg<D>::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attn_bwd_dq_sm100_kernel<D><<<g, 320, DqCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+        attn_bwd_dq_sm100_kernel<D, SP><<<g, 320, DqCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream) {
-    if (a.g.d == 128) return launch_bwd_d<128>(a, stream);
-    return launch_bwd_d<64>(a, stream);
+    const bool sp = a.g.block_mask != nullptr;
+    if (a.g.d == 128) return sp ? launch_bwd_d<128, true>(a, stream) : launch_bwd_d<128, false>(a, stream);
+    return sp ? launch_bwd_d<64, true>(a, stream) : launch_bwd_d<64, false>(a, stream);
 }
 
 }  // namespace attn

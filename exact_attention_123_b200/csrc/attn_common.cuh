@@ -24,6 +24,8 @@ struct Geom {
     int varlen;                 // 0 dense, 1 packed (cu_seqlens)
     const int32_t *cu_seqlens;  // device, B+1 entries (packed only)
     const uint8_t *key_keep;    // device, nullable
+    const uint8_t *block_mask;  // device [H][nbt][nbt] tile mask (dense layout, nbt <= 64), nullable
+    int nbt;                    // tiles per side of block_mask
     __device__ __forceinline__ void slice(int b, int &start, int &len) const {
         if (varlen) {
             start = cu_seqlens[b];
@@ -49,6 +51,51 @@ struct Geom {
     __device__ __forceinline__ int tma_row0(int start) const { return varlen ? start : 0; }
     __device__ __forceinline__ int tma_slab(int b, int h) const { return varlen ? h : b * H + h; }
 };
+
+// A set of 128-row tiles [lo, hi) of one unit's sweep, all of them or (with a tile
+// mask) those whose bit is set.  next(x) is the first member >= x, or hi.
+struct TileSet {
+    uint64_t bits;  // members (only with a tile mask; then hi <= 64)
+    int lo, hi;
+    bool sparse;
+    __device__ __forceinline__ int next(int x) const {
+        if (!sparse) return x < hi ? max(x, lo) : hi;
+        if (x >= hi) return hi;
+        const uint64_t m = bits & (~0ull << x);
+        return m ? min(__ffsll(static_cast<long long>(m)) - 1, hi) : hi;
+    }
+    __device__ __forceinline__ bool has(int x) const {
+        return x >= lo && x < hi && (!sparse || ((bits >> x) & 1ull));
+    }
+    __device__ __forceinline__ int count() const { return sparse ? __popcll(bits) : max(0, hi - lo); }
+    __device__ __forceinline__ int last() const {  // largest member, or lo - 1 if none
+        if (!sparse) return hi - 1;
+        return bits ? 63 - __clzll(static_cast<long long>(bits)) : lo - 1;
+    }
+};
+
+// Key tiles [0, n) of query tile qt that head h attends (SP: a tile mask is given;
+// a compile-time flag, so that kernels without one carry none of this).
+template <bool SP>
+__device__ __forceinline__ TileSet row_tiles(const Geom &g, int h, int qt, int n) {
+    TileSet t{0ull, 0, n, SP};
+    if (SP) {
+        const uint8_t *r = g.block_mask + (static_cast<long long>(h) * g.nbt + qt) * g.nbt;
+        for (int j = 0; j < n; ++j) t.bits |= static_cast<uint64_t>(r[j] != 0) << j;
+    }
+    return t;
+}
+
+// Query tiles [lo, n) that attend key tile kt of head h.
+template <bool SP>
+__device__ __forceinline__ TileSet col_tiles(const Geom &g, int h, int kt, int lo, int n) {
+    TileSet t{0ull, lo, n, SP};
+    if (SP) {
+        const uint8_t *c = g.block_mask + static_cast<long long>(h) * g.nbt * g.nbt + kt;
+        for (int i = lo; i < n; ++i) t.bits |= static_cast<uint64_t>(c[static_cast<long long>(i) * g.nbt] != 0) << i;
+    }
+    return t;
+}
 
 struct SyncCtl {
     int *status;             // device status word (first error wins)

@@ -96,11 +96,22 @@ struct FwdParams {
 // CTA c of G takes ranks c, 2G-1-c, 2G+c, 4G-1-c, ... (snake order).
 struct FwdUnit {
     int b, h, start, len, m0;
-    int nkv0, nkv1;  // key tiles seen by Q0 and Q1 (0: the tile lies past the sequence)
+    int nkv0, nkv1;  // key tiles in reach of Q0 and Q1 (0: the tile lies past the sequence)
+    TileSet ts0, ts1;  // the key tiles Q0 / Q1 actually attend (all of them without a tile mask)
     __device__ __forceinline__ int nkv(int t) const { return t ? nkv1 : nkv0; }
     __device__ __forceinline__ int nkv_max() const { return max(nkv0, nkv1); }
+    __device__ __forceinline__ bool live(int t, int j) const { return t ? ts1.has(j) : ts0.has(j); }
+    // first key tile >= x that either tile attends (nkv_max() if none): the key/value
+    // tiles the unit loads.  A set with no member >= x returns its own end, which
+    // must not win the minimum.
+    __device__ __forceinline__ int unext(int x) const {
+        const int a = ts0.next(x), b = ts1.next(x);
+        const int r = min(a < ts0.hi ? a : INT_MAX, b < ts1.hi ? b : INT_MAX);
+        return r == INT_MAX ? nkv_max() : r;
+    }
 };
 
+template <bool SP>
 __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int G, FwdUnit &u) {
     const int BH = p.g.B * p.g.H;
     const int r = k * G + ((k & 1) ? (G - 1 - cta) : cta);
@@ -115,13 +126,16 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int
     const int r1 = u.m0 + 128;
     u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
     u.nkv1 = (r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
+    u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
+    u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
     return true;
 }
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-template <int D>
+// SP: a tile mask (block-sparse attention) is given.
+template <int D, bool SP>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
@@ -143,7 +157,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #define FOR_EACH_UNIT(u)                                                        \
     for (int k_ = 0; k_ * G < n_ranks; ++k_)                                     \
         if (FwdUnit u; (k_ * G + ((k_ & 1) ? (G - 1 - cta) : cta)) < n_ranks && \
-                       fwd_unit(p, k_, cta, G, u))
+                       fwd_unit<SP>(p, k_, cta, G, u))
 
     if (warp == 9) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -176,6 +190,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             int idx = 0;  // ring position, continuing across units
             FOR_EACH_UNIT(u) {
                 if (!ok) break;
+                const int nkv_max = u.nkv_max();
+                if (u.unext(0) >= nkv_max) continue;  // no tile pair to compute (tile mask)
                 const int row0 = p.g.tma_row0(u.start), slab = p.g.tma_slab(u.b, u.h);
                 // Q0/Q1 once the previous unit's last S products have read theirs
                 if (!wait_phase(bar(C::kBarQEmpty), (n_qload & 1) ^ 1, p.ctl, abort_flag)) break;
@@ -187,8 +203,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
                                     row0 + u.m0 + 128 * t, slab);
                 ++n_qload;
-                const int nkv_max = u.nkv_max();
-                for (int j = 0; j < nkv_max && ok; ++j) {
+                for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
 #pragma unroll
                     for (int kv = 0; kv < 2; ++kv, ++idx) {
                         const int s = idx % C::kStages;
@@ -214,9 +229,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
-            auto issue_S = [&](int t, int base, int j) {
+            // S_t from the K tile at ring position kpos
+            auto issue_S = [&](int t, int kpos) {
                 const uint32_t qs = sbase + t * C::kTileBytes;
-                const uint32_t ks = slot((base + 2 * j) % C::kStages);
+                const uint32_t ks = slot(kpos % C::kStages);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -225,12 +241,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 tc_commit(bar(C::kBarS + t));
             };
-            auto issue_PV = [&](int t, int base, int j) {
-                const uint32_t vs = slot((base + 2 * j + 1) % C::kStages);
+            // O_t (+)= P_t V, V at ring position vpos; `acc` false for the tile's first P V
+            auto issue_PV = [&](int t, int vpos, bool acc) {
+                const uint32_t vs = slot(vpos % C::kStages);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sw128_desc(vs + kk * 2048, 16384, 1024), idPV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                           (acc || kk > 0) ? 1u : 0u);
             };
             bool ok = true;
             int base = 0;          // ring position of the unit's K_0
@@ -239,51 +256,62 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             int go[2] = {0, 0};    // units in which tile t was active
             FOR_EACH_UNIT(u) {
                 if (!ok) break;
-                const int nkv_max = u.nkv_max();
+                const int hi = u.nkv_max();
+                int j = u.unext(0);  // the unit's key tiles are j, unext(j + 1), ... (< hi)
+                if (j >= hi) continue;  // no tile pair to compute (tile mask)
+                int pos = base;         // ring position of K_j (V_j follows it)
                 ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
-                if (ok) ok = wait_phase(bar(C::kBarFull + base % C::kStages), (base / C::kStages) & 1, p.ctl, abort_flag);
+                if (ok) ok = wait_phase(bar(C::kBarFull + pos % C::kStages), (pos / C::kStages) & 1, p.ctl, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // S_t(0) may overwrite S_t / P_t: PV_t of the previous unit was issued
-                // earlier (in-order completion) after its softmax had read S_t.
+                // The unit's first S_t may overwrite S_t / P_t: PV_t of the previous unit
+                // was issued earlier (in-order completion) after its softmax had read S_t.
                 for (int t = 0; t < 2; ++t)
-                    if (u.nkv(t) > 0) issue_S(t, base, 0);
-                tc_commit(bar(C::kBarEmpty + base % C::kStages));
-                if (nkv_max == 1) tc_commit(bar(C::kBarQEmpty));
-                for (int j = 0; ok && j < nkv_max; ++j) {
-                    const int vidx = base + 2 * j + 1, kidx = base + 2 * j + 2;
-                    ok = wait_phase(bar(C::kBarFull + vidx % C::kStages), (vidx / C::kStages) & 1, p.ctl, abort_flag);
+                    if (u.live(t, j)) issue_S(t, pos);
+                tc_commit(bar(C::kBarEmpty + pos % C::kStages));
+                int nxt = u.unext(j + 1);
+                if (nxt >= hi) tc_commit(bar(C::kBarQEmpty));
+                bool started[2] = {false, false};
+                const int last[2] = {u.ts0.last(), u.ts1.last()};
+                while (ok) {
+                    ok = wait_phase(bar(C::kBarFull + (pos + 1) % C::kStages), ((pos + 1) / C::kStages) & 1, p.ctl,
+                                    abort_flag);
                     if (!ok) break;
                     bool k_next = false;
                     for (int t = 0; t < 2 && ok; ++t) {
-                        if (j < u.nkv(t)) {
+                        if (u.live(t, j)) {
                             ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
                             if (!ok) break;
                             ++gs[t];
                             tc_fence_after();
-                            issue_PV(t, base, j);
-                            if (j == u.nkv(t) - 1) tc_commit(bar(C::kBarO + t));
+                            issue_PV(t, pos + 1, started[t]);
+                            started[t] = true;
+                            if (j == last[t]) tc_commit(bar(C::kBarO + t));
                         }
-                        if (j + 1 < u.nkv(t)) {
+                        if (nxt < hi && u.live(t, nxt)) {
                             if (!k_next) {
-                                ok = wait_phase(bar(C::kBarFull + kidx % C::kStages), (kidx / C::kStages) & 1, p.ctl,
-                                                abort_flag);
+                                ok = wait_phase(bar(C::kBarFull + (pos + 2) % C::kStages), ((pos + 2) / C::kStages) & 1,
+                                                p.ctl, abort_flag);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_next = true;
                             }
-                            issue_S(t, base, j + 1);
+                            issue_S(t, pos + 2);
                         }
                     }
                     if (!ok) break;
-                    tc_commit(bar(C::kBarEmpty + vidx % C::kStages));
-                    if (k_next) tc_commit(bar(C::kBarEmpty + kidx % C::kStages));
-                    if (j + 2 == nkv_max) tc_commit(bar(C::kBarQEmpty));  // the unit's last S products
+                    tc_commit(bar(C::kBarEmpty + (pos + 1) % C::kStages));
+                    if (k_next) tc_commit(bar(C::kBarEmpty + (pos + 2) % C::kStages));
+                    pos += 2;
+                    if (nxt >= hi) break;
+                    j = nxt;
+                    nxt = u.unext(j + 1);
+                    if (nxt >= hi) tc_commit(bar(C::kBarQEmpty));  // the S products just issued were the unit's last
                 }
                 if (!ok) break;
-                base += 2 * nkv_max;
+                base = pos;
                 ++n_u;
-                for (int t = 0; t < 2; ++t) go[t] += (u.nkv(t) > 0);
+                for (int t = 0; t < 2; ++t) go[t] += started[t];
             }
             (void)go;
             // Every MMA issued above must have finished before TMEM / smem go away.
@@ -304,11 +332,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         int go = 0;  // units in which this tile was active
         FOR_EACH_UNIT(u) {
         if (!ok) break;
+        // only what this tile needs is kept from the unit (registers)
         const int len = u.len;
         const int row = u.m0 + 128 * t + q4 * 32 + lane;  // query row within the slice
+        const int nkv_t = u.nkv(t);
         const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(u.b, u.start) : nullptr;
         float m_used = -INFINITY, l = 0.f;
-        for (int j = 0; j < u.nkv(t); ++j, ++gs) {
+        const TileSet ts = t ? u.ts1 : u.ts0;  // the key tiles this tile attends
+        bool first_step = true;
+        for (int j = ts.next(0); j < ts.hi; j = ts.next(j + 1), ++gs) {
             ok = wait_phase(bar(C::kBarS + t), gs & 1, p.ctl, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -391,7 +423,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             // Lazy correction of O_t, after the scores are dead (fewer live registers)
             // but before P_t is published: PV_t(j) is issued only after the arrive.
-            if (warp_rescale && j > 0) {
+            if (warp_rescale && !first_step) {
 #pragma unroll
                 for (int q = 0; q < D / 32; ++q) {
                     uint32_t orr[32];
@@ -405,19 +437,34 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(C::kBarP + t));
+            first_step = false;
         }
 
         // ---- epilogue: O / l in bf16, lse in natural log.  The next unit's PV_t(0),
         // which overwrites O_t, is issued only after this thread's next P_t arrive.
-        if (ok && u.nkv(t) > 0) ok = wait_phase(bar(C::kBarO + t), go & 1, p.ctl, abort_flag);
-        if (ok && u.nkv(t) > 0) {
+        if (ok && nkv_t > 0 && first_step) {
+            // The tile mask leaves this tile no key tile: O = 0 and lse = -inf, like any
+            // row that sees no key; nothing was computed for it.
+            FwdUnit e;
+            fwd_unit<SP>(p, k_, cta, G, e);
+            if (row < len) {
+                const long long r = static_cast<long long>(row);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.o + p.g.base(e.b, e.h, e.start, D) + r * p.g.row_stride(D));
+#pragma unroll 1
+                for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                p.lse[p.g.base(e.b, e.h, e.start, 1) + r * p.g.row_stride(1)] = -INFINITY;
+            }
+            continue;
+        }
+        if (ok && nkv_t > 0) ok = wait_phase(bar(C::kBarO + t), go & 1, p.ctl, abort_flag);
+        if (ok && nkv_t > 0) {
             ++go;
             tc_fence_after();
             const bool valid = row < len;
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
-            fwd_unit(p, k_, cta, G, e);
+            fwd_unit<SP>(p, k_, cta, G, e);
             __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
 #pragma unroll 1  // (unrolled, the 128-wide key loop above runs out of registers)
             for (int q = 0; q < D / 32; ++q) {
@@ -460,7 +507,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
 }
 
-template <int D>
+template <int D, bool SP>
 static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     using C = FwdCfg<D>;
     FwdParams p{};
@@ -471,27 +518,28 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.causal = a.causal;
     p.n_pairs = (a.g.N + 255) / 256;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The in-kernel register reallocation assumes the launch register count it was
     // sized for; with fewer, an increase could never be satisfied, so refuse.
     static const cudaError_t regs_ok = [] {
         cudaFuncAttributes fa{};
-        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D>);
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP>);
         if (r != cudaSuccess) return r;
         return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
     }();
     if (regs_ok != cudaSuccess) return regs_ok;
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
     const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-    attn_fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    attn_fwd_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {
-    if (a.g.d == 128) return launch_fwd_d<128>(a, stream);
-    return launch_fwd_d<64>(a, stream);
+    const bool sp = a.g.block_mask != nullptr;
+    if (a.g.d == 128) return sp ? launch_fwd_d<128, true>(a, stream) : launch_fwd_d<128, false>(a, stream);
+    return sp ? launch_fwd_d<64, true>(a, stream) : launch_fwd_d<64, false>(a, stream);
 }
 
 }  // namespace attn

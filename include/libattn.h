@@ -166,6 +166,33 @@ ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void 
                             int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Block-sparse attention ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", §7.1,
+ * Block-Sparse FlashAttention: only the important pairs are computed, a sparsity
+ * pattern combined with the tiling).  Dense layout only, as attn_fwd / attn_bwd
+ * with cu_seqlens = NULL and no key mask, plus:
+ *   block_mask  device array of uint8 [H][nb][nb], nb = ceil(N / 128), shared by
+ *               the B sequences.  Entry [h][i][j] == 0 leaves the pair (query rows
+ *               128 i .. 128 i + 127, keys 128 j .. 128 j + 127) of head h out:
+ *               those key/value tiles are never loaded or multiplied for those
+ *               rows and their scores count as -inf.  Any nonzero value keeps the
+ *               pair.  It combines with is_causal (a score must pass both).  A query
+ *               row left with no key at all gets O = 0, lse = -inf and contributes
+ *               no gradient; key rows that no query reaches get dK = dV = 0.
+ *               Must not be NULL (ATTN_ERR_INVALID_ARG).  Owned by the caller, read
+ *               during the call's kernels only.
+ *   N <= 8192 (nb <= 64), else ATTN_ERR_UNSUPPORTED.
+ * The backward takes the same workspace as attn_bwd (attn_bwd_workspace_bytes).
+ */
+ATTN_API int attn_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  int B, int H, int N, int d, float scale, int is_causal,
+                                  const uint8_t *block_mask, void *stream);
+ATTN_API int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
+                                  const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                                  int B, int H, int N, int d, float scale, int is_causal,
+                                  const uint8_t *block_mask, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -27,7 +27,8 @@ def L():
 def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
-              "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen"):
+              "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen", "attn_fwd_blocksparse",
+              "attn_bwd_blocksparse"):
         assert n in names
 
 
@@ -90,6 +91,23 @@ def test_host_argument_errors(L):
     assert L.attn_bwd(*args, vp(FAKE), 16, None) == ea.ATTN_ERR_WORKSPACE
     need = ea.attn_bwd_workspace_bytes(1, 1, 16, 64)
     assert L.attn_bwd(*args, vp(FAKE + 16), need, None) == ea.ATTN_ERR_MISALIGNED
+
+
+def test_blocksparse_host_argument_errors(L):
+    import exact_attention_123_b200 as ea
+    vp = ctypes.c_void_p
+    f = ctypes.c_float(0.1)
+    # the tile mask is required, and a mask row must fit the kernels' 64 bits (N <= 8192)
+    assert L.attn_fwd_blocksparse(*[vp(FAKE)] * 5, 1, 1, 256, 64, f, 0, None, None) == ea.ATTN_ERR_INVALID_ARG
+    assert L.attn_fwd_blocksparse(*[vp(FAKE)] * 5, 1, 1, 8193, 64, f, 0, vp(FAKE), None) == ea.ATTN_ERR_UNSUPPORTED
+    assert L.attn_fwd_blocksparse(*[vp(FAKE)] * 5, 1, 1, 256, 96, f, 0, vp(FAKE), None) == ea.ATTN_ERR_UNSUPPORTED
+    need = ea.attn_bwd_workspace_bytes(1, 1, 256, 64)
+    args = [vp(FAKE)] * 9 + [1, 1, 256, 64, f, 0]
+    assert L.attn_bwd_blocksparse(*args, None, vp(FAKE), need, None) == ea.ATTN_ERR_INVALID_ARG
+    args[11] = 8320
+    assert L.attn_bwd_blocksparse(*args, vp(FAKE), vp(FAKE), need, None) == ea.ATTN_ERR_UNSUPPORTED
+    args[11] = 256
+    assert L.attn_bwd_blocksparse(*args, vp(FAKE), None, 0, None) == ea.ATTN_ERR_WORKSPACE
 
 
 def test_wait_limit_and_fault_hook_setters(L):
