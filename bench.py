@@ -302,6 +302,45 @@ def run_ours(args):
     if st != ea.ATTN_OK:
         raise RuntimeError(f"end-to-end steps reported status {st}")
 
+    # ---- block-sparse variant: the same workload with half of the (query tile, key
+    # tile) pairs left out by a seeded per-head tile mask; timed after the headline
+    # steps, L2 flushed before each call.  FLOPs are those of the pairs computed
+    # (causal convention: a diagonal pair counts half, as in the dense count).
+    bsp = None
+    if not args.no_blocksparse and ws == 1:
+        from attn_inputs import tile_mask
+        nbt = (N + 127) // 128
+        bm = tile_mask(H, N, SEED + 7, 0.5)
+        tri = torch.tril(torch.ones(nbt, nbt, dtype=torch.uint8))
+        live = bm & tri if CAUSAL else bm
+        diag = torch.eye(nbt, dtype=torch.uint8)
+        pair_units = float(live.sum().item()) - (0.5 * float((live & diag).sum().item()) if CAUSAL else 0.0)
+        fl_fwd = B * pair_units * 4.0 * 128 * 128 * D
+        bmd = bm.to(dev)
+        for _ in range(3):
+            ea.attn_fwd_blocksparse(q, k, v, bmd, o, lse, **kw)
+            ea.attn_bwd_blocksparse(q, k, v, o, lse, do, bmd, dq, dk, dv, workspace=wsbuf, **kw)
+        n_bs = 20
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bs)]
+        for e in ev:
+            flush.zero_()
+            e[0].record(stream)
+            ea.attn_fwd_blocksparse(q, k, v, bmd, o, lse, **kw)
+            e[1].record(stream)
+            ea.attn_bwd_blocksparse(q, k, v, o, lse, do, bmd, dq, dk, dv, workspace=wsbuf, **kw)
+            e[2].record(stream)
+        torch.cuda.synchronize(dev)
+        st = ea.attn_status(stream)
+        if st != ea.ATTN_OK:
+            raise RuntimeError(f"block-sparse steps reported status {st}")
+        f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        dense_units = nbt * (nbt + 1) / 2 - nbt / 2 if CAUSAL else nbt * nbt
+        bsp = {"tile_density": 0.5, "tile_mask_seed": SEED + 7, "pairs_computed_frac_of_dense": pair_units / (H * dense_units),
+               "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": fl_fwd / (f_ms * 1e-3) / 1e12,
+               "bwd_tflops": 2.5 * fl_fwd / (b_ms * 1e-3) / 1e12,
+               "note": "attn_fwd_blocksparse / attn_bwd_blocksparse on the bench workload; FLOPs of the computed tile pairs"}
+
     step_flops = flops_fwd() + flops_bwd()
     value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12
     e2e_value = step_flops * e2e_n * ws / (float(e2e_ms.item()) * 1e-3) / 1e12
@@ -356,6 +395,7 @@ def run_ours(args):
         "clocks": clk.summary(),
         "wall_s_timed_region": wall,
         "cpu_baseline": cpu,
+        "blocksparse": bsp,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -370,6 +410,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-heads", type=int, default=4, help="(b,h) slices in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
