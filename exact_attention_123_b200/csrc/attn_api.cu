@@ -71,18 +71,23 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // 3-D map (col, row, slab) with a 128-byte swizzle; box = one 128-byte column group
 // (64 bf16 or 32 fp32 elements) x box_rows rows x 1.  Strides are in elements.
+// 3-D map (column, row, slab).  Loads use 64-column (128-byte) boxes with the
+// 128-byte swizzle; the backward's output stores use 32 x 32 boxes with the 64-byte
+// swizzle (box_cols = 32).
 int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long slabs, long long row_stride,
-             long long slab_stride, int box_rows, bool fp32 = false) {
+             long long slab_stride, int box_rows, bool fp32 = false, int box_cols = 0) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return ATTN_ERR_CUDA;
     const cuuint64_t esz = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * esz, static_cast<cuuint64_t>(slab_stride) * esz};
-    cuuint32_t box[3] = {fp32 ? 32u : 64u, static_cast<cuuint32_t>(box_rows), 1};
+    if (box_cols == 0) box_cols = fp32 ? 32 : 64;
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle swz = (box_cols * esz == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUresult r = enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -92,10 +97,12 @@ struct Shape {
     const int32_t *cu;
 };
 
-int map_for(CUtensorMap *m, const void *base, const Shape &s, int box_rows = 128, bool fp32 = false) {
-    if (s.cu) return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d, box_rows, fp32);
+int map_for(CUtensorMap *m, const void *base, const Shape &s, int box_rows = 128, bool fp32 = false,
+            int box_cols = 0) {
+    if (s.cu)
+        return make_map(m, base, s.d, s.total, s.H, static_cast<long long>(s.H) * s.d, s.d, box_rows, fp32, box_cols);
     return make_map(m, base, s.d, s.N, static_cast<long long>(s.B) * s.H, s.d, static_cast<long long>(s.N) * s.d,
-                    box_rows, fp32);
+                    box_rows, fp32, box_cols);
 }
 
 int check_common(const Shape &s, float scale) {
@@ -143,7 +150,9 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     if ((rc = device_state(&ds))) return rc;
     if (s.cu && s.total == 0) return ATTN_OK;  // nothing to do
     attn::FwdLaunch a{};
-    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s))) return rc;
+    if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
+        (rc = map_for(&a.tm_o_st, o, s, 32, false, 32)))
+        return rc;
     a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);
     a.o = o;
@@ -179,7 +188,8 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     if (s.cu && s.total == 0) return ATTN_OK;
     attn::BwdLaunch a{};
     if ((rc = map_for(&a.tm_q, q, s)) || (rc = map_for(&a.tm_k, k, s)) || (rc = map_for(&a.tm_v, v, s)) ||
-        (rc = map_for(&a.tm_do, dout, s)))
+        (rc = map_for(&a.tm_do, dout, s)) || (rc = map_for(&a.tm_dk_st, dk, s, 32, false, 32)) ||
+        (rc = map_for(&a.tm_dv_st, dv, s, 32, false, 32)))
         return rc;
     a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);

@@ -48,26 +48,41 @@ namespace attn {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ============================================================================ preprocess
-// One row of d elements per (d/8) threads.  Rows are in the lse layout order,
-// which is also the row order of the flat [rows, d] view of O and dO.
+// One row of d elements per (d/8) threads (16 bytes of O and of dO each); a CTA
+// covers kPreRows consecutive rows in kPreRows / (256 / (d/8)) passes whose loads
+// are all issued before any is used, so that each thread keeps several loads in
+// flight (the kernel is HBM-bound).  Rows are in the lse layout order, which is
+// also the row order of the flat [rows, d] view of O and dO.
+constexpr int kPrePasses = 4;
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *__restrict__ o,
                                                           const __nv_bfloat16 *__restrict__ dout,
                                                           const float *__restrict__ lse, float *__restrict__ dvec,
                                                           float *__restrict__ lse2, long long rows,
                                                           const int32_t *cu_seqlens, int nseq, int H) {
-    constexpr int TPR = D / 8;  // threads per row
+    constexpr int TPR = D / 8;          // threads per row
+    constexpr int RPP = 256 / TPR;      // rows per pass
     long long limit = rows;
     if (cu_seqlens) limit = min(rows, static_cast<long long>(cu_seqlens[nseq]) * H);
-    const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const long long row = gt / TPR;
-    const int part = static_cast<int>(gt % TPR);
-    const bool active = row < limit;
-    float acc = 0.f;
-    if (active) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(o + row * D + part * 8);
-        const uint4 g = *reinterpret_cast<const uint4 *>(dout + row * D + part * 8);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    const int part = threadIdx.x % TPR;
+    const long long row0 = static_cast<long long>(blockIdx.x) * (RPP * kPrePasses) + threadIdx.x / TPR;
+    uint4 a[kPrePasses], g[kPrePasses];
+#pragma unroll
+    for (int u = 0; u < kPrePasses; ++u) {
+        const long long row = row0 + u * RPP;
+        if (row < limit) {
+            a[u] = *reinterpret_cast<const uint4 *>(o + row * D + part * 8);
+            g[u] = *reinterpret_cast<const uint4 *>(dout + row * D + part * 8);
+        } else {
+            a[u] = make_uint4(0u, 0u, 0u, 0u);
+            g[u] = a[u];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kPrePasses; ++u) {
+        const long long row = row0 + u * RPP;
+        const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, gw[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
+        float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 x = unpack_bf16x2(aw[e]);
@@ -75,13 +90,13 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *
             acc = fmaf(x.x, y.x, acc);
             acc = fmaf(x.y, y.y, acc);
         }
-    }
 #pragma unroll
-    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (active && part == 0) {
-        dvec[row] = acc;
-        const float L = lse[row];
-        lse2[row] = (L == -INFINITY) ? INFINITY : L * kLog2e;
+        for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (row < limit && part == 0) {
+            dvec[row] = acc;
+            const float L = lse[row];
+            lse2[row] = (L == -INFINITY) ? INFINITY : L * kLog2e;
+        }
     }
 }
 
@@ -142,6 +157,7 @@ struct DkdvCfg {
 template <int D, bool SP>
 __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                                 const CUtensorMap &tm_v, const CUtensorMap &tm_do,
+                                                const CUtensorMap &tm_dk_st, const CUtensorMap &tm_dv_st,
                                                 const BwdParams &p, uint8_t *smem_raw) {
     using C = DkdvCfg<D>;
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -454,6 +470,12 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
             const float mul = is_dv ? 1.f : p.scale;
             const uint32_t col = is_dv ? C::kColDV : C::kColDK;
             const uint32_t stage = sbase + C::kOffStage + warp * 2048;
+            // A full 32-row block goes out by TMA store from the stage (its layout is
+            // the 64-byte swizzle of a 32 x 32 box), so the warp does not wait for the
+            // global writes; a block reaching past the sequence's end (which a packed
+            // layout could not clip) is written row by row.
+            const bool by_tma = t.len - key_w0 >= 32;
+            const CUtensorMap *tm_out = is_dv ? &tm_dv_st : &tm_dk_st;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t rr[32];
@@ -467,11 +489,29 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     pk[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
-                warp_store_rows32(stage, pk, out0 + c0, p.g.row_stride(D), t.len - key_w0, lane);
+                if (by_tma) {
+                    if (lane == 0) bulk_wait_read0();  // the previous store has read the stage
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        st_shared_v4(stage + lane * 64 + (((c ^ (lane >> 1)) & 3) << 4), pk[4 * c], pk[4 * c + 1],
+                                     pk[4 * c + 2], pk[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(tm_out, stage, c0, p.g.tma_row0(t.start) + key_w0, p.g.tma_slab(t.b, t.h));
+                        bulk_commit();
+                    }
+                } else {
+                    if (lane == 0) bulk_wait_read0();
+                    __syncwarp();
+                    warp_store_rows32(stage, pk, out0 + c0, p.g.row_stride(D), t.len - key_w0, lane);
+                }
             }
             gbase += t.nq;
             ++n_t;
         }
+        if (lane == 0) bulk_wait0();  // this warp's output stores are complete
     }
 
     __syncwarp();
@@ -860,9 +900,10 @@ template <int D, bool SP>
 __global__ void __launch_bounds__(320, 1)
 attn_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                           const __grid_constant__ CUtensorMap tm_dk_st, const __grid_constant__ CUtensorMap tm_dv_st,
                            const __grid_constant__ BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
-    dkdv_persistent<D, SP>(tm_q, tm_k, tm_v, tm_do, p, smem_raw);
+    dkdv_persistent<D, SP>(tm_q, tm_k, tm_v, tm_do, tm_dk_st, tm_dv_st, p, smem_raw);
 }
 
 template <int D, bool SP>
@@ -892,8 +933,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
     p.causal = a.causal;
     p.n_tiles = (a.g.N + 127) / 128;
     if (a.phases & 1) {
-        const long long threads = a.rows_total * (D / 8);
-        const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+        const long long rows_per_cta = (256 / (D / 8)) * kPrePasses;
+        const unsigned blocks = static_cast<unsigned>((a.rows_total + rows_per_cta - 1) / rows_per_cta);
         attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(a.o),
                                                            static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.dvec,
                                                            a.lse2, a.rows_total, cu, nseq, a.g.H);
@@ -909,7 +950,8 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
         e = cudaFuncSetAttribute(attn_bwd_dkdv_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  DkdvCfg<D>::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attn_bwd_dkdv_sm100_kernel<D, SP><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+        attn_bwd_dkdv_sm100_kernel<D, SP><<<g, 320, DkdvCfg<D>::kSmemBytes, stream>>>(
+            a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dk_st, a.tm_dv_st, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.phases & 4) {

@@ -75,7 +75,8 @@ struct FwdCfg {
     static constexpr int kBarQEmpty = 8 + 2 * kStages;       // the unit's last S products are done
     static constexpr int kNumBars = 9 + 2 * kStages;
     static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
-    static constexpr int kOffBar = kSmemTiles;
+    static constexpr int kOffStage = kSmemTiles;  // 8 softmax warps x 2 KB output stage
+    static constexpr int kOffBar = kOffStage + 8 * 2048;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
@@ -138,7 +139,8 @@ constexpr float kRescaleThreshold = 8.0f;
 template <int D, bool SP>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o_st,
+                      const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -466,6 +468,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
             fwd_unit<SP>(p, k_, cta, G, e);
             __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
+            // A warp's full 32-row block goes out by TMA store from its stage (laid out
+            // as the 64-byte swizzle of a 32 x 32 box), so the warp moves on to the next
+            // unit without waiting for the global writes; a block reaching past the
+            // sequence's end (which a packed layout could not clip) is stored row by row.
+            const int row_w0 = row - lane;
+            const bool by_tma = len - row_w0 >= 32;
+            const uint32_t stage = sbase + C::kOffStage + warp * 2048;
 #pragma unroll 1  // (unrolled, the 128-wide key loop above runs out of registers)
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t orr[32];
@@ -475,7 +484,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     pk[c] = pack_bf16x2(__uint_as_float(orr[2 * c]) * inv, __uint_as_float(orr[2 * c + 1]) * inv);
-                if (valid) {
+                if (by_tma) {
+                    if (lane == 0) bulk_wait_read0();  // the previous store has read the stage
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        st_shared_v4(stage + lane * 64 + (((c ^ (lane >> 1)) & 3) << 4), pk[4 * c], pk[4 * c + 1],
+                                     pk[4 * c + 2], pk[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&tm_o_st, stage, q * 32, p.g.tma_row0(e.start) + row_w0, p.g.tma_slab(e.b, e.h));
+                        bulk_commit();
+                    }
+                } else if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 32);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
@@ -485,6 +507,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (valid) p.lse[p.g.base(e.b, e.h, e.start, 1) + static_cast<long long>(row) * p.g.row_stride(1)] = lse_v;
         }
         }
+        if (lane == 0) bulk_wait0();  // this warp's output stores are complete
     }
 #undef FOR_EACH_UNIT
 
@@ -532,7 +555,7 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     if (regs_ok != cudaSuccess) return regs_ok;
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
     const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-    attn_fwd_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+    attn_fwd_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st, p);
     return cudaGetLastError();
 }
 

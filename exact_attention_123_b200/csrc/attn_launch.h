@@ -10,6 +10,7 @@ namespace attn {
 
 struct FwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v;  // 3-D bf16 maps, box {64, 128, 1}, 128-byte swizzle
+    CUtensorMap tm_o_st;           // O stores: box {32, 32, 1}, 64-byte swizzle
     Geom g;
     SyncCtl ctl;
     void *o;
@@ -21,6 +22,7 @@ struct FwdLaunch {
 
 struct BwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;  // same map shape as the forward (128-row boxes)
+    CUtensorMap tm_dk_st, tm_dv_st;       // dK, dV stores: 32 x 32 boxes, 64-byte swizzle
     Geom g;
     SyncCtl ctl;
     const void *o, *dout;

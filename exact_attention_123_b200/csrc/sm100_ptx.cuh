@@ -71,6 +71,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *m, uint32_t
         "r"(src), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// Tiled TMA store of a shared-memory box to global memory (bulk async-group; the
+// issuing thread waits with bulk_wait_read0 before reusing the box, bulk_wait0
+// before exiting).  Coordinates must be >= 0; rows past the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, uint32_t src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(m),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk group has finished reading its shared-memory source.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
