@@ -261,10 +261,8 @@ def run_ours(args):
     seg = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events]  # ms: fwd, pre, dK/dV, dQ
     step_ms = [sum(x) for x in seg]
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t.item())
+    from exact_attention_123_b200.sharding import max_over_ranks
+    total_ms_max = max_over_ranks(total_ms, device=dev)  # the job is as slow as its slowest rank
 
     # ---- end to end through the public API with host buffers
     pin = {n: x.cpu().pin_memory() for n, x in (("q", q), ("k", k), ("v", v), ("do", do))}
@@ -295,9 +293,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
     st = ea.attn_status(stream)
     if st != ea.ATTN_OK:
         raise RuntimeError(f"end-to-end steps reported status {st}")
@@ -343,7 +339,7 @@ def run_ours(args):
 
     step_flops = flops_fwd() + flops_bwd()
     value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12
-    e2e_value = step_flops * e2e_n * ws / (float(e2e_ms.item()) * 1e-3) / 1e12
+    e2e_value = step_flops * e2e_n * ws / (e2e_ms * 1e-3) / 1e12
 
     peaks, peak_src = measured_peaks()
     peak = float(peaks["bf16_tflops"])
