@@ -792,54 +792,58 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
             const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(t.b, t.start) : nullptr;
             for (int jt = 0, j = t.ks.next(0); jt < t.nkv; ++jt, j = t.ks.next(j + 1)) {
                 const int gj = gbase + jt;
+                // P = 2^(S c - lse2) first: it needs only S, so the exponentials run
+                // while the tensor core is still computing dP
                 ok = __all_sync(0xffffffffu,
                                 wait_phase(bar(C::kBarSFull + (gj & 1)), (gj >> 1) & 1, p.ctl, abort_flag));
-                if (ok) ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), gj & 1, p.ctl, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t scol = (gj & 1) ? C::kColS1 : C::kColS0;
-                uint32_t sr[2][32], dr[2][32];
+                float pf[64];
+                {
+                    uint32_t sr[2][32];
 #pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    tmem_ld32(tmem + lane_off + scol + hf * 64 + x * 32, sr[x]);
-                    tmem_ld32(tmem + lane_off + C::kColDP + hf * 64 + x * 32, dr[x]);
+                    for (int x = 0; x < 2; ++x) tmem_ld32(tmem + lane_off + scol + hf * 64 + x * 32, sr[x]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2));
                 }
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(bar(C::kBarDPFree));
                 // masking: keys outside the sequence, above the diagonal, or padded
                 const int kb = j * 128 + hf * 64;  // first key of this warp's columns
                 int limit = t.len - kb;
                 if (p.causal) limit = min(limit, qrow - kb + 1);
-                uint32_t kmask[2] = {0xffffffffu, 0xffffffffu};
+                if (limit < 64) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c >= limit) pf[c] = 0.f;
+                }
                 if (keep != nullptr) {
 #pragma unroll
                     for (int x = 0; x < 2; ++x) {
                         const int c = x * 32 + lane;
-                        kmask[x] = __ballot_sync(0xffffffffu, (c < t.len - kb) && keep[kb + c] != 0);
+                        const uint32_t km = __ballot_sync(0xffffffffu, (c < t.len - kb) && keep[kb + c] != 0);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (!((km >> e) & 1u)) pf[x * 32 + e] = 0.f;
                     }
                 }
+                // dS = P o (dP - D), written over S as bf16
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), gj & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t dr[2][32];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) tmem_ld32(tmem + lane_off + C::kColDP + hf * 64 + x * 32, dr[x]);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarDPFree));
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    float pf[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) pf[c] = ex2_approx(fmaf(__uint_as_float(sr[x][c]), c2, -l2));
-                    const int lim_x = limit - 32 * x;  // columns c >= lim_x are masked
-                    if (lim_x < 32) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (c >= lim_x) pf[c] = 0.f;
-                    }
-                    if (keep != nullptr) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (!((kmask[x] >> c) & 1u)) pf[c] = 0.f;
-                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 32; c += 2)
-                        pk[c >> 1] = pack_bf16x2(pf[c] * (__uint_as_float(dr[x][c]) - dd),
-                                                 pf[c + 1] * (__uint_as_float(dr[x][c + 1]) - dd));
+                        pk[c >> 1] = pack_bf16x2(pf[x * 32 + c] * (__uint_as_float(dr[x][c]) - dd),
+                                                 pf[x * 32 + c + 1] * (__uint_as_float(dr[x][c + 1]) - dd));
                     tmem_st16(tmem + lane_off + scol + hf * 64 + x * 16, pk);
                 }
                 tmem_wait_st();
