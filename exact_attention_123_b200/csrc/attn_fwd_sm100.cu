@@ -255,7 +255,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             int base = 0;          // ring position of the unit's K_0
             int n_u = 0;           // units started
             int gs[2] = {0, 0};    // S_t products issued (all units): phase counters
-            int go[2] = {0, 0};    // units in which tile t was active
             FOR_EACH_UNIT(u) {
                 if (!ok) break;
                 const int hi = u.nkv_max();
@@ -313,9 +312,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (!ok) break;
                 base = pos;
                 ++n_u;
-                for (int t = 0; t < 2; ++t) go[t] += started[t];
             }
-            (void)go;
             // Every MMA issued above must have finished before TMEM / smem go away.
             tc_commit(bar(C::kBarDone));
             drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
