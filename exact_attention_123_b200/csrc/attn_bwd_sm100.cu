@@ -255,7 +255,7 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
                     vec[128 + u * 32 + lane] = dd;
                 }
                 __syncwarp();
-                if (lane == 0) {
+                if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
                     mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x) {
@@ -521,7 +521,8 @@ __device__ __forceinline__ void dkdv_persistent(const CUtensorMap &tm_q, const C
         // After an abort, every copy the loader started must land before the CTA exits.
         if (n_kv > 0) drain_phase(bar(C::kBarKVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
-            drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+            if (gi != p.ctl.inject_skip_load)
+                drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
     }
     if (warp == 9) {
         tc_fence_after();
@@ -640,11 +641,14 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
                 // Q_i, dO_i once the previous tile's last S / dP have read theirs
                 if (!wait_phase(bar(C::kBarQEmpty), (n_qt & 1) ^ 1, p.ctl, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(C::kBarQFull), 2 * C::kTile);
+                if (n_qt != p.ctl.inject_skip_load) {  // (test hook: this tile never arrives)
+                    mbar_arrive_expect_tx(bar(C::kBarQFull), 2 * C::kTile);
 #pragma unroll
-                for (int x = 0; x < C::kBoxes; ++x) {
-                    tma_load_3d(sbase + C::kOffQ + x * 16384, &tm_q, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
-                    tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
+                    for (int x = 0; x < C::kBoxes; ++x) {
+                        tma_load_3d(sbase + C::kOffQ + x * 16384, &tm_q, bar(C::kBarQFull), x * 64, row0 + t.q0, slab);
+                        tma_load_3d(sbase + C::kOffDO + x * 16384, &tm_do, bar(C::kBarQFull), x * 64, row0 + t.q0,
+                                    slab);
+                    }
                 }
                 ++n_qt;
                 for (int jt = 0, j = t.ks.next(0); jt < t.nkv; ++jt, j = t.ks.next(j + 1)) {
@@ -886,7 +890,8 @@ __device__ __forceinline__ void dq_persistent(const CUtensorMap &tm_q, const CUt
     __syncthreads();
     if (warp == 8 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        if (n_qt > 0) drain_phase(bar(C::kBarQFull), (n_qt - 1) & 1, p.ctl, abort_flag);
+        if (n_qt > 0 && n_qt - 1 != p.ctl.inject_skip_load)
+            drain_phase(bar(C::kBarQFull), (n_qt - 1) & 1, p.ctl, abort_flag);
         for (int g = max(0, n_k - C::kKStages); g < n_k; ++g)
             drain_phase(bar(C::kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, p.ctl, abort_flag);
         for (int g = max(0, n_v - C::kVStages); g < n_v; ++g)

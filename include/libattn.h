@@ -243,10 +243,12 @@ ATTN_API const char *attn_strerror(int code);
 ATTN_API int attn_set_wait_limit_ms(int ms);
 
 /*
- * Test hook for the failure-detection path.  For later forward launches from this
- * process, the tile loader skips pipeline load number `load_index` (counting the
- * K and V tile loads of one CTA from 0), so that slot never fills and the
- * consumer's bounded wait expires; every kernel then stops cleanly and
+ * Test hook for the failure-detection path.  For later launches from this
+ * process, each CTA's tile loader skips one pipeline load: in the forward the
+ * K/V stage load number `load_index` (counting the K and V tile loads of one CTA
+ * from 0), in the backward the query-side load (Q and dO of one query tile)
+ * number `load_index` of the dK/dV and of the dQ kernel.  That slot never fills,
+ * the consumer's bounded wait expires, every kernel stops cleanly and
  * attn_status() reports ATTN_ERR_TIMEOUT.  -1 (the default) disables it.
  * Returns the previous value.  Nothing faults: all waits are time-limited.
  */

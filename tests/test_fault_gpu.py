@@ -42,3 +42,27 @@ def test_expired_wait_reports_timeout_and_context_survives(ea, skip):
     ro, _ = oracle.fwd(inp.q, inp.k, inp.v, inp.scale, True)
     err = (o.double().cpu().numpy() - ro)
     assert abs(err).max() < 2e-2
+
+
+@pytest.mark.parametrize("skip", [0, 2])
+def test_backward_expired_wait_reports_timeout_and_context_survives(ea, skip):
+    # Both backward kernels skip their query-side load number `skip`; every CTA stops
+    # at the bounded wait, and the next call is correct.
+    inp = make_dense(1, 2, 640, 64, seed=7100, with_grad=True)
+    q, k, v, do = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.do.cuda()
+    o, lse = ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
+    assert ea.attn_status() == ea.ATTN_OK
+    prev_limit = ea.attn_set_wait_limit_ms(200)
+    ea.attn_debug_skip_load(skip)
+    try:
+        ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True)
+        assert ea.attn_status() == ea.ATTN_ERR_TIMEOUT
+    finally:
+        ea.attn_debug_skip_load(-1)
+        ea.attn_set_wait_limit_ms(prev_limit)
+    dq, dk, dv = ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True)
+    assert ea.attn_status() == ea.ATTN_OK
+    rq, rk, rv = oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, True)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert abs(got.double().cpu().numpy() - ref).max() < 5e-2
+
