@@ -174,3 +174,40 @@ def make_workload(name: str, **over) -> Inputs:
         return make_varlen(lengths, w.H, w.d, w.seed, w.causal, keep, over.get("with_grad", w.with_grad))
     return make_dense(w.B, w.H, w.N, w.d, w.seed, over.get("causal", w.causal), w.qk_sigma,
                       over.get("with_grad", w.with_grad))
+
+
+@dataclass
+class Fp8Inputs:
+    q8: torch.Tensor  # uint8 e4m3 codes [B, H, N, d]
+    k8: torch.Tensor
+    v8: torch.Tensor
+    q_scale: float    # per-tensor dequantisation factors: value = decode(code) * factor
+    k_scale: float
+    v_scale: float
+    B: int
+    H: int
+    N: int
+    d: int
+    scale: float
+    causal: bool
+
+
+def e4m3_codes(x: torch.Tensor):
+    """Per-tensor e4m3 quantisation of float32 draws, the way a caller prepares FP8
+    inputs: factor = amax / 448 (e4m3's largest finite value), codes = x / factor
+    rounded by torch's float8_e4m3fn conversion.  Returns (uint8 codes, factor)."""
+    amax = float(x.abs().max())
+    factor = amax / 448.0 if amax > 0 else 1.0
+    return (x / factor).to(torch.float8_e4m3fn).view(torch.uint8), factor
+
+
+def make_fp8(B, H, N, d, seed, causal=True, qk_sigma=1.0, scale: Optional[float] = None) -> Fp8Inputs:
+    """N(0, sigma^2) float32 draws for Q, K (sigma = qk_sigma) and V (sigma 1), in
+    that order, each quantised per tensor with ``e4m3_codes``."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) * qk_sigma
+    k = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) * qk_sigma
+    v = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
+    (q8, qs), (k8, ks), (v8, vs) = e4m3_codes(q), e4m3_codes(k), e4m3_codes(v)
+    return Fp8Inputs(q8, k8, v8, qs, ks, vs, B, H, N, d, scale if scale is not None else 1.0 / math.sqrt(d), causal)
+

@@ -91,6 +91,22 @@ int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// 3-D map over e4m3 bytes: `cols` bytes per row (contiguous), box {128, box_rows, 1}
+// with the 128-byte swizzle.
+int make_map_u8(CUtensorMap *m, const void *base, long long cols, long long rows, long long slabs,
+                long long row_stride, long long slab_stride, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return ATTN_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride), static_cast<cuuint64_t>(slab_stride)};
+    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 struct Shape {
     int B, H, N, d;
     long long total;  // packed token rows, or 0 for dense
@@ -161,6 +177,48 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     a.causal = is_causal ? 1 : 0;
     a.num_sms = ds->num_sms > 0 ? ds->num_sms : 1;
     return attn::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+long long fp8_vt_cols(int N) { return (static_cast<long long>(N) + 127) / 128 * 128; }
+
+int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
+                 float *lse, const Shape &s, float scale, int is_causal, void *workspace, size_t workspace_bytes,
+                 void *stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    int rc = check_common(s, scale);
+    if (rc) return rc;
+    for (float f : {q_scale, k_scale, v_scale})
+        if (!(f > 0.f) || !std::isfinite(f)) return ATTN_ERR_INVALID_ARG;
+    if (s.d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_MISALIGNED;
+    const long long np = fp8_vt_cols(s.N);
+    const size_t need = static_cast<size_t>(s.B) * s.H * s.d * np;
+    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
+    DeviceState *ds = nullptr;
+    if ((rc = device_state(&ds))) return rc;
+    attn::FwdLaunch a{};
+    const long long slabs = static_cast<long long>(s.B) * s.H;
+    if ((rc = make_map_u8(&a.tm_q, q, s.d, s.N, slabs, s.d, static_cast<long long>(s.N) * s.d, 128)) ||
+        (rc = make_map_u8(&a.tm_k, k, s.d, s.N, slabs, s.d, static_cast<long long>(s.N) * s.d, 128)) ||
+        (rc = make_map_u8(&a.tm_v, workspace, np, s.d, slabs, np, np * s.d, s.d)) ||
+        (rc = map_for(&a.tm_o_st, o, s, 32, false, 32)))
+        return rc;
+    a.g = geom_of(s, nullptr);
+    a.ctl = ctl_of(ds);
+    a.o = o;
+    a.lse = lse;
+    a.scale = scale;
+    a.causal = is_causal ? 1 : 0;
+    a.num_sms = ds->num_sms > 0 ? ds->num_sms : 1;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.v8 = v;
+    a.vt = workspace;
+    a.vt_cols = static_cast<int>(np);
+    return attn::launch_fwd_fp8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 size_t bwd_ws_bytes(long long rows_x_heads, int /*d*/) {
@@ -241,6 +299,19 @@ int attn_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, f
     if (N > 64 * 128) return ATTN_ERR_UNSUPPORTED;  // the kernels hold a row of the mask in 64 bits
     Shape s{B, H, N, d, 0, nullptr};
     return fwd_impl(q, k, v, o, lse, s, scale, is_causal, nullptr, stream, block_mask);
+}
+
+size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
+    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+    return static_cast<size_t>(B) * H * d * fp8_vt_cols(N);
+}
+
+int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
+                 float *lse, int B, int H, int N, int d, float scale, int is_causal, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    Shape s{B, H, N, d, 0, nullptr};
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, workspace, workspace_bytes,
+                        stream);
 }
 
 int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,

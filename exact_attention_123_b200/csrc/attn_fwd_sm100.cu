@@ -49,11 +49,17 @@
 
 namespace attn {
 
-template <int D>
+// F8: Q, K and V in e4m3 (the V tiles then come from a transposed copy, d rows x
+// 128 keys, so that both products take K-major operands), P rounded to e4m3 in
+// shared memory, fp32 accumulation.
+template <int D, bool F8 = false>
 struct FwdCfg {
-    static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
-    static constexpr int kBoxes = D / 64;           // 128-byte-swizzle boxes per tile
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kEsz = F8 ? 1 : 2;                // bytes per Q/K/V element
+    static constexpr int kTileBytes = 128 * D * kEsz;      // one 128-row tile (e4m3 V^T: d rows x 128 keys)
+    static constexpr int kBoxes = D * kEsz / 128;          // 128-byte-swizzle boxes per tile
+    static constexpr int kKSteps = D * kEsz / 32;          // 32-byte K steps of S = Q K^T
+    static constexpr int kStages = F8 ? 8 : (D == 128) ? 4 : 8;
+    static_assert(!F8 || D == 128, "the e4m3 path has 128-byte rows (d = 128)");
     // 3 warpgroups: two softmax groups, and one with the TMA producer, the MMA issuer
     // and two idle warps (registers move by whole warpgroups).  Launched at 168
     // registers per thread (the most 384 threads allow), the control group gives
@@ -75,7 +81,8 @@ struct FwdCfg {
     static constexpr int kBarQEmpty = 8 + 2 * kStages;       // the unit's last S products are done
     static constexpr int kNumBars = 9 + 2 * kStages;
     static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
-    static constexpr int kOffStage = kSmemTiles;  // 8 softmax warps x 2 KB output stage
+    static constexpr int kOffP = kSmemTiles;                   // e4m3 P_0, P_1: 128 x 128 bytes each
+    static constexpr int kOffStage = kOffP + (F8 ? 2 * 16384 : 0);  // 8 softmax warps x 2 KB output stage
     static constexpr int kOffBar = kOffStage + 8 * 2048;
     static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
@@ -87,7 +94,8 @@ struct FwdParams {
     SyncCtl ctl;
     __nv_bfloat16 *o;
     float *lse;
-    float scale_log2;  // scale * log2(e)
+    float scale_log2;  // scale * log2(e) (e4m3: times the Q and K dequantisation scales)
+    float o_scale;     // 1, or the V dequantisation scale (e4m3)
     int causal;
     int n_pairs;       // 256-row query blocks per slice
 };
@@ -135,13 +143,14 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-// SP: a tile mask (block-sparse attention) is given.
-template <int D, bool SP>
+// SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs (tm_v then maps
+// the transposed V).
+template <int D, bool SP, bool F8>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o_st,
                       const __grid_constant__ FwdParams p) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
@@ -202,7 +211,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int t = 0; t < 2; ++t)
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x)
-                        tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * 64,
+                        tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * (128 / C::kEsz),
                                     row0 + u.m0 + 128 * t, slab);
                 ++n_qload;
                 for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
@@ -215,10 +224,17 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                         if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
                         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
+                        if constexpr (F8) {
+                            if (kv)  // V^T: columns are keys, rows the d features
+                                tma_load_3d(slot(s), &tm_v, bar(C::kBarFull + s), 128 * j, 0, slab);
+                            else
+                                tma_load_3d(slot(s), &tm_k, bar(C::kBarFull + s), 0, row0 + 128 * j, slab);
+                        } else {
 #pragma unroll
-                        for (int x = 0; x < C::kBoxes; ++x)
-                            tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
-                                        row0 + 128 * j, slab);
+                            for (int x = 0; x < C::kBoxes; ++x)
+                                tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
+                                            row0 + 128 * j, slab);
+                        }
                         n_issued = idx + 1;
                     }
                 }
@@ -227,8 +243,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
             // S_t from the K tile at ring position kpos
@@ -236,20 +252,33 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint32_t qs = sbase + t * C::kTileBytes;
                 const uint32_t ks = slot(kpos % C::kStages);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024), idS,
-                           kk > 0);
+                    if constexpr (F8)
+                        mma_ss_f8(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024),
+                                  idS, kk > 0);
+                    else
+                        mma_ss(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024), idS,
+                               kk > 0);
                 }
                 tc_commit(bar(C::kBarS + t));
             };
             // O_t (+)= P_t V, V at ring position vpos; `acc` false for the tile's first P V
             auto issue_PV = [&](int t, int vpos, bool acc) {
                 const uint32_t vs = slot(vpos % C::kStages);
+                if constexpr (F8) {
+                    // A = P_t (shared memory, 128 queries x 128 keys), B = V^T (d x 128 keys)
+                    const uint32_t ps = sbase + C::kOffP + t * 16384;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sw128_desc(vs + kk * 2048, 16384, 1024), idPV,
-                           (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss_f8(tmem + colO[t], sw128_desc(ps + kk * 32, 16, 1024), sw128_desc(vs + kk * 32, 16, 1024),
+                                  idPV, (acc || kk > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sw128_desc(vs + kk * 2048, 16384, 1024), idPV,
+                               (acc || kk > 0) ? 1u : 0u);
+                }
             };
             bool ok = true;
             int base = 0;          // ring position of the unit's K_0
@@ -410,9 +439,25 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float p0 = ex2_approx(x0);
                     const float p1 = ex2_approx(x1);
                     ps2[c & 1] = f2_add(ps2[c & 1], f2_pack(p0, p1));
-                    pk[c] = pack_bf16x2(p0, p1);
+                    if constexpr (F8) {
+                        const uint32_t h2 = pack_e4m3x2(p0, p1);
+                        pk[c >> 1] = (c & 1) ? (pk[c >> 1] | (h2 << 16)) : h2;
+                    } else {
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
                 }
-                tmem_st32(tS + half * 32, pk);
+                if constexpr (F8) {
+                    // this row's 64 keys as 4 chunks of 16 bytes, at the 128-byte-swizzle
+                    // positions of a K-major tile (chunk c of row r at r*128 + ((c ^ r%8) * 16))
+                    const int r = q4 * 32 + lane;
+                    const uint32_t prow = sbase + C::kOffP + t * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        st_shared_v4(prow + ((((half * 4 + cc) ^ (r & 7)) & 7) << 4), pk[4 * cc], pk[4 * cc + 1],
+                                     pk[4 * cc + 2], pk[4 * cc + 3]);
+                } else {
+                    tmem_st32(tS + half * 32, pk);
+                }
             }
             {
                 float a0, a1, b0, b1;
@@ -434,6 +479,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
             tmem_wait_st();
+            if constexpr (F8) fence_proxy_async_smem();  // P_t is read by the tensor core (async proxy)
             tc_fence_before();
             mbar_arrive(bar(C::kBarP + t));
             first_step = false;
@@ -460,7 +506,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ++go;
             tc_fence_after();
             const bool valid = row < len;
-            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const float inv = (l > 0.f) ? p.o_scale / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
             fwd_unit<SP>(p, k_, cta, G, e);
@@ -527,33 +573,79 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
 }
 
-template <int D, bool SP>
+template <int D, bool SP, bool F8 = false>
 static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F8>;
     FwdParams p{};
     p.g = a.g;
     p.ctl = a.ctl;
     p.o = static_cast<__nv_bfloat16 *>(a.o);
     p.lse = a.lse;
     p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.o_scale = 1.f;
+    if constexpr (F8) {
+        p.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * a.q_scale * a.k_scale * 1.4426950408889634);
+        p.o_scale = a.v_scale;
+    }
     p.causal = a.causal;
     p.n_pairs = (a.g.N + 255) / 256;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The in-kernel register reallocation assumes the launch register count it was
     // sized for; with fewer, an increase could never be satisfied, so refuse.
     static const cudaError_t regs_ok = [] {
         cudaFuncAttributes fa{};
-        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP>);
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP, F8>);
         if (r != cudaSuccess) return r;
         return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
     }();
     if (regs_ok != cudaSuccess) return regs_ok;
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
     const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-    attn_fwd_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st, p);
+    attn_fwd_sm100_kernel<D, SP, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st, p);
     return cudaGetLastError();
+}
+
+// V (e4m3, [slab][N][D]) -> V^T ([slab][D][np], np = N rounded up to 128; the
+// columns from N on are zero).  One CTA per (slab, 128-key tile).
+template <int D>
+__global__ void __launch_bounds__(256) attn_fp8_vt_kernel(const uint8_t *__restrict__ v, uint8_t *__restrict__ vt,
+                                                          int N, int np) {
+    __shared__ __align__(16) uint8_t tile[128][D + 16];
+    const long long slab = blockIdx.x;
+    const int kt = blockIdx.y;
+    const uint8_t *src = v + slab * N * D;
+    for (int i = threadIdx.x; i < 128 * (D / 16); i += 256) {
+        const int r = i / (D / 16), c = i % (D / 16);
+        const int key = kt * 128 + r;
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (key < N) x = *reinterpret_cast<const uint4 *>(src + static_cast<long long>(key) * D + c * 16);
+        *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = x;
+    }
+    __syncthreads();
+    uint8_t *dst = vt + slab * D * np + kt * 128;
+    for (int i = threadIdx.x; i < D * 8; i += 256) {
+        const int kc = i / D, dr = i % D;  // 16-key chunk, feature row
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int k0 = kc * 16 + 4 * e;
+            w[e] = static_cast<uint32_t>(tile[k0][dr]) | (static_cast<uint32_t>(tile[k0 + 1][dr]) << 8) |
+                   (static_cast<uint32_t>(tile[k0 + 2][dr]) << 16) | (static_cast<uint32_t>(tile[k0 + 3][dr]) << 24);
+        }
+        *reinterpret_cast<uint4 *>(dst + static_cast<long long>(dr) * np + kc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
+    if (a.g.d != 128) return cudaErrorInvalidValue;
+    const dim3 tg(static_cast<unsigned>(a.g.B * a.g.H), static_cast<unsigned>(a.vt_cols / 128));
+    attn_fp8_vt_kernel<128><<<tg, 256, 0, stream>>>(static_cast<const uint8_t *>(a.v8), static_cast<uint8_t *>(a.vt),
+                                                    a.g.N, a.vt_cols);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_fwd_d<128, false, true>(a, stream);
 }
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {

@@ -18,6 +18,11 @@ struct FwdLaunch {
     float scale;
     int causal;
     int num_sms;  // persistent grid size
+    // e4m3 forward only: dequantisation scales, the V codes and their transposed copy
+    float q_scale, k_scale, v_scale;
+    const void *v8;
+    void *vt;      // [B*H][d][vt_cols] bytes (workspace)
+    int vt_cols;   // N rounded up to 128
 };
 
 struct BwdLaunch {
@@ -38,6 +43,7 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);
+cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream);  // tm_q/tm_k: e4m3 maps, tm_v: V^T map
 cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream);
 
 }  // namespace attn

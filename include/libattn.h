@@ -193,6 +193,34 @@ ATTN_API int attn_bwd_blocksparse(const void *q, const void *k, const void *v, c
                                   const uint8_t *block_mask, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/*
+ * FP8 forward ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程" / codechina
+ * FlashAttention article §9, future directions: mixed precision with FP8 matrix
+ * products and higher-precision accumulation).  The products Q K^T and P V run on
+ * 8-bit floating-point operands with fp32 accumulation; the result is the same
+ * attention as attn_fwd of the dequantised inputs, up to the rounding below.
+ *   q, k, v  : DEVICE e4m3 codes (1 byte each: sign, 4 exponent bits with bias 7,
+ *              3 mantissa bits; no infinities, 0x7F / 0xFF are NaN, largest
+ *              finite 448), dense contiguous [B, H, N, d].
+ *   q_scale, k_scale, v_scale : per-tensor dequantisation factors (finite, > 0):
+ *              the element value is decode(code) * scale.
+ *   o        : output (bf16) [B, H, N, d];  lse : output (fp32) [B, H, N], as for
+ *              attn_fwd (natural-log logsumexp of the scaled dequantised scores).
+ *   scale, is_causal : as for attn_fwd (dense layout, no key mask).
+ *   workspace: caller-owned DEVICE memory of at least
+ *              attn_fwd_fp8_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
+ *              scratch for a transposed copy of v (d rows of the keys per
+ *              (b, h)), needs no initialisation.
+ * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise).  Rounding beyond attn_fwd's:
+ * the probabilities enter P V as e4m3 (relative error <= 2^-4, absolute <= 2^-10
+ * below 2^-6 on the scale where the row's running maximum is 1); the row sums and
+ * lse use the unrounded fp32 probabilities.
+ */
+ATTN_API size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
+ATTN_API int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_scale, float k_scale,
+                          float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
+                          int is_causal, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -6,6 +6,8 @@ there is no fallback from the product path into it.
 
 ``fwd`` / ``bwd`` wrap the C implementation in ``attn_oracle.c`` (plain float64,
 OpenMP over rows, no BLAS).  Inputs are upcast exactly from bf16 to float64.
+``e4m3_decode`` / ``fwd_fp8`` give the attention of 8-bit e4m3 inputs: the codes are
+decoded exactly to float64 (times their per-tensor factor), then ``fwd`` runs.
 See ``attn_oracle.c`` for the definition and the passages it follows.
 """
 from __future__ import annotations
@@ -37,6 +39,8 @@ def lib():
                                       ip, up, up, ctypes.c_int, ip, ctypes.c_int, ctypes.c_int]
         L.oracle_attn_bwd.restype = ctypes.c_int
         L.oracle_max_threads.restype = ctypes.c_int
+        L.oracle_e4m3_decode.argtypes = [up, ctypes.c_long, ctypes.c_double, dp]
+        L.oracle_e4m3_decode.restype = None
         _lib = L
     return _lib
 
@@ -146,3 +150,29 @@ def bwd(q, k, v, dout, scale, causal, cu_seqlens=None, key_keep=None, slices=Non
     if rc != 0:
         raise ValueError("oracle_attn_bwd rejected its arguments")
     return dq, dk, dv
+
+
+def e4m3_decode(codes, factor=1.0):
+    """float64 values of e4m3 codes (uint8 array-like or a torch float8_e4m3fn / uint8
+    tensor) times ``factor``; same shape."""
+    try:
+        import torch
+        if isinstance(codes, torch.Tensor):
+            codes = codes.detach().cpu()
+            if codes.dtype != torch.uint8:
+                codes = codes.view(torch.uint8)
+            codes = codes.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.empty(c.shape, dtype=np.float64)
+    lib().oracle_e4m3_decode(_ptr(c, ctypes.c_ubyte), c.size, float(factor), _ptr(out, ctypes.c_double))
+    return out
+
+
+def fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale, causal, slices=None, nthreads=None):
+    """Forward of dense [B,H,N,d] e4m3 inputs: the attention of the decoded values
+    (code value x per-tensor factor).  Returns (o, lse) float64 like ``fwd``."""
+    return fwd(e4m3_decode(q8, q_scale), e4m3_decode(k8, k_scale), e4m3_decode(v8, v_scale), scale, causal,
+               slices=slices, nthreads=nthreads)
+

@@ -38,6 +38,13 @@
  * block-row query tile and a block-column key tile either takes part or is left
  * out as a whole; left-out pairs behave exactly like masked scores.
  *
+ * FP8 inputs (the mixed-precision direction of the codechina FlashAttention
+ * article, §9: FP8 matrix products with higher-precision accumulation) are
+ * 8-bit e4m3 codes with one dequantisation factor per tensor.  The attention
+ * they define is the one above applied to the decoded values code -> value *
+ * factor; oracle_e4m3_decode turns codes into those float64 values (format
+ * below), and the forward then runs unchanged.
+ *
  * Layouts (element offsets, double precision arrays):
  *   dense   (cu_seqlens == NULL): Q,K,V,O,dO,dQ,dK,dV are [B,H,N,d]; lse is [B,H,N];
  *           key_keep (optional) is [B,N]; block_mask (optional) is [H, nb, nb] with
@@ -303,4 +310,28 @@ int oracle_max_threads(void)
 #else
     return 1;
 #endif
+}
+
+/*
+ * e4m3 (the OCP 8-bit floating-point format's E4M3 encoding): bit 7 sign, bits 3-6
+ * a biased exponent e (bias 7), bits 0-2 a mantissa m.
+ *   e == 0              : subnormal, (m / 8) * 2^(1 - 7)
+ *   e == 15 and m == 7  : NaN (the encoding has no infinities)
+ *   otherwise           : (1 + m / 8) * 2^(e - 7)        (largest: 448)
+ * out[i] = sign * value(codes[i]) * factor.
+ */
+void oracle_e4m3_decode(const unsigned char *codes, long n, double factor, double *out)
+{
+    for (long i = 0; i < n; ++i) {
+        const int c = codes[i];
+        const int e = (c >> 3) & 15, m = c & 7;
+        double v;
+        if (e == 15 && m == 7)
+            v = NAN;
+        else if (e == 0)
+            v = ldexp((double)m / 8.0, 1 - 7);
+        else
+            v = ldexp(1.0 + (double)m / 8.0, e - 7);
+        out[i] = ((c & 128) ? -v : v) * factor;
+    }
 }

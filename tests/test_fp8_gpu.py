@@ -1,0 +1,150 @@
+"""FP8 (e4m3) forward parity: the sm_100a kernel through the C ABI against the
+float64 oracle's attention of the decoded inputs.
+
+Tolerance, derived from the kernel's arithmetic.  Q K^T and P V take e4m3 operands
+with fp32 accumulation; the one rounding beyond the bf16 path's is P, rounded to
+e4m3 on a scale where the row's running maximum is at most 2^8 (lazy rescaling)
+and the row sum is at least the true one (the running maximum never exceeds the
+true maximum).  Round-to-nearest e4m3 errs by at most 2^-4 of a normal value and
+by 2^-10 absolute below 2^-6, so each weight w_ij = softmax_j errs by at most
+    e_ij = max(2^-4 w_ij, 2^-10 / l'_i),   l'_i = sum_j exp(S_ij - max_j S_ij)
+(0 for masked keys), and the output element by sum_j e_ij |V_jc|.  On top: bf16
+rounding of O (2^-8 relative), and an allowance of 1e-3 on every score for the
+fp32 (or narrower) accumulation of the e4m3 products, which moves O by at most
+1e-3 (sum_j w_ij |V_jc| + |O_ic|).  lse: |err| <= 1e-3 (scores only).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attn_inputs import make_fp8
+
+pytestmark = pytest.mark.gpu
+
+LSE_ATOL = 1e-3
+S_ALLOW = 1e-3
+
+
+@pytest.fixture(scope="module")
+def ea():
+    from exact_attention_123_b200 import build
+    build.build()
+    import exact_attention_123_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def gpu_fp8(ea, inp, causal=None, workspace=None):
+    causal = inp.causal if causal is None else causal
+    q8, k8, v8 = inp.q8.cuda(), inp.k8.cuda(), inp.v8.cuda()
+    o = torch.full((inp.B, inp.H, inp.N, inp.d), float("nan"), device="cuda", dtype=torch.bfloat16)
+    lse = torch.full((inp.B, inp.H, inp.N), float("nan"), device="cuda")
+    ea.attn_fwd_fp8(q8, k8, v8, inp.q_scale, inp.k_scale, inp.v_scale, o, lse, scale=inp.scale, causal=causal,
+                    workspace=workspace)
+    assert ea.attn_status() == ea.ATTN_OK
+    return o.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref):
+    """Elementwise error bound for one (b, h) slice (float64 numpy, n x d)."""
+    n = qd.shape[0]
+    S = scale * (qd @ kd.T)
+    if causal:
+        S[np.triu_indices(n, 1)] = -np.inf
+    m = S.max(axis=1)
+    W = np.exp(S - lse_ref[:, None])
+    lp = np.exp(lse_ref - m)
+    E = np.where(np.isfinite(S), np.maximum(2.0 ** -4 * W, (2.0 ** -10 / lp)[:, None]), 0.0)
+    A = np.abs(vd)
+    return E @ A + S_ALLOW * (W @ A + np.abs(o_ref)) + 2.0 ** -8 * np.abs(o_ref) + 1e-6
+
+
+def check(inp, got_o, got_l, causal, slices=None):
+    ro, rl = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, inp.v_scale, inp.scale, causal,
+                            slices=slices)
+    qd = oracle.e4m3_decode(inp.q8, inp.q_scale)
+    kd = oracle.e4m3_decode(inp.k8, inp.k_scale)
+    vd = oracle.e4m3_decode(inp.v8, inp.v_scale)
+    todo = slices if slices is not None else range(inp.B * inp.H)
+    worst = 0.0
+    for sidx in todo:
+        b, h = divmod(int(sidx), inp.H)
+        tol = bound_slice(qd[b, h], kd[b, h], vd[b, h], inp.scale, causal, ro[b, h], rl[b, h])
+        err = np.abs(got_o[b, h] - ro[b, h])
+        assert not np.isnan(got_o[b, h]).any(), f"NaN in slice {sidx}"
+        bad = err > tol
+        if bad.any():
+            i = np.unravel_index(np.argmax(err - tol), err.shape)
+            raise AssertionError(f"slice {sidx}: {bad.sum()} elements out of bound; worst at {i}: gpu {got_o[b, h][i]} "
+                                 f"ref {ro[b, h][i]} bound {tol[i]}")
+        worst = max(worst, float((err / tol).max()))
+        lerr = np.abs(got_l[b, h] - rl[b, h])
+        assert lerr.max() <= LSE_ATOL, f"slice {sidx}: lse err {lerr.max()}"
+    return worst
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_ragged_tiles(ea, causal):
+    # 5 query tiles: two full 256-row units and a half one; keys end mid-tile too
+    inp = make_fp8(1, 2, 640 - 37, 128, seed=8200, causal=causal)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, causal)
+
+
+def test_fp8_several_slices_and_short_rows(ea):
+    inp = make_fp8(2, 3, 333, 128, seed=8201, causal=False)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, False)
+
+
+@pytest.mark.parametrize("N", [1, 17, 128, 129])
+def test_fp8_edge_lengths(ea, N):
+    inp = make_fp8(1, 1, N, 128, seed=8210 + N, causal=True)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, True)
+
+
+def test_fp8_wide_scores_exercise_rescaling(ea):
+    # Q, K ~ N(0, 4^2): scores spread over tens of units, so running maxima move by
+    # more than the lazy-rescale threshold and P values reach far below 2^-6
+    inp = make_fp8(1, 2, 512, 128, seed=8220, causal=True, qk_sigma=4.0)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, True)
+
+
+def test_fp8_bound_is_not_vacuous(ea):
+    # the rounding bound must be tight enough to catch a wrong P: the observed error
+    # uses a sizeable part of it, but nowhere near all of it
+    inp = make_fp8(1, 2, 512, 128, seed=8230, causal=True)
+    o, l = gpu_fp8(ea, inp)
+    worst = check(inp, o, l, True)
+    assert 0.01 < worst <= 1.0
+
+
+def test_fp8_zero_inputs(ea):
+    inp = make_fp8(1, 1, 200, 128, seed=8240, causal=True)
+    z = torch.zeros_like(inp.q8)
+    inp.q8, inp.k8, inp.v8 = z, z.clone(), z.clone()
+    o, l = gpu_fp8(ea, inp)
+    assert np.all(o == 0.0)
+    # all scores 0: row i sees i+1 equal keys
+    assert np.allclose(l[0, 0], np.log(np.arange(1, 201)), atol=1e-5)
+
+
+def test_fp8_caller_workspace_and_repeat(ea):
+    inp = make_fp8(1, 2, 300, 128, seed=8250, causal=True)
+    ws = torch.empty(ea.attn_fwd_fp8_workspace_bytes(1, 2, 300, 128), dtype=torch.uint8, device="cuda")
+    o1, l1 = gpu_fp8(ea, inp, workspace=ws)
+    o2, l2 = gpu_fp8(ea, inp, workspace=ws)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)  # deterministic
+    check(inp, o1, l1, True)
+
+
+def test_fp8_full_size_sampled_slices(ea):
+    # the benchmark workload (causal, B2 H16 N4096 d128), checked on sampled slices
+    inp = make_fp8(2, 16, 4096, 128, seed=8260, causal=True)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, True, slices=[0, 13, 31])

@@ -505,3 +505,46 @@ def test_block_mask_rejected_with_packed_layout():
     q = np.zeros((8, 1, 4))
     with pytest.raises(ValueError):
         oracle.fwd(q, q, q, 1.0, False, cu_seqlens=[0, 3, 8], block_mask=np.ones((1, 1, 1), np.uint8), block=128)
+
+
+# ---------------------------------------------------------------- e4m3 (FP8) inputs
+def test_e4m3_decode_closed_forms():
+    # values fixed by the format: sign bit, 4-bit exponent with bias 7, 3-bit mantissa,
+    # subnormals at exponent 0, NaN only at S.1111.111, no infinities
+    want = {0x00: 0.0, 0x38: 1.0, 0x3C: 1.5, 0x40: 2.0, 0x30: 0.5, 0x7E: 448.0, 0x77: 240.0,
+            0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x0F: 1.875 * 2.0 ** -6,
+            0xB8: -1.0, 0xFE: -448.0, 0x81: -(2.0 ** -9), 0x7D: 416.0, 0x78: 256.0}
+    codes = np.array(sorted(want), dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    assert list(got) == [want[c] for c in sorted(want)]
+    z = oracle.e4m3_decode(np.array([0x80], dtype=np.uint8))
+    assert z[0] == 0.0 and math.copysign(1.0, z[0]) == -1.0  # negative zero
+    nan = oracle.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))
+    assert np.isnan(nan).all()
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    lib_vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_decode(codes), lib_vals, equal_nan=True)
+    # finite codes are strictly increasing in magnitude with the code, sign aside
+    pos = oracle.e4m3_decode(codes[:0x7F])
+    assert np.all(np.diff(pos) > 0)
+
+
+def test_e4m3_decode_applies_the_factor():
+    codes = np.arange(0, 0x7F, dtype=np.uint8)
+    base = oracle.e4m3_decode(codes)
+    for f in (0.25, 3.0, 1.0 / 448.0):
+        assert np.array_equal(oracle.e4m3_decode(codes, f), base * f)
+
+
+def test_fwd_fp8_is_attention_of_the_decoded_inputs():
+    # distinct factors per tensor, so a swapped operand or factor shows up
+    from attn_inputs import make_fp8
+    inp = make_fp8(1, 2, 96, 16, seed=8100, causal=True)
+    dec = [torch.from_numpy(t.numpy()).view(torch.float8_e4m3fn).to(torch.float64) * f
+           for t, f in ((inp.q8, inp.q_scale), (inp.k8, inp.k_scale), (inp.v8, 3.0 * inp.v_scale))]
+    o8, l8 = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, 3.0 * inp.v_scale, inp.scale, True)
+    o, l = oracle.fwd(dec[0], dec[1], dec[2], inp.scale, True)
+    assert np.array_equal(o8, o) and np.array_equal(l8, l)
