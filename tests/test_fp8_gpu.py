@@ -6,12 +6,17 @@ with fp32 accumulation; the one rounding beyond the bf16 path's is P, rounded to
 e4m3 on a scale where the row's running maximum is at most 2^8 (lazy rescaling)
 and the row sum is at least the true one (the running maximum never exceeds the
 true maximum).  Round-to-nearest e4m3 errs by at most 2^-4 of a normal value and
-by 2^-10 absolute below 2^-6, so each weight w_ij = softmax_j errs by at most
-    e_ij = max(2^-4 w_ij, 2^-10 / l'_i),   l'_i = sum_j exp(S_ij - max_j S_ij)
-(0 for masked keys), and the output element by sum_j e_ij |V_jc|.  On top: bf16
-rounding of O (2^-8 relative), and an allowance of 1e-3 on every score for the
-fp32 (or narrower) accumulation of the e4m3 products, which moves O by at most
-1e-3 (sum_j w_ij |V_jc| + |O_ic|).  lse: |err| <= 1e-3 (scores only).
+by 2^-10 absolute below 2^-6.  The probabilities themselves carry the relative
+error eps of the exponential (1.02e-4 for the quarter computed by the cubic on the
+FMA pipe, 2^-22 for the MUFU ones), so each weight w_ij = softmax_j of the
+rounded P errs by at most
+    e_ij = max((2^-4 + 2^-12) w_ij, 2^-10 / l'_i),  l'_i = sum_j exp(S_ij - max_j S_ij)
+(0 for masked keys; 2^-12 > eps (1 + 2^-4)), and the output element by
+sum_j e_ij |V_jc|.  The row sum, made of the unrounded probabilities, carries eps
+too: O moves by at most eps |O_ic| (taken as 2^-13).  On top: bf16 rounding of O
+(2^-8 relative), and an allowance of 1e-3 on every score for the fp32 (or
+narrower) accumulation of the e4m3 products, which moves O by at most
+1e-3 (sum_j w_ij |V_jc| + |O_ic|).  lse: |err| <= 1e-3 (scores and eps).
 """
 import math
 
@@ -57,9 +62,9 @@ def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref):
     m = S.max(axis=1)
     W = np.exp(S - lse_ref[:, None])
     lp = np.exp(lse_ref - m)
-    E = np.where(np.isfinite(S), np.maximum(2.0 ** -4 * W, (2.0 ** -10 / lp)[:, None]), 0.0)
+    E = np.where(np.isfinite(S), np.maximum((2.0 ** -4 + 2.0 ** -12) * W, (2.0 ** -10 / lp)[:, None]), 0.0)
     A = np.abs(vd)
-    return E @ A + S_ALLOW * (W @ A + np.abs(o_ref)) + 2.0 ** -8 * np.abs(o_ref) + 1e-6
+    return E @ A + S_ALLOW * (W @ A + np.abs(o_ref)) + (2.0 ** -8 + 2.0 ** -13) * np.abs(o_ref) + 1e-6
 
 
 def check(inp, got_o, got_l, causal, slices=None):
