@@ -337,6 +337,37 @@ def run_ours(args):
                "bwd_tflops": 2.5 * fl_fwd / (b_ms * 1e-3) / 1e12,
                "note": "attn_fwd_blocksparse / attn_bwd_blocksparse on the bench workload; FLOPs of the computed tile pairs"}
 
+    # ---- FP8 (e4m3) forward on the same workload: q, k, v quantised per tensor
+    # (factor = amax / 448) on the device; timed like the block-sparse variant.
+    # FLOPs as the bf16 forward's; the peak is the measured bf16 one times the
+    # nominal e4m3 : bf16 dense ratio (2).
+    fp8 = None
+    if not args.no_fp8 and ws == 1:
+        q8s = []
+        for t in (q, k, v):
+            fct = float(t.abs().max().float().item()) / 448.0
+            q8s.append(((t.float() / fct).to(torch.float8_e4m3fn), fct))
+        (q8, qf), (k8, kf), (v8, vf) = q8s
+        ws8 = torch.empty(ea.attn_fwd_fp8_workspace_bytes(B, H, N, D), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, workspace=ws8, **kw)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
+        for e in ev:
+            flush.zero_()
+            e[0].record(stream)
+            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, workspace=ws8, **kw)
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        st = ea.attn_status(stream)
+        if st != ea.ATTN_OK:
+            raise RuntimeError(f"fp8 forward reported status {st}")
+        f8_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        f8_tf = flops_fwd() / (f8_ms * 1e-3) / 1e12
+        pk8 = 2.0 * float(measured_peaks()[0]["bf16_tflops"])
+        fp8 = {"fwd_ms": f8_ms, "fwd_tflops": f8_tf, "peak_tflops": pk8, "frac_of_peak": f8_tf / pk8,
+               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal e4m3 : bf16 dense ratio)",
+               "note": "attn_fwd_fp8 (V transpose + forward kernel) on the bench workload, e4m3 inputs"}
+
     step_flops = flops_fwd() + flops_bwd()
     value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12
     e2e_value = step_flops * e2e_n * ws / (e2e_ms * 1e-3) / 1e12
@@ -392,6 +423,7 @@ def run_ours(args):
         "wall_s_timed_region": wall,
         "cpu_baseline": cpu,
         "blocksparse": bsp,
+        "fp8": fp8,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -407,6 +439,7 @@ def main():
     ap.add_argument("--cpu-heads", type=int, default=4, help="(b,h) slices in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward's timing")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
