@@ -348,14 +348,13 @@ def run_ours(args):
             fct = float(t.abs().max().float().item()) / 448.0
             q8s.append(((t.float() / fct).to(torch.float8_e4m3fn), fct))
         (q8, qf), (k8, kf), (v8, vf) = q8s
-        ws8 = torch.empty(ea.attn_fwd_fp8_workspace_bytes(B, H, N, D), dtype=torch.uint8, device=dev)
         for _ in range(3):
-            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, workspace=ws8, **kw)
+            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, **kw)
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
         for e in ev:
             flush.zero_()
             e[0].record(stream)
-            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, workspace=ws8, **kw)
+            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, **kw)
             e[1].record(stream)
         torch.cuda.synchronize(dev)
         st = ea.attn_status(stream)
@@ -366,7 +365,7 @@ def run_ours(args):
         pk8 = 2.0 * float(measured_peaks()[0]["bf16_tflops"])
         fp8 = {"fwd_ms": f8_ms, "fwd_tflops": f8_tf, "peak_tflops": pk8, "frac_of_peak": f8_tf / pk8,
                "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal e4m3 : bf16 dense ratio)",
-               "note": "attn_fwd_fp8 (V transpose + forward kernel) on the bench workload, e4m3 inputs"}
+               "note": "attn_fwd_fp8 on the bench workload, e4m3 inputs"}
 
     step_flops = flops_fwd() + flops_bwd()
     value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12

@@ -8,7 +8,6 @@ missing, importing the entry points raises.
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
 ``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
 ``attn_fwd_blocksparse``, ``attn_bwd_blocksparse``, ``attn_fwd_fp8``,
-``attn_fwd_fp8_workspace_bytes``,
 ``attn_bwd_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
 ``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
@@ -66,9 +65,7 @@ def lib() -> ctypes.CDLL:
     L.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
     L.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, sz, vp]
     L.attn_bwd_noalloc.restype = i
-    L.attn_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
-    L.attn_fwd_fp8_workspace_bytes.restype = sz
-    L.attn_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    L.attn_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp]
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
     L.attn_strerror.restype = ctypes.c_char_p
@@ -246,13 +243,8 @@ def attn_bwd_blocksparse(q, k, v, o, lse, do, block_mask, dq=None, dk=None, dv=N
     return dq, dk, dv
 
 
-def attn_fwd_fp8_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
-    return int(lib().attn_fwd_fp8_workspace_bytes(int(B), int(H), int(N), int(d)))
-
-
 def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None, lse=None, *,
-                 scale: Optional[float] = None, causal: bool = True, workspace: Optional[torch.Tensor] = None,
-                 stream=None):
+                 scale: Optional[float] = None, causal: bool = True, stream=None):
     """FP8 forward.  q, k, v: dense [B,H,N,d] e4m3 codes (torch.float8_e4m3fn or uint8
     views of them) whose values are code * {q,k,v}_scale.  Returns (o bf16, lse fp32)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
@@ -263,12 +255,8 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None
         scale = 1.0 / math.sqrt(d)
     o = torch.empty((B, H, N, d), device=q.device, dtype=torch.bfloat16) if o is None else o
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
-    if workspace is None:
-        workspace = torch.empty(max(attn_fwd_fp8_workspace_bytes(B, H, N, d), 256), dtype=torch.uint8,
-                                device=q.device)
     rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale), float(v_scale), _ptr(o),
-                            _ptr(lse), B, H, N, d, float(scale), int(causal), _ptr(workspace), workspace.numel(),
-                            _stream(stream))
+                            _ptr(lse), B, H, N, d, float(scale), int(causal), _stream(stream))
     _check(rc, "attn_fwd_fp8")
     return o, lse
 

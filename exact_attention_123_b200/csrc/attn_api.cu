@@ -179,11 +179,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
     return attn::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-long long fp8_vt_cols(int N) { return (static_cast<long long>(N) + 127) / 128 * 128; }
-
 int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
-                 float *lse, const Shape &s, float scale, int is_causal, void *workspace, size_t workspace_bytes,
-                 void *stream) {
+                 float *lse, const Shape &s, float scale, int is_causal, void *stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -192,17 +189,13 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
     if (s.d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_MISALIGNED;
-    const long long np = fp8_vt_cols(s.N);
-    const size_t need = static_cast<size_t>(s.B) * s.H * s.d * np;
-    if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
     DeviceState *ds = nullptr;
     if ((rc = device_state(&ds))) return rc;
     attn::FwdLaunch a{};
-    const long long slabs = static_cast<long long>(s.B) * s.H;
-    if ((rc = make_map_u8(&a.tm_q, q, s.d, s.N, slabs, s.d, static_cast<long long>(s.N) * s.d, 128)) ||
-        (rc = make_map_u8(&a.tm_k, k, s.d, s.N, slabs, s.d, static_cast<long long>(s.N) * s.d, 128)) ||
-        (rc = make_map_u8(&a.tm_v, workspace, np, s.d, slabs, np, np * s.d, s.d)) ||
+    const long long slabs = static_cast<long long>(s.B) * s.H, slab_stride = static_cast<long long>(s.N) * s.d;
+    if ((rc = make_map_u8(&a.tm_q, q, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
+        (rc = make_map_u8(&a.tm_k, k, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
+        (rc = make_map_u8(&a.tm_v, v, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
         (rc = map_for(&a.tm_o_st, o, s, 32, false, 32)))
         return rc;
     a.g = geom_of(s, nullptr);
@@ -215,9 +208,6 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
     a.q_scale = q_scale;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
-    a.v8 = v;
-    a.vt = workspace;
-    a.vt_cols = static_cast<int>(np);
     return attn::launch_fwd_fp8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -301,17 +291,10 @@ int attn_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, f
     return fwd_impl(q, k, v, o, lse, s, scale, is_causal, nullptr, stream, block_mask);
 }
 
-size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
-    if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-    return static_cast<size_t>(B) * H * d * fp8_vt_cols(N);
-}
-
 int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
-                 float *lse, int B, int H, int N, int d, float scale, int is_causal, void *workspace,
-                 size_t workspace_bytes, void *stream) {
+                 float *lse, int B, int H, int N, int d, float scale, int is_causal, void *stream) {
     Shape s{B, H, N, d, 0, nullptr};
-    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, workspace, workspace_bytes,
-                        stream);
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, stream);
 }
 
 int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,

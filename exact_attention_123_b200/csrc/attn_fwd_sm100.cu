@@ -49,13 +49,12 @@
 
 namespace attn {
 
-// F8: Q, K and V in e4m3 (the V tiles then come from a transposed copy, d rows x
-// 128 keys, so that both products take K-major operands), P rounded to e4m3 in
-// shared memory, fp32 accumulation.
+// F8: Q, K and V in e4m3 (V, keys x d, is the MN-major B operand of P V as in the
+// bf16 path), P rounded to e4m3 in shared memory, fp32 accumulation.
 template <int D, bool F8 = false>
 struct FwdCfg {
     static constexpr int kEsz = F8 ? 1 : 2;                // bytes per Q/K/V element
-    static constexpr int kTileBytes = 128 * D * kEsz;      // one 128-row tile (e4m3 V^T: d rows x 128 keys)
+    static constexpr int kTileBytes = 128 * D * kEsz;      // one 128-row tile
     static constexpr int kBoxes = D * kEsz / 128;          // 128-byte-swizzle boxes per tile
     static constexpr int kKSteps = D * kEsz / 32;          // 32-byte K steps of S = Q K^T
     static constexpr int kStages = F8 ? 8 : (D == 128) ? 4 : 8;
@@ -143,8 +142,7 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-// SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs (tm_v then maps
-// the transposed V).
+// SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs.
 template <int D, bool SP, bool F8>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -224,17 +222,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                         if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
                         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
-                        if constexpr (F8) {
-                            if (kv)  // V^T: columns are keys, rows the d features
-                                tma_load_3d(slot(s), &tm_v, bar(C::kBarFull + s), 128 * j, 0, slab);
-                            else
-                                tma_load_3d(slot(s), &tm_k, bar(C::kBarFull + s), 0, row0 + 128 * j, slab);
-                        } else {
 #pragma unroll
-                            for (int x = 0; x < C::kBoxes; ++x)
-                                tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s), x * 64,
-                                            row0 + 128 * j, slab);
-                        }
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s),
+                                        x * (128 / C::kEsz), row0 + 128 * j, slab);
                         n_issued = idx + 1;
                     }
                 }
@@ -243,8 +234,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D, 1) : idesc_bf16_f32(128, D, 0, 1);
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
             // S_t from the K tile at ring position kpos
@@ -267,12 +258,13 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             auto issue_PV = [&](int t, int vpos, bool acc) {
                 const uint32_t vs = slot(vpos % C::kStages);
                 if constexpr (F8) {
-                    // A = P_t (shared memory, 128 queries x 128 keys), B = V^T (d x 128 keys)
+                    // A = P_t (shared memory, 128 queries x 128 keys, K-major), B = V (128 keys
+                    // x d, MN-major: each 32-key step is 32 rows of 128 bytes)
                     const uint32_t ps = sbase + C::kOffP + t * 16384;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ss_f8(tmem + colO[t], sw128_desc(ps + kk * 32, 16, 1024), sw128_desc(vs + kk * 32, 16, 1024),
-                                  idPV, (acc || kk > 0) ? 1u : 0u);
+                        mma_ss_f8(tmem + colO[t], sw128_desc(ps + kk * 32, 16, 1024),
+                                  sw128_desc(vs + kk * 4096, 16384, 1024), idPV, (acc || kk > 0) ? 1u : 0u);
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
@@ -615,44 +607,8 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// V (e4m3, [slab][N][D]) -> V^T ([slab][D][np], np = N rounded up to 128; the
-// columns from N on are zero).  One CTA per (slab, 128-key tile).
-template <int D>
-__global__ void __launch_bounds__(256) attn_fp8_vt_kernel(const uint8_t *__restrict__ v, uint8_t *__restrict__ vt,
-                                                          int N, int np) {
-    __shared__ __align__(16) uint8_t tile[128][D + 16];
-    const long long slab = blockIdx.x;
-    const int kt = blockIdx.y;
-    const uint8_t *src = v + slab * N * D;
-    for (int i = threadIdx.x; i < 128 * (D / 16); i += 256) {
-        const int r = i / (D / 16), c = i % (D / 16);
-        const int key = kt * 128 + r;
-        uint4 x = make_uint4(0u, 0u, 0u, 0u);
-        if (key < N) x = *reinterpret_cast<const uint4 *>(src + static_cast<long long>(key) * D + c * 16);
-        *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = x;
-    }
-    __syncthreads();
-    uint8_t *dst = vt + slab * D * np + kt * 128;
-    for (int i = threadIdx.x; i < D * 8; i += 256) {
-        const int kc = i / D, dr = i % D;  // 16-key chunk, feature row
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int k0 = kc * 16 + 4 * e;
-            w[e] = static_cast<uint32_t>(tile[k0][dr]) | (static_cast<uint32_t>(tile[k0 + 1][dr]) << 8) |
-                   (static_cast<uint32_t>(tile[k0 + 2][dr]) << 16) | (static_cast<uint32_t>(tile[k0 + 3][dr]) << 24);
-        }
-        *reinterpret_cast<uint4 *>(dst + static_cast<long long>(dr) * np + kc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
     if (a.g.d != 128) return cudaErrorInvalidValue;
-    const dim3 tg(static_cast<unsigned>(a.g.B * a.g.H), static_cast<unsigned>(a.vt_cols / 128));
-    attn_fp8_vt_kernel<128><<<tg, 256, 0, stream>>>(static_cast<const uint8_t *>(a.v8), static_cast<uint8_t *>(a.vt),
-                                                    a.g.N, a.vt_cols);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     return launch_fwd_d<128, false, true>(a, stream);
 }
 

@@ -18,11 +18,7 @@ struct FwdLaunch {
     float scale;
     int causal;
     int num_sms;  // persistent grid size
-    // e4m3 forward only: dequantisation scales, the V codes and their transposed copy
-    float q_scale, k_scale, v_scale;
-    const void *v8;
-    void *vt;      // [B*H][d][vt_cols] bytes (workspace)
-    int vt_cols;   // N rounded up to 128
+    float q_scale, k_scale, v_scale;  // e4m3 forward only: dequantisation factors
 };
 
 struct BwdLaunch {
@@ -43,7 +39,7 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);
-cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream);  // tm_q/tm_k: e4m3 maps, tm_v: V^T map
+cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream);  // tm_q/tm_k/tm_v: e4m3 maps
 cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream);
 
 }  // namespace attn

@@ -219,9 +219,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
 }
 
 // Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0 in bits
-// 7-9 and 10-12), fp32 D, both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
-    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// 7-9 and 10-12), fp32 D, A K-major; B K-major or MN-major (bit 16; the MN-major
+// form is defined for the 8-bit formats, not for the 6- and 4-bit ones).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int b_mn_major) {
+    return (1u << 4) | (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ math

@@ -207,19 +207,15 @@ ATTN_API int attn_bwd_blocksparse(const void *q, const void *k, const void *v, c
  *   o        : output (bf16) [B, H, N, d];  lse : output (fp32) [B, H, N], as for
  *              attn_fwd (natural-log logsumexp of the scaled dequantised scores).
  *   scale, is_causal : as for attn_fwd (dense layout, no key mask).
- *   workspace: caller-owned DEVICE memory of at least
- *              attn_fwd_fp8_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
- *              scratch for a transposed copy of v (d rows of the keys per
- *              (b, h)), needs no initialisation.
- * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise).  Rounding beyond attn_fwd's:
- * the probabilities enter P V as e4m3 (relative error <= 2^-4, absolute <= 2^-10
- * below 2^-6 on the scale where the row's running maximum is 1); the row sums and
- * lse use the unrounded fp32 probabilities.
+ * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise).  Nothing is allocated and no
+ * workspace is needed.  Rounding beyond attn_fwd's: the probabilities enter P V as
+ * e4m3 (half an e4m3 step: 2^-4 relative, or 2^-10 absolute below 2^-6, on the
+ * kernel's scale, where the row sum is at least 1), after exponentials accurate to
+ * 1.1e-4 relative; the row sums and lse use the unrounded fp32 probabilities.
  */
-ATTN_API size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
 ATTN_API int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_scale, float k_scale,
                           float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
-                          int is_causal, void *workspace, size_t workspace_bytes, void *stream);
+                          int is_causal, void *stream);
 
 /* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -28,7 +28,7 @@ def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
               "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen", "attn_fwd_blocksparse",
-              "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_workspace_bytes"):
+              "attn_bwd_blocksparse", "attn_fwd_fp8"):
         assert n in names
 
 
@@ -110,29 +110,22 @@ def test_blocksparse_host_argument_errors(L):
     assert L.attn_bwd_blocksparse(*args, vp(FAKE), None, 0, None) == ea.ATTN_ERR_WORKSPACE
 
 
-def test_fp8_host_argument_errors_and_workspace_size(L):
+def test_fp8_host_argument_errors(L):
     import exact_attention_123_b200 as ea
     vp, f = ctypes.c_void_p, ctypes.c_float
-    # the transposed V: d rows of N keys rounded up to 128, per (b, h)
-    assert ea.attn_fwd_fp8_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 128 * 4096
-    assert ea.attn_fwd_fp8_workspace_bytes(1, 1, 1, 128) == 128 * 128
-    assert ea.attn_fwd_fp8_workspace_bytes(1, 3, 200, 128) == 3 * 128 * 256
-    assert ea.attn_fwd_fp8_workspace_bytes(0, 1, 1, 128) == 0
-    need = ea.attn_fwd_fp8_workspace_bytes(1, 1, 256, 128)
 
-    def call(ptrs=(FAKE,) * 5, scales=(1.0, 1.0, 1.0), d=128, ws=FAKE, ws_bytes=need, scale=0.1):
+    def call(ptrs=(FAKE,) * 5, scales=(1.0, 1.0, 1.0), d=128, scale=0.1, B=1):
         p = [vp(x) if x else None for x in ptrs]
-        return L.attn_fwd_fp8(p[0], p[1], p[2], f(scales[0]), f(scales[1]), f(scales[2]), p[3], p[4], 1, 1, 256,
-                              d, f(scale), 1, vp(ws) if ws else None, ws_bytes, None)
+        return L.attn_fwd_fp8(p[0], p[1], p[2], f(scales[0]), f(scales[1]), f(scales[2]), p[3], p[4], B, 1, 256,
+                              d, f(scale), 1, None)
     assert call(ptrs=(FAKE, 0, FAKE, FAKE, FAKE)) == ea.ATTN_ERR_INVALID_ARG
     assert call(scales=(1.0, 0.0, 1.0)) == ea.ATTN_ERR_INVALID_ARG
     assert call(scales=(1.0, 1.0, float("inf"))) == ea.ATTN_ERR_INVALID_ARG
     assert call(scale=-1.0) == ea.ATTN_ERR_INVALID_ARG
     assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
     assert call(ptrs=(FAKE, FAKE, FAKE + 4, FAKE, FAKE)) == ea.ATTN_ERR_MISALIGNED
-    assert call(ws=0) == ea.ATTN_ERR_WORKSPACE
-    assert call(ws_bytes=need - 1) == ea.ATTN_ERR_WORKSPACE
-    assert call(ws=FAKE + 16) == ea.ATTN_ERR_MISALIGNED
+    assert call(ptrs=(FAKE, FAKE, FAKE, FAKE, FAKE + 8)) == ea.ATTN_ERR_MISALIGNED
+    assert call(B=0) == ea.ATTN_ERR_INVALID_ARG
 
 
 def test_wait_limit_and_fault_hook_setters(L):
