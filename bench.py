@@ -435,7 +435,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--cpu-heads", type=int, default=4, help="(b,h) slices in the CPU-oracle baseline sample")
+    ap.add_argument("--cpu-heads", type=int, default=32,
+                    help="(b,h) slices in the CPU-oracle baseline sample (32 = the whole workload, about 14 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward's timing")
