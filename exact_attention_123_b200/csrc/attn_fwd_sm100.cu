@@ -428,9 +428,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int c = 0; c < 32; ++c) {
                     const uint64_t x2 = f2_fma(f2_pack(s[half * 64 + 2 * c], s[half * 64 + 2 * c + 1]), c2x2, negm2);
                     float p0, p1;
-                    if (F8 && (c & 3) == 3) {
-                        // e4m3 path: the tensor core needs half the time of the bf16 one, so
-                        // the MUFU unit sets the pace; one pair in four goes to the FMA pipe
+                    if ((F8 || D == 64) && (c & 7) == 7) {
+                        // Where the products take half the time of the exponentials (e4m3
+                        // operands at d = 128, bf16 at d = 64) the MUFU unit sets the pace, so
+                        // one pair in eight goes to the FMA pipe
                         ex2_poly_x2(x2, p0, p1);
                     } else {
                         float x0, x1;

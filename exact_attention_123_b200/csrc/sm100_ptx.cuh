@@ -267,30 +267,32 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 }
 
 // Two base-2 exponentials on the FMA pipe instead of the MUFU unit.  2^x = 2^j 2^f
-// with j = rint(x) (added to the exponent field) and f = x - j in [-1/2, 1/2];
-// 2^f is the cubic 1 + f (a1 + f (a2 + f a3)) whose coefficients were fitted for
-// this kernel (Lawson-weighted least squares towards the minimax relative error
-// on [-1/2, 1/2]; max relative error 1.0e-4 in float32 Horner evaluation).  Valid
-// for x <= 2^22; x below -125 (-inf included) gives about 2^-125 instead of 0.
-// rint: adding 1.5 * 2^23 leaves j in the low mantissa bits, and shifting those
-// bits up by 23 moves j into the exponent field (the constant's own bits shift out).
+// with j = rint(x) and f = x - j in [-1/2, 1/2]; 2^f is the cubic
+// 1 + f (a1 + f (a2 + f a3)) whose coefficients were fitted for this kernel
+// (Lawson-weighted least squares towards the minimax relative error on [-1/2, 1/2];
+// max relative error 1.0e-4 in float32 Horner evaluation), and 2^j is built as a
+// float of its own, bits (j + 127) << 23.  x is first clamped to -127 (-inf
+// included), where that float is +0, so everything below about 2^-126.5 comes out
+// as exactly 0.  Valid for x <= 2^22.  rint: adding 1.5 * 2^23 leaves j in the low
+// mantissa bits of t; shifting t's bits up by 23 moves j into the exponent field
+// (the constant's own bits shift out), and 127 << 23 adds the bias.
 __device__ __forceinline__ void ex2_poly_x2(uint64_t x2, float &y0, float &y1) {
     constexpr float kA1 = 0.6932829022407532f, kA2 = 0.2422109693288803f, kA3 = 0.05500892922282219f;
     constexpr float kRint = 12582912.0f;  // 1.5 * 2^23
     float x0, x1;
     f2_unpack(x2, x0, x1);
-    const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t xc = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
     const uint64_t t = f2_add(xc, f2_pack(kRint, kRint));
     const uint64_t r = f2_add(t, f2_pack(-kRint, -kRint));
     const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), xc);
     uint64_t q = f2_fma(f, f2_pack(kA3, kA3), f2_pack(kA2, kA2));
     q = f2_fma(q, f, f2_pack(kA1, kA1));
     q = f2_fma(q, f, f2_pack(1.f, 1.f));
-    float q0, q1, t0, t1;
-    f2_unpack(q, q0, q1);
+    float t0, t1;
     f2_unpack(t, t0, t1);
-    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+    const uint64_t p2j = f2_pack(__uint_as_float((__float_as_uint(t0) << 23) + 0x3F800000u),
+                                 __uint_as_float((__float_as_uint(t1) << 23) + 0x3F800000u));
+    f2_unpack(f2_fma(q, p2j, f2_pack(0.f, 0.f)), y0, y1);
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

@@ -7,7 +7,7 @@ e4m3 on a scale where the row's running maximum is at most 2^8 (lazy rescaling)
 and the row sum is at least the true one (the running maximum never exceeds the
 true maximum).  Round-to-nearest e4m3 errs by at most 2^-4 of a normal value and
 by 2^-10 absolute below 2^-6.  The probabilities themselves carry the relative
-error eps of the exponential (1.02e-4 for the quarter computed by the cubic on the
+error eps of the exponential (1.02e-4 for the eighth computed by the cubic on the
 FMA pipe, 2^-22 for the MUFU ones), so each weight w_ij = softmax_j of the
 rounded P errs by at most
     e_ij = max((2^-4 + 2^-12) w_ij, 2^-10 / l'_i),  l'_i = sum_j exp(S_ij - max_j S_ij)
