@@ -7,13 +7,15 @@
 // sum l and an un-normalised output accumulator, rescaled when m moves, divided by
 // l at the end.  The 128 x 128 score tile lives only in tensor memory.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for Q0 (warp w owns TMEM lanes 32*(w%4)..+31, one row/thread)
 //   warps 4-7  softmax for Q1
 //   warp  8    TMA producer: Q0/Q1 once, then K_j, V_j into a ring of shared-memory
 //              slots guarded by full/empty mbarriers (the pages' double buffering,
 //              done by the copy engine instead of the SMs)
 //   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle: with warps 8-9 they form the warpgroup that hands registers
+//              to the two softmax warpgroups (setmaxnreg)
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   S0 = cols [0,128)  S1 = [128,256)   fp32 scores Q_t K_j^T;
@@ -39,6 +41,11 @@
 // the same m, which keeps the final O / l and lse = (m + log2 l) ln 2 exact.
 // A row that sees no key keeps m = -inf and l = 0 and writes O = 0, lse = -inf
 // (the _safe_softmax rule of "Profiling in PyTorch (part 3)", math backend).
+//
+// With e4m3 operands (F8, the FP8 direction of the codechina article's §9) both
+// products are kind::f8f6f4 with fp32 accumulation; P is rounded to e4m3 and
+// written to a swizzled shared-memory tile (the A operand of P V) instead of TMEM,
+// and V is read as it is stored, as the MN-major B operand.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
