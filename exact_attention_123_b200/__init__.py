@@ -99,8 +99,42 @@ def _check(rc: int, where: str):
 
 
 def _need(t: torch.Tensor, dtype, name: str):
-    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    dtypes = dtype if isinstance(dtype, tuple) else (dtype,)
+    if not isinstance(t, torch.Tensor) or t.dtype not in dtypes or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {' or '.join(str(x) for x in dtypes)} tensor")
+
+
+# The library takes raw pointers and the sizes passed with them, so every tensor's
+# shape and device are checked here: a buffer smaller than the sizes say would be
+# read or written out of bounds on the device.
+def _shaped(t, shape, dtype, name: str, device):
+    _need(t, dtype, name)
+    if tuple(t.shape) != tuple(shape) or t.device != device:
+        raise ValueError(f"{name} must have shape {tuple(shape)} on {device}, got {tuple(t.shape)} on {t.device}")
+
+
+def _inputs(tensors, dtype, packed: bool):
+    """(name, tensor) pairs that must all be shaped like the first: [B,H,N,d] dense or
+    [total,H,d] packed, contiguous, on one CUDA device."""
+    (n0, t0), rest = tensors[0], tensors[1:]
+    _need(t0, dtype, n0)
+    if t0.dim() != (3 if packed else 4):
+        raise ValueError(f"{n0} must be {'[total, H, d]' if packed else '[B, H, N, d]'}, got shape {tuple(t0.shape)}")
+    for n, t in rest:
+        _shaped(t, t0.shape, dtype, n, t0.device)
+    return t0
+
+
+def _side(q, cu_seqlens, key_keep, keys: int):
+    """cu_seqlens: 1-D int32 on q's device; key_keep: uint8 with `keys` elements."""
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, "cu_seqlens")
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2 or cu_seqlens.device != q.device:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor of B+1 offsets on q's device")
+    if key_keep is not None:
+        _need(key_keep, torch.uint8, "key_keep")
+        if key_keep.numel() != keys or key_keep.device != q.device:
+            raise ValueError(f"key_keep must hold {keys} uint8 flags on q's device, got {key_keep.numel()}")
 
 
 def attn_fwd(q, k, v, o=None, lse=None, *, scale: Optional[float] = None, causal: bool = True,
@@ -108,18 +142,21 @@ def attn_fwd(q, k, v, o=None, lse=None, *, scale: Optional[float] = None, causal
              max_seqlen: Optional[int] = None, stream=None):
     """Forward pass.  Dense q/k/v are [B,H,N,d]; packed ones are [total,H,d] with
     ``cu_seqlens`` (int32, device).  Returns (o, lse)."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, torch.bfloat16, n)
+    packed = cu_seqlens is not None
+    _inputs([("q", q), ("k", k), ("v", v)], torch.bfloat16, packed)
+    _side(q, cu_seqlens, key_keep, q.shape[0] if packed else q.shape[0] * q.shape[2])
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if o is None:
         o = torch.empty_like(q)
+    _shaped(o, q.shape, torch.bfloat16, "o", q.device)
     if cu_seqlens is not None:
         total, H = q.shape[0], q.shape[1]
         B = cu_seqlens.numel() - 1
         if lse is None:
             lse = torch.empty((total, H), device=q.device, dtype=torch.float32)
+        _shaped(lse, (total, H), torch.float32, "lse", q.device)
         if max_seqlen is None:
             raise ValueError("max_seqlen is required with cu_seqlens")
         rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, total, int(max_seqlen), H, d,
@@ -129,6 +166,7 @@ def attn_fwd(q, k, v, o=None, lse=None, *, scale: Optional[float] = None, causal
     B, H, N, _ = q.shape
     if lse is None:
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
     if key_keep is None:
         rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal),
                             None, _stream(stream))
@@ -170,17 +208,20 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
              causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
              workspace: Optional[torch.Tensor] = None, stream=None):
     """Backward pass.  Returns (dq, dk, dv)."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, torch.bfloat16, n)
-    _need(lse, torch.float32, "lse")
-    d = q.shape[-1]
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
+    packed = cu_seqlens is not None
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _inputs([("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)],
+            torch.bfloat16, packed)
+    _shaped(lse, q.shape[:2] if packed else q.shape[:3], torch.float32, "lse", q.device)
+    _side(q, cu_seqlens, key_keep, q.shape[0] if packed else q.shape[0] * q.shape[2])
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
     if workspace is None:
         workspace = workspace_for(q, cu_seqlens)
+    _need(workspace, torch.uint8, "workspace")
     if cu_seqlens is not None:
         total, H = q.shape[0], q.shape[1]
         B = cu_seqlens.numel() - 1
@@ -205,14 +246,16 @@ def attn_fwd_blocksparse(q, k, v, block_mask, o=None, lse=None, *, scale: Option
     """Block-sparse forward (dense [B,H,N,d] layout).  block_mask: uint8 device tensor
     [H, ceil(N/128), ceil(N/128)]; a zero leaves that (query tile, key tile) pair out.
     Returns (o, lse)."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, torch.bfloat16, n)
-    _need(block_mask, torch.uint8, "block_mask")
+    _inputs([("q", q), ("k", k), ("v", v)], torch.bfloat16, False)
     B, H, N, d = q.shape
+    nb = (N + 127) // 128
+    _shaped(block_mask, (H, nb, nb), torch.uint8, "block_mask", q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _shaped(o, q.shape, torch.bfloat16, "o", q.device)
+    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
     rc = lib().attn_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
                                     int(causal), _ptr(block_mask), _stream(stream))
     _check(rc, "attn_fwd_blocksparse")
@@ -224,18 +267,20 @@ def attn_bwd_blocksparse(q, k, v, o, lse, do, block_mask, dq=None, dk=None, dv=N
                          workspace: Optional[torch.Tensor] = None, stream=None):
     """Block-sparse backward (dense layout, same block_mask as the forward).
     Returns (dq, dk, dv)."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, torch.bfloat16, n)
-    _need(lse, torch.float32, "lse")
-    _need(block_mask, torch.uint8, "block_mask")
-    B, H, N, d = q.shape
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _inputs([("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)],
+            torch.bfloat16, False)
+    B, H, N, d = q.shape
+    nb = (N + 127) // 128
+    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
+    _shaped(block_mask, (H, nb, nb), torch.uint8, "block_mask", q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
     if workspace is None:
         workspace = workspace_for(q)
+    _need(workspace, torch.uint8, "workspace")
     rc = lib().attn_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
                                     _ptr(dv), B, H, N, d, float(scale), int(causal), _ptr(block_mask),
                                     _ptr(workspace), workspace.numel(), _stream(stream))
@@ -247,14 +292,19 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None
                  scale: Optional[float] = None, causal: bool = True, stream=None):
     """FP8 forward.  q, k, v: dense [B,H,N,d] e4m3 codes (torch.float8_e4m3fn or uint8
     views of them) whose values are code * {q,k,v}_scale.  Returns (o bf16, lse fp32)."""
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype not in (torch.float8_e4m3fn, torch.uint8) or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{n} must be a contiguous CUDA float8_e4m3fn (or uint8) tensor")
+    codes = (torch.float8_e4m3fn, torch.uint8)
+    _need(q, codes, "q")
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, H, N, d], got shape {tuple(q.shape)}")
+    _shaped(k, q.shape, codes, "k", q.device)
+    _shaped(v, q.shape, codes, "v", q.device)
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     o = torch.empty((B, H, N, d), device=q.device, dtype=torch.bfloat16) if o is None else o
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _shaped(o, q.shape, torch.bfloat16, "o", q.device)
+    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
     rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale), float(v_scale), _ptr(o),
                             _ptr(lse), B, H, N, d, float(scale), int(causal), _stream(stream))
     _check(rc, "attn_fwd_fp8")
@@ -265,6 +315,12 @@ def attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, *, workspace, sc
                    causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
                    stream=None):
     """Launch one backward phase (0 preprocess, 1 dK/dV, 2 dQ)."""
+    packed = cu_seqlens is not None
+    _inputs([("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)],
+            torch.bfloat16, packed)
+    _shaped(lse, q.shape[:2] if packed else q.shape[:3], torch.float32, "lse", q.device)
+    _side(q, cu_seqlens, key_keep, q.shape[0] if packed else q.shape[0] * q.shape[2])
+    _need(workspace, torch.uint8, "workspace")
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -284,15 +340,16 @@ def attn_bwd_noalloc(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: O
     """Dense-layout backward that uses the library's own scratch array instead of a
     caller workspace, for callers that cannot allocate device memory (see the C
     declaration for the size limit and the sharing rules).  Returns (dq, dk, dv)."""
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _need(t, torch.bfloat16, n)
-    _need(lse, torch.float32, "lse")
-    B, H, N, d = q.shape
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _inputs([("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)],
+            torch.bfloat16, False)
+    _shaped(lse, q.shape[:3], torch.float32, "lse", q.device)
+    _side(q, None, key_keep, q.shape[0] * q.shape[2])
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
     rc = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
                                 _ptr(dv), B, H, N, d, float(scale), int(causal), None, _ptr(key_keep),
                                 _stream(stream))

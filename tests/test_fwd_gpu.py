@@ -228,3 +228,31 @@ def test_full_size_varlen_sampled(ea):
         assert torch.all(o[cu[b]:cu[b] + p, h].float().cpu() == 0)          # padded rows: 0, not NaN
         assert torch.all(torch.isneginf(lse[cu[b]:cu[b] + p, h].cpu()))
     assert not torch.isnan(o.float()).any()
+
+
+def test_binding_rejects_mismatched_buffers(ea):
+    # The C ABI takes raw pointers with sizes; the binding checks every tensor's shape,
+    # dtype and device first, so no kernel ever sees a buffer smaller than its sizes.
+    dev = "cuda"
+    q = torch.zeros(1, 2, 256, 64, device=dev, dtype=torch.bfloat16)
+    small = torch.zeros(1, 2, 128, 64, device=dev, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 256, device=dev)
+    cases = [
+        lambda: ea.attn_fwd(q, small, q),                                     # k shorter than q
+        lambda: ea.attn_fwd(q, q, q, small),                                  # o too small
+        lambda: ea.attn_fwd(q, q, q, None, torch.zeros(1, 2, 128, device=dev)),  # lse too small
+        lambda: ea.attn_fwd(q, q, q.float()),                                 # v not bf16
+        lambda: ea.attn_fwd(q, q, q, key_keep=torch.ones(1, 255, device=dev, dtype=torch.uint8)),
+        lambda: ea.attn_fwd(q[0], q[0], q[0]),                                # not 4-D
+        lambda: ea.attn_bwd(q, q, q, q, lse, small),                          # dO too small
+        lambda: ea.attn_bwd(q, q, q, q, lse, q, small),                       # dQ too small
+        lambda: ea.attn_bwd(q, q, q, q, torch.zeros(2, 256, device=dev), q),  # lse shape
+        lambda: ea.attn_bwd_noalloc(q, q, q, q, lse, q, None, small),         # dK too small
+        lambda: ea.attn_fwd_blocksparse(q, q, q, torch.ones(2, 1, 1, device=dev, dtype=torch.uint8)),
+        lambda: ea.attn_fwd_fp8(q.view(torch.uint8)[..., :64].contiguous(), q, q, 1.0, 1.0, 1.0),
+    ]
+    for i, call in enumerate(cases):
+        with pytest.raises(ValueError):
+            call()
+            pytest.fail(f"case {i} was accepted")
+    assert ea.attn_status() == ea.ATTN_OK
