@@ -175,6 +175,21 @@ def source_digest():
     return h.hexdigest()[:16]
 
 
+def recorded_ncu():
+    """Per-kernel figures of the committed ncu captures, if they were taken on the
+    current kernel code; otherwise None."""
+    p = os.path.join(HERE, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    keys = ("tensor_pipe_active_pct", "hbm_gbs", "dram_bytes_per_launch", "smem_bank_conflicts_ld",
+            "smem_bank_conflicts_st", "registers_per_thread", "smem_per_cta_kb", "duration_us_ncu")
+    out = {k: {f: e[f] for f in keys if f in e} for k, e in rec.items()
+           if isinstance(e, dict) and e.get("source_digest") == source_digest()}
+    return out or None
+
+
 def recorded_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on the
     current kernel sources; otherwise None."""
@@ -391,6 +406,9 @@ def run_ours(args):
     # the headline value; the recomputed S and dP of the dQ pass are not.)
     dkdv_tf = 2.0 * flops_fwd() / (dkdv_ms * 1e-3) / 1e12
     dq_tf = 1.5 * flops_fwd() / (dq_ms * 1e-3) / 1e12
+    # the preprocess kernel is HBM-bound: O and dO read (bf16), lse read, D and lse2 written
+    pre_bytes = B * H * N * (2 * D * 2 + 4 + 8)
+    pre_gbs = pre_bytes / (pre_ms * 1e-3) / 1e9
     per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf), "attn_bwd_dkdv_sm100_kernel": (dkdv_ms, dkdv_tf),
                   "attn_bwd_dq_sm100_kernel": (dq_ms, dq_tf)}
     dominant = max(per_kernel, key=lambda kname: per_kernel[kname][0])
@@ -421,6 +439,10 @@ def run_ours(args):
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "traffic": recorded_traffic(dominant),
                      "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src}, burst)"},
+        "hbm": {"kernel": "attn_bwd_pre_kernel", "achieved": pre_gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": pre_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": pre_bytes,
+                "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"},
+        "ncu_recorded": recorded_ncu(),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_n},
         "gpu_launches": 4 * args.steps,
