@@ -201,6 +201,20 @@ def e4m3_codes(x: torch.Tensor):
     return (x / factor).to(torch.float8_e4m3fn).view(torch.uint8), factor
 
 
+def make_fp8_varlen(lengths, H, d, seed, causal=True, scale: Optional[float] = None):
+    """Packed [total, H, d] e4m3 inputs (as ``make_fp8``) and cu_seqlens.  Returns
+    (Fp8Inputs with N = max length, cu_seqlens)."""
+    total = int(sum(lengths))
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(total, H, d, generator=g, dtype=torch.float32)
+    k = torch.randn(total, H, d, generator=g, dtype=torch.float32)
+    v = torch.randn(total, H, d, generator=g, dtype=torch.float32)
+    (q8, qs), (k8, ks), (v8, vs) = e4m3_codes(q), e4m3_codes(k), e4m3_codes(v)
+    inp = Fp8Inputs(q8, k8, v8, qs, ks, vs, len(lengths), H, max(lengths), d,
+                    scale if scale is not None else 1.0 / math.sqrt(d), causal)
+    return inp, cu_seqlens_of(lengths)
+
+
 def make_fp8(B, H, N, d, seed, causal=True, qk_sigma=1.0, scale: Optional[float] = None) -> Fp8Inputs:
     """N(0, sigma^2) float32 draws for Q, K (sigma = qk_sigma) and V (sigma 1), in
     that order, each quantised per tensor with ``e4m3_codes``."""

@@ -7,7 +7,8 @@ missing, importing the entry points raises.
 
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
 ``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
-``attn_fwd_blocksparse``, ``attn_bwd_blocksparse``, ``attn_fwd_fp8``,
+``attn_fwd_blocksparse``, ``attn_bwd_blocksparse``, ``attn_fwd_fp8``, ``attn_fwd_fp8_masked``,
+``attn_fwd_fp8_varlen``,
 ``attn_bwd_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
 ``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
@@ -66,13 +67,16 @@ def lib() -> ctypes.CDLL:
     L.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, sz, vp]
     L.attn_bwd_noalloc.restype = i
     L.attn_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp]
+    L.attn_fwd_fp8_masked.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp, vp]
+    L.attn_fwd_fp8_varlen.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
     L.attn_strerror.restype = ctypes.c_char_p
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
     for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen", "attn_bwd_phase",
-                 "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_status", "attn_set_wait_limit_ms",
+                 "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked",
+                 "attn_fwd_fp8_varlen", "attn_status", "attn_set_wait_limit_ms",
                  "attn_debug_skip_load"):
         getattr(L, name).restype = i
     _lib = L
@@ -289,25 +293,43 @@ def attn_bwd_blocksparse(q, k, v, o, lse, do, block_mask, dq=None, dk=None, dv=N
 
 
 def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None, lse=None, *,
-                 scale: Optional[float] = None, causal: bool = True, stream=None):
-    """FP8 forward.  q, k, v: dense [B,H,N,d] e4m3 codes (torch.float8_e4m3fn or uint8
-    views of them) whose values are code * {q,k,v}_scale.  Returns (o bf16, lse fp32)."""
+                 scale: Optional[float] = None, causal: bool = True, cu_seqlens: Optional[torch.Tensor] = None,
+                 key_keep: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None, stream=None):
+    """FP8 forward.  q, k, v: e4m3 codes (torch.float8_e4m3fn, or uint8 views of them)
+    whose values are code * {q,k,v}_scale, dense [B,H,N,d] or packed [total,H,d] with
+    ``cu_seqlens`` (int32, device) and ``max_seqlen``; optional per-key ``key_keep``.
+    Returns (o bf16, lse fp32)."""
     codes = (torch.float8_e4m3fn, torch.uint8)
-    _need(q, codes, "q")
-    if q.dim() != 4:
-        raise ValueError(f"q must be [B, H, N, d], got shape {tuple(q.shape)}")
-    _shaped(k, q.shape, codes, "k", q.device)
-    _shaped(v, q.shape, codes, "v", q.device)
-    B, H, N, d = q.shape
+    packed = cu_seqlens is not None
+    _inputs([("q", q), ("k", k), ("v", v)], codes, packed)
+    _side(q, cu_seqlens, key_keep, q.shape[0] if packed else q.shape[0] * q.shape[2])
+    d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o = torch.empty((B, H, N, d), device=q.device, dtype=torch.bfloat16) if o is None else o
-    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    o = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16) if o is None else o
     _shaped(o, q.shape, torch.bfloat16, "o", q.device)
-    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
-    rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale), float(v_scale), _ptr(o),
-                            _ptr(lse), B, H, N, d, float(scale), int(causal), _stream(stream))
-    _check(rc, "attn_fwd_fp8")
+    lse_shape = q.shape[:2] if packed else q.shape[:3]
+    lse = torch.empty(lse_shape, device=q.device, dtype=torch.float32) if lse is None else lse
+    _shaped(lse, lse_shape, torch.float32, "lse", q.device)
+    sc = (float(q_scale), float(k_scale), float(v_scale))
+    if packed:
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        total, H = q.shape[0], q.shape[1]
+        rc = lib().attn_fwd_fp8_varlen(_ptr(q), _ptr(k), _ptr(v), *sc, _ptr(o), _ptr(lse), cu_seqlens.numel() - 1,
+                                       total, int(max_seqlen), H, d, float(scale), int(causal), _ptr(cu_seqlens),
+                                       _ptr(key_keep), _stream(stream))
+        _check(rc, "attn_fwd_fp8_varlen")
+        return o, lse
+    B, H, N, _ = q.shape
+    if key_keep is None:
+        rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), *sc, _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                int(causal), _stream(stream))
+        _check(rc, "attn_fwd_fp8")
+    else:
+        rc = lib().attn_fwd_fp8_masked(_ptr(q), _ptr(k), _ptr(v), *sc, _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                                       int(causal), _ptr(key_keep), _stream(stream))
+        _check(rc, "attn_fwd_fp8_masked")
     return o, lse
 
 

@@ -180,7 +180,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
 }
 
 int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
-                 float *lse, const Shape &s, float scale, int is_causal, void *stream) {
+                 float *lse, const Shape &s, float scale, int is_causal, const uint8_t *key_keep, void *stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -192,13 +192,18 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
     DeviceState *ds = nullptr;
     if ((rc = device_state(&ds))) return rc;
     attn::FwdLaunch a{};
-    const long long slabs = static_cast<long long>(s.B) * s.H, slab_stride = static_cast<long long>(s.N) * s.d;
-    if ((rc = make_map_u8(&a.tm_q, q, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
-        (rc = make_map_u8(&a.tm_k, k, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
-        (rc = make_map_u8(&a.tm_v, v, s.d, s.N, slabs, s.d, slab_stride, 128)) ||
+    if (s.cu && s.total == 0) return ATTN_OK;  // nothing to do
+    // e4m3 maps with the bf16 maps' geometry (dense: slab b*H+h, row stride d; packed:
+    // slab h, rows = tokens, row stride H*d), in bytes
+    const long long rows = s.cu ? s.total : s.N, slabs = s.cu ? s.H : static_cast<long long>(s.B) * s.H;
+    const long long rstride = s.cu ? static_cast<long long>(s.H) * s.d : s.d;
+    const long long sstride = s.cu ? s.d : static_cast<long long>(s.N) * s.d;
+    if ((rc = make_map_u8(&a.tm_q, q, s.d, rows, slabs, rstride, sstride, 128)) ||
+        (rc = make_map_u8(&a.tm_k, k, s.d, rows, slabs, rstride, sstride, 128)) ||
+        (rc = make_map_u8(&a.tm_v, v, s.d, rows, slabs, rstride, sstride, 128)) ||
         (rc = map_for(&a.tm_o_st, o, s, 32, false, 32)))
         return rc;
-    a.g = geom_of(s, nullptr);
+    a.g = geom_of(s, key_keep);
     a.ctl = ctl_of(ds);
     a.o = o;
     a.lse = lse;
@@ -294,7 +299,22 @@ int attn_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, f
 int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
                  float *lse, int B, int H, int N, int d, float scale, int is_causal, void *stream) {
     Shape s{B, H, N, d, 0, nullptr};
-    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, stream);
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, nullptr, stream);
+}
+
+int attn_fwd_fp8_masked(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale,
+                        void *o, float *lse, int B, int H, int N, int d, float scale, int is_causal,
+                        const uint8_t *key_keep, void *stream) {
+    Shape s{B, H, N, d, 0, nullptr};
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, key_keep, stream);
+}
+
+int attn_fwd_fp8_varlen(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale,
+                        void *o, float *lse, int num_seqs, int total_tokens, int max_seqlen, int H, int d, float scale,
+                        int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep, void *stream) {
+    if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
+    Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, key_keep, stream);
 }
 
 int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,

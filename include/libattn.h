@@ -217,6 +217,26 @@ ATTN_API int attn_fwd_fp8(const void *q, const void *k, const void *v, float q_s
                           float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
                           int is_causal, void *stream);
 
+/*
+ * FP8 forward with a per-key padding mask (key_keep, nullable DEVICE uint8 [B, N],
+ * as for attn_fwd_masked), dense layout.  Other arguments as attn_fwd_fp8.
+ */
+ATTN_API int attn_fwd_fp8_masked(const void *q, const void *k, const void *v, float q_scale, float k_scale,
+                                 float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
+                                 int is_causal, const uint8_t *key_keep, void *stream);
+
+/*
+ * FP8 forward on the packed variable-length layout: q, k, v are e4m3 codes
+ * [total_tokens, H, d], o is bf16 [total_tokens, H, d], lse fp32 [total_tokens, H];
+ * num_seqs, total_tokens, max_seqlen, cu_seqlens (DEVICE int32, must not be NULL)
+ * and key_keep (nullable, [total_tokens]) as for attn_fwd_varlen.  Other arguments
+ * as attn_fwd_fp8.
+ */
+ATTN_API int attn_fwd_fp8_varlen(const void *q, const void *k, const void *v, float q_scale, float k_scale,
+                                 float v_scale, void *o, float *lse, int num_seqs, int total_tokens, int max_seqlen,
+                                 int H, int d, float scale, int is_causal, const int32_t *cu_seqlens,
+                                 const uint8_t *key_keep, void *stream);
+
 /* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

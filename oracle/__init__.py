@@ -170,9 +170,11 @@ def e4m3_decode(codes, factor=1.0):
     return out
 
 
-def fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale, causal, slices=None, nthreads=None):
-    """Forward of dense [B,H,N,d] e4m3 inputs: the attention of the decoded values
-    (code value x per-tensor factor).  Returns (o, lse) float64 like ``fwd``."""
+def fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale, causal, cu_seqlens=None, key_keep=None, slices=None,
+            nthreads=None, N=None):
+    """Forward of e4m3 inputs (dense [B,H,N,d] or packed [total,H,d] with cu_seqlens):
+    the attention of the decoded values (code value x per-tensor factor), with the
+    same masks as ``fwd``.  Returns (o, lse) float64 like ``fwd``."""
     return fwd(e4m3_decode(q8, q_scale), e4m3_decode(k8, k_scale), e4m3_decode(v8, v_scale), scale, causal,
-               slices=slices, nthreads=nthreads)
+               cu_seqlens=cu_seqlens, key_keep=key_keep, slices=slices, nthreads=nthreads, N=N)
 

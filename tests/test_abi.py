@@ -28,7 +28,7 @@ def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
               "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen", "attn_fwd_blocksparse",
-              "attn_bwd_blocksparse", "attn_fwd_fp8"):
+              "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked", "attn_fwd_fp8_varlen"):
         assert n in names
 
 
@@ -126,6 +126,12 @@ def test_fp8_host_argument_errors(L):
     assert call(ptrs=(FAKE, FAKE, FAKE + 4, FAKE, FAKE)) == ea.ATTN_ERR_MISALIGNED
     assert call(ptrs=(FAKE, FAKE, FAKE, FAKE, FAKE + 8)) == ea.ATTN_ERR_MISALIGNED
     assert call(B=0) == ea.ATTN_ERR_INVALID_ARG
+    # packed layout: cu_seqlens is required; masked dense layout: d must still be 128
+    p5 = [vp(FAKE)] * 3
+    assert L.attn_fwd_fp8_varlen(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 2, 100, 64, 1, 128, f(0.1), 1,
+                                 None, None, None) == ea.ATTN_ERR_INVALID_ARG
+    assert L.attn_fwd_fp8_masked(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 1, 1, 256, 64, f(0.1), 1,
+                                 vp(FAKE), None) == ea.ATTN_ERR_UNSUPPORTED
 
 
 def test_wait_limit_and_fault_hook_setters(L):

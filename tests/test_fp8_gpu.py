@@ -42,51 +42,70 @@ def ea():
     return m
 
 
-def gpu_fp8(ea, inp, causal=None):
+def gpu_fp8(ea, inp, causal=None, key_keep=None, cu_seqlens=None):
     causal = inp.causal if causal is None else causal
     q8, k8, v8 = inp.q8.cuda(), inp.k8.cuda(), inp.v8.cuda()
-    o = torch.full((inp.B, inp.H, inp.N, inp.d), float("nan"), device="cuda", dtype=torch.bfloat16)
-    lse = torch.full((inp.B, inp.H, inp.N), float("nan"), device="cuda")
-    ea.attn_fwd_fp8(q8, k8, v8, inp.q_scale, inp.k_scale, inp.v_scale, o, lse, scale=inp.scale, causal=causal)
+    o = torch.full(q8.shape, float("nan"), device="cuda", dtype=torch.bfloat16)
+    lse = torch.full(q8.shape[:2] if cu_seqlens is not None else q8.shape[:3], float("nan"), device="cuda")
+    kw = {}
+    if cu_seqlens is not None:
+        kw = dict(cu_seqlens=cu_seqlens.cuda(), max_seqlen=inp.N)
+    ea.attn_fwd_fp8(q8, k8, v8, inp.q_scale, inp.k_scale, inp.v_scale, o, lse, scale=inp.scale, causal=causal,
+                    key_keep=None if key_keep is None else key_keep.cuda(), **kw)
     assert ea.attn_status() == ea.ATTN_OK
     return o.double().cpu().numpy(), lse.double().cpu().numpy()
 
 
-def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref):
-    """Elementwise error bound for one (b, h) slice (float64 numpy, n x d)."""
+def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref, keep=None):
+    """Elementwise error bound for one (sequence, head) slice (float64 numpy, n x d),
+    over the rows that see at least one key (the others are checked exactly)."""
     n = qd.shape[0]
     S = scale * (qd @ kd.T)
     if causal:
         S[np.triu_indices(n, 1)] = -np.inf
+    if keep is not None:
+        S[:, ~keep] = -np.inf
+    live = np.isfinite(lse_ref)
+    S, o_l, lse_l = S[live], o_ref[live], lse_ref[live]
     m = S.max(axis=1)
-    W = np.exp(S - lse_ref[:, None])
-    lp = np.exp(lse_ref - m)
+    W = np.exp(S - lse_l[:, None])
+    lp = np.exp(lse_l - m)
     E = np.where(np.isfinite(S), np.maximum((2.0 ** -4 + 2.0 ** -12) * W, (2.0 ** -10 / lp)[:, None]), 0.0)
     A = np.abs(vd)
-    return E @ A + S_ALLOW * (W @ A + np.abs(o_ref)) + (2.0 ** -8 + 2.0 ** -13) * np.abs(o_ref) + 1e-6
+    tol = np.zeros_like(o_ref)
+    tol[live] = E @ A + S_ALLOW * (W @ A + np.abs(o_l)) + (2.0 ** -8 + 2.0 ** -13) * np.abs(o_l) + 1e-6
+    return tol, live
 
 
-def check(inp, got_o, got_l, causal, slices=None):
+def check_slice(tag, qd, kd, vd, scale, causal, got_o, got_l, ro, rl, keep=None):
+    tol, live = bound_slice(qd, kd, vd, scale, causal, ro, rl, keep)
+    assert not np.isnan(got_o).any(), f"NaN in {tag}"
+    # rows that see no key: exactly O = 0 and lse = -inf
+    assert np.all(got_o[~live] == 0.0) and np.all(np.isneginf(got_l[~live])), f"{tag}: empty rows"
+    err = np.abs(got_o - ro)
+    bad = (err > tol) & live[:, None]
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(live[:, None], err - tol, -np.inf)), err.shape)
+        raise AssertionError(f"{tag}: {bad.sum()} elements out of bound; worst at {i}: gpu {got_o[i]} ref {ro[i]} "
+                             f"bound {tol[i]}")
+    lerr = np.abs(got_l[live] - rl[live])
+    assert lerr.size == 0 or lerr.max() <= LSE_ATOL, f"{tag}: lse err {lerr.max()}"
+    return float((err[live] / tol[live]).max()) if live.any() else 0.0
+
+
+def check(inp, got_o, got_l, causal, slices=None, key_keep=None):
+    keep = None if key_keep is None else key_keep.numpy().astype(bool)
     ro, rl = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, inp.v_scale, inp.scale, causal,
-                            slices=slices)
+                            key_keep=key_keep, slices=slices)
     qd = oracle.e4m3_decode(inp.q8, inp.q_scale)
     kd = oracle.e4m3_decode(inp.k8, inp.k_scale)
     vd = oracle.e4m3_decode(inp.v8, inp.v_scale)
-    todo = slices if slices is not None else range(inp.B * inp.H)
     worst = 0.0
-    for sidx in todo:
+    for sidx in (slices if slices is not None else range(inp.B * inp.H)):
         b, h = divmod(int(sidx), inp.H)
-        tol = bound_slice(qd[b, h], kd[b, h], vd[b, h], inp.scale, causal, ro[b, h], rl[b, h])
-        err = np.abs(got_o[b, h] - ro[b, h])
-        assert not np.isnan(got_o[b, h]).any(), f"NaN in slice {sidx}"
-        bad = err > tol
-        if bad.any():
-            i = np.unravel_index(np.argmax(err - tol), err.shape)
-            raise AssertionError(f"slice {sidx}: {bad.sum()} elements out of bound; worst at {i}: gpu {got_o[b, h][i]} "
-                                 f"ref {ro[b, h][i]} bound {tol[i]}")
-        worst = max(worst, float((err / tol).max()))
-        lerr = np.abs(got_l[b, h] - rl[b, h])
-        assert lerr.max() <= LSE_ATOL, f"slice {sidx}: lse err {lerr.max()}"
+        worst = max(worst, check_slice(f"slice {sidx}", qd[b, h], kd[b, h], vd[b, h], inp.scale, causal,
+                                       got_o[b, h], got_l[b, h], ro[b, h], rl[b, h],
+                                       None if keep is None else keep[b]))
     return worst
 
 
@@ -151,3 +170,39 @@ def test_fp8_full_size_sampled_slices(ea):
     inp = make_fp8(2, 16, 4096, 128, seed=8260, causal=True)
     o, l = gpu_fp8(ea, inp)
     check(inp, o, l, True, slices=[0, 13, 31])
+
+
+def test_fp8_dense_key_mask_with_empty_rows(ea):
+    # the first 40 keys of sequence 0 are padding: under causal masking its first 40
+    # query rows see no key (O = 0, lse = -inf); a scattering of other keys is masked
+    from attn_inputs import make_fp8
+    inp = make_fp8(2, 2, 300, 128, seed=8270, causal=True)
+    g = torch.Generator("cpu").manual_seed(8271)
+    keep = (torch.rand(2, 300, generator=g) > 0.1).to(torch.uint8)
+    keep[0, :40] = 0
+    keep[1, 0] = 1
+    o, l = gpu_fp8(ea, inp, key_keep=keep)
+    check(inp, o, l, True, key_keep=keep)
+    assert np.all(o[0, :, :40] == 0.0) and np.all(np.isneginf(l[0, :, :40]))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_varlen_with_padding_mask(ea, causal):
+    from attn_inputs import make_fp8_varlen, padding_key_mask
+    lengths = [300, 129, 1, 517, 128]
+    inp, cu = make_fp8_varlen(lengths, 2, 128, seed=8280, causal=causal)
+    keep = padding_key_mask(lengths, seed=8281)
+    o, l = gpu_fp8(ea, inp, key_keep=keep, cu_seqlens=cu)
+    ro, rl = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, inp.v_scale, inp.scale, causal,
+                            cu_seqlens=cu, key_keep=keep, N=inp.N)
+    qd = oracle.e4m3_decode(inp.q8, inp.q_scale)
+    kd = oracle.e4m3_decode(inp.k8, inp.k_scale)
+    vd = oracle.e4m3_decode(inp.v8, inp.v_scale)
+    kp = keep.numpy().astype(bool)
+    cuv = cu.tolist()
+    for b in range(len(lengths)):
+        st, en = cuv[b], cuv[b + 1]
+        for h in range(2):
+            check_slice(f"seq {b} head {h}", qd[st:en, h], kd[st:en, h], vd[st:en, h], inp.scale, causal,
+                        o[st:en, h], l[st:en, h], ro[st:en, h], rl[st:en, h], kp[st:en])
+
