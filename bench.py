@@ -119,12 +119,18 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
+_ORACLE_INPUTS = None
+
+
 def time_oracle_sample(n_heads: int):
     """float64 oracle forward + backward on the first n_heads (b, h) slices of the
     workload, all host cores.  Returns (TFLOPS, seconds, cores, sample text)."""
     import oracle
-    from attn_inputs import make_dense
-    inp = make_dense(B, H, N, D, seed=SEED, causal=CAUSAL, with_grad=True)
+    global _ORACLE_INPUTS
+    if _ORACLE_INPUTS is None:  # drawn once, reused by every timed sample
+        from attn_inputs import make_dense
+        _ORACLE_INPUTS = make_dense(B, H, N, D, seed=SEED, causal=CAUSAL, with_grad=True)
+    inp = _ORACLE_INPUTS
     threads = oracle.default_threads()
     picks = list(range(n_heads))
     t0 = time.perf_counter()

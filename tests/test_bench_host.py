@@ -1,0 +1,75 @@
+"""Host-side logic of bench.py that needs no GPU: the FLOP conventions, the digest
+that ties committed ncu counters to the kernel code, and the reference arm's line."""
+import importlib.util
+import json
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_flop_conventions(bench):
+    # forward 2*B*H*N^2*d causal (4* non-causal), backward credited 2.5x the forward
+    assert bench.flops_fwd() == 2.0 * 2 * 16 * 4096 ** 2 * 128 == pytest.approx(137.44e9, rel=1e-3)
+    assert bench.flops_fwd(causal=False) == 2 * bench.flops_fwd()
+    assert bench.flops_bwd() == 2.5 * bench.flops_fwd()
+
+
+def _copy_sources(tmp_path):
+    dst = tmp_path / "exact_attention_123_b200" / "csrc"
+    shutil.copytree(os.path.join(ROOT, "exact_attention_123_b200", "csrc"), dst,
+                    ignore=shutil.ignore_patterns("*.o", "*.so"))
+    return dst
+
+
+def test_digest_ignores_comments_but_not_code(bench, tmp_path, monkeypatch):
+    base = bench.source_digest()
+    src = _copy_sources(tmp_path)
+    monkeypatch.setattr(bench, "HERE", str(tmp_path))
+    assert bench.source_digest() == base
+    f = src / "attn_fwd_sm100.cu"
+    text = f.read_text(encoding="utf-8")
+    f.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n", "\n\n", 3),
+                 encoding="utf-8")
+    assert bench.source_digest() == base
+    f.write_text(text.replace("kRescaleThreshold = 8.0f", "kRescaleThreshold = 9.0f"), encoding="utf-8")
+    assert bench.source_digest() != base
+
+
+def test_recorded_counters_only_for_matching_code(bench, tmp_path, monkeypatch):
+    _copy_sources(tmp_path)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "HERE", str(tmp_path))
+    good = bench.source_digest()
+    rec = {"k_match": {"source_digest": good, "dram_bytes_per_launch": 123, "tensor_pipe_active_pct": 50.0},
+           "k_stale": {"source_digest": "0000000000000000", "dram_bytes_per_launch": 456}}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("k_match") == 123
+    assert bench.recorded_traffic("k_stale") is None
+    assert bench.recorded_traffic("absent") is None
+    got = bench.recorded_ncu()
+    assert set(got) == {"k_match"} and got["k_match"]["tensor_pipe_active_pct"] == 50.0
+
+
+def test_reference_arm_prints_the_contract_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOPS" and line["value"] > 0
+    assert line["higher_is_better"] is True and line["steps"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
