@@ -23,6 +23,7 @@ import math
 import os
 import re
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -189,8 +190,9 @@ def recorded_ncu():
         return None
     with open(p) as f:
         rec = json.load(f)
-    keys = ("tensor_pipe_active_pct", "hbm_gbs", "dram_bytes_per_launch", "smem_bank_conflicts_ld",
-            "smem_bank_conflicts_st", "registers_per_thread", "smem_per_cta_kb", "duration_us_ncu")
+    keys = ("tensor_pipe_active_pct", "mufu_pipe_active_pct", "issue_active_pct", "hbm_gbs", "dram_bytes_per_launch",
+            "l2_hit_pct", "smem_bank_conflicts_ld", "smem_bank_conflicts_st", "registers_per_thread", "smem_per_cta_kb",
+            "duration_us_ncu")
     out = {k: {f: e[f] for f in keys if f in e} for k, e in rec.items()
            if isinstance(e, dict) and e.get("source_digest") == source_digest()}
     return out or None
@@ -481,6 +483,85 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- ncu reports
+# Figures read from one `ncu --set full` capture (raw page, CSV), per kernel launch.
+NCU_METRICS = {
+    "duration_us_ncu": ("gpu__time_duration.sum", "us"),
+    "dram_read": ("dram__bytes_read.sum", "bytes"),
+    "dram_write": ("dram__bytes_write.sum", "bytes"),
+    "tensor_pipe_active_pct": ("sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed", None),
+    "mufu_pipe_active_pct": ("sm__inst_executed_pipe_xu.avg.pct_of_peak_sustained_active", None),
+    "issue_active_pct": ("smsp__issue_active.avg.pct_of_peak_sustained_active", None),
+    "l2_hit_pct": ("lts__t_sector_hit_rate.pct", None),
+    "warp_instructions": ("smsp__inst_executed.sum", None),
+    "smem_bank_conflicts_ld": ("l1tex__data_bank_conflicts_pipe_lsu_mem_shared_op_ld.sum", None),
+    "smem_bank_conflicts_st": ("l1tex__data_bank_conflicts_pipe_lsu_mem_shared_op_st.sum", None),
+    "registers_per_thread": ("launch__registers_per_thread", None),
+    "smem_per_cta_kb": ("launch__shared_mem_per_block_dynamic", "kb"),
+}
+_SCALE = {"us": {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6},
+          "bytes": {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9},
+          "kb": {"byte": 1e-3, "Kbyte": 1.0, "Mbyte": 1e3}}
+
+
+def ncu_kernel_key(name: str) -> str:
+    """Record key of a kernel: the bare name for the dense bf16 d=128 instantiations
+    the bench times, the name with its template arguments otherwise."""
+    base = name.split("(")[0].replace("void ", "").replace("attn::", "").strip()
+    short, _, args = base.partition("<")
+    return short if args.rstrip(">") in ("128, 0", "128, 0, 0") else base
+
+
+def ncu_rows(csv_text: str):
+    """Per-launch figures from `ncu -i REPORT --page raw --csv` output."""
+    import csv
+    import io
+    rows = list(csv.reader(io.StringIO(csv_text)))
+    head, units = rows[0], rows[1]
+    col = {h: i for i, h in enumerate(head)}
+    out = []
+    for r in rows[2:]:
+        if len(r) != len(head):
+            continue
+        e = {"kernel": ncu_kernel_key(r[col["Kernel Name"]])}
+        for key, (metric, kind) in NCU_METRICS.items():
+            if metric not in col or r[col[metric]] in ("", "n/a"):
+                continue
+            v = float(r[col[metric]].replace(",", ""))
+            if kind:
+                v *= _SCALE[kind].get(units[col[metric]], 1.0)
+            e[key] = v
+        if "dram_read" in e and "dram_write" in e:
+            e["dram_bytes_per_launch"] = int(round(e["dram_read"] + e["dram_write"]))
+            if e.get("duration_us_ncu"):
+                e["hbm_gbs"] = e["dram_bytes_per_launch"] / (e["duration_us_ncu"] * 1e-6) / 1e9
+        out.append(e)
+    return out
+
+
+def ncu_summary(report: str, record: bool) -> int:
+    """Print one JSON line per captured launch; with `record`, store them in
+    profiles/ncu_traffic.json under the current kernel-code digest."""
+    text = subprocess.run(["ncu", "-i", report, "--page", "raw", "--csv"], capture_output=True, text=True,
+                          check=True).stdout
+    rows = ncu_rows(text)
+    for e in rows:
+        print(json.dumps(e), flush=True)
+    if record:
+        p = os.path.join(HERE, "profiles", "ncu_traffic.json")
+        rec = json.load(open(p)) if os.path.exists(p) else {}
+        dg = source_digest()
+        rec["source_digest"] = dg
+        for e in rows:
+            ent = {k: v for k, v in e.items() if k != "kernel"}
+            ent["source_digest"] = dg
+            rec[e["kernel"]] = ent
+        with open(p, "w") as f:
+            json.dump(rec, f, indent=2)
+            f.write("\n")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -493,7 +574,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward's timing")
+    ap.add_argument("--ncu-summary", metavar="REPORT",
+                    help="print the per-kernel figures of an ncu --set full report (no GPU needed) and exit")
+    ap.add_argument("--record", action="store_true",
+                    help="with --ncu-summary: store them in profiles/ncu_traffic.json for the current kernel code")
     args = ap.parse_args()
+    if args.ncu_summary:
+        return ncu_summary(args.ncu_summary, args.record)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

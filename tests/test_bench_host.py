@@ -73,3 +73,25 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_ncu_report_rows(bench):
+    # the raw-page CSV of `ncu -i REPORT --page raw --csv`: a header row, a units row,
+    # then one row per captured launch
+    head = ["ID", "Kernel Name", "gpu__time_duration.sum", "dram__bytes_read.sum", "dram__bytes_write.sum",
+            "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed",
+            "launch__shared_mem_per_block_dynamic", "l1tex__data_bank_conflicts_pipe_lsu_mem_shared_op_st.sum"]
+    units = ["", "", "usecond", "Mbyte", "Kbyte", "%", "Kbyte", ""]
+    rows = [["0", "void attn::attn_bwd_dkdv_sm100_kernel<128, 0>(CUtensorMap_st, BwdParams)", "200", "150.5",
+             "2,048", "51.5", "216.184", "7"],
+            ["1", "void attn::attn_fwd_sm100_kernel<128, 0, 1>(CUtensorMap_st, FwdParams)", "100", "50", "5",
+             "27.5", "214.2", "0"]]
+    text = "\n".join(",".join(f'"{c}"' for c in r) for r in [head, units] + rows)
+    got = bench.ncu_rows(text)
+    assert [e["kernel"] for e in got] == ["attn_bwd_dkdv_sm100_kernel", "attn_fwd_sm100_kernel<128, 0, 1>"]
+    e = got[0]
+    assert e["dram_bytes_per_launch"] == 150_500_000 + 2_048_000
+    assert e["hbm_gbs"] == pytest.approx(152_548_000 / 200e-6 / 1e9)
+    assert e["tensor_pipe_active_pct"] == 51.5 and e["smem_per_cta_kb"] == 216.184
+    assert e["smem_bank_conflicts_st"] == 7
+    assert bench.ncu_kernel_key("void attn::attn_fwd_sm100_kernel<64, 1, 0>(X)") == "attn_fwd_sm100_kernel<64, 1, 0>"
