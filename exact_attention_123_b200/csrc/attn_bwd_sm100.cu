@@ -35,6 +35,9 @@
 // still writing the previous unit's result.
 // Every product is a full 128 x 128 (x d) tensor-core tile; the extra S and dP
 // products of the dQ pass cost less than the reductions they replace.
+// With a tile mask (block-sparse attention, the SP instantiations) a unit sweeps only
+// the partner tiles the mask keeps; a unit left with none writes zeros and computes
+// nothing.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -49,9 +52,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // ============================================================================ preprocess
 // One row of d elements per (d/8) threads (16 bytes of O and of dO each); a CTA
-// covers kPreRows consecutive rows in kPreRows / (256 / (d/8)) passes whose loads
-// are all issued before any is used, so that each thread keeps several loads in
-// flight (the kernel is HBM-bound).  Rows are in the lse layout order, which is
+// covers kPrePasses passes of 256 / (d/8) consecutive rows, whose loads are all
+// issued before any is used, so that each thread keeps several loads in flight (the
+// kernel is HBM-bound).  Rows are in the lse layout order, which is
 // also the row order of the flat [rows, d] view of O and dO.
 constexpr int kPrePasses = 4;
 template <int D>
