@@ -91,19 +91,20 @@ int make_map(CUtensorMap *m, const void *base, int d, long long rows, long long 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// 3-D map over e4m3 bytes: `cols` bytes per row (contiguous), box {128, box_rows, 1}
-// with the 128-byte swizzle.
+// 3-D map over e4m3 bytes: `cols` bytes per row (contiguous), box {cols, box_rows, 1}
+// with the 128-byte swizzle for 128-byte rows and the 64-byte swizzle for 64-byte rows.
 int make_map_u8(CUtensorMap *m, const void *base, long long cols, long long rows, long long slabs,
                 long long row_stride, long long slab_stride, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return ATTN_ERR_CUDA;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride), static_cast<cuuint64_t>(slab_stride)};
-    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), 1u};
+    if (cols != 64 && cols != 128) return ATTN_ERR_UNSUPPORTED;
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(cols), static_cast<cuuint32_t>(box_rows), 1u};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -186,7 +187,6 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
     if (rc) return rc;
     for (float f : {q_scale, k_scale, v_scale})
         if (!(f > 0.f) || !std::isfinite(f)) return ATTN_ERR_INVALID_ARG;
-    if (s.d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_MISALIGNED;
     DeviceState *ds = nullptr;

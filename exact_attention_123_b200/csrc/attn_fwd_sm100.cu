@@ -62,10 +62,11 @@ template <int D, bool F8 = false>
 struct FwdCfg {
     static constexpr int kEsz = F8 ? 1 : 2;                // bytes per Q/K/V element
     static constexpr int kTileBytes = 128 * D * kEsz;      // one 128-row tile
-    static constexpr int kBoxes = D * kEsz / 128;          // 128-byte-swizzle boxes per tile
+    // swizzled boxes per tile: 64-column bf16 boxes (128-byte swizzle); one e4m3 box of
+    // d bytes per row (128-byte swizzle at d = 128, 64-byte swizzle at d = 64)
+    static constexpr int kBoxes = F8 ? 1 : D / 64;
     static constexpr int kKSteps = D * kEsz / 32;          // 32-byte K steps of S = Q K^T
-    static constexpr int kStages = F8 ? 8 : (D == 128) ? 4 : 8;
-    static_assert(!F8 || D == 128, "the e4m3 path has 128-byte rows (d = 128)");
+    static constexpr int kStages = F8 ? (D == 128 ? 8 : 16) : (D == 128) ? 4 : 8;
     // 3 warpgroups: two softmax groups, and one with the TMA producer, the MMA issuer
     // and two idle warps (registers move by whole warpgroups).  Launched at 168
     // registers per thread (the most 384 threads allow), the control group gives
@@ -245,6 +246,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D, 1) : idesc_bf16_f32(128, D, 0, 1);
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
+            // K-major operand descriptor of a Q or K tile (e4m3 at d = 64: 64-byte rows)
+            auto kdesc = [](uint32_t a) -> uint64_t {
+                if constexpr (F8 && D == 64) return sw64_desc(a, 16, 512);
+                else return sw128_desc(a, 16, 1024);
+            };
             // S_t from the K tile at ring position kpos
             auto issue_S = [&](int t, int kpos) {
                 const uint32_t qs = sbase + t * C::kTileBytes;
@@ -253,8 +259,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                     if constexpr (F8)
-                        mma_ss_f8(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024),
-                                  idS, kk > 0);
+                        mma_ss_f8(tmem + colS[t], kdesc(qs + off), kdesc(ks + off), idS, kk > 0);
                     else
                         mma_ss(tmem + colS[t], sw128_desc(qs + off, 16, 1024), sw128_desc(ks + off, 16, 1024), idS,
                                kk > 0);
@@ -266,12 +271,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint32_t vs = slot(vpos % C::kStages);
                 if constexpr (F8) {
                     // A = P_t (shared memory, 128 queries x 128 keys, K-major), B = V (128 keys
-                    // x d, MN-major: each 32-key step is 32 rows of 128 bytes)
+                    // x d, MN-major: each 32-key step is 32 rows of d bytes)
                     const uint32_t ps = sbase + C::kOffP + t * 16384;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss_f8(tmem + colO[t], sw128_desc(ps + kk * 32, 16, 1024),
-                                  sw128_desc(vs + kk * 4096, 16384, 1024), idPV, (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bdesc = (D == 64) ? sw64_desc(vs + kk * 2048, 16384, 512)
+                                                         : sw128_desc(vs + kk * 4096, 16384, 1024);
+                        mma_ss_f8(tmem + colO[t], sw128_desc(ps + kk * 32, 16, 1024), bdesc, idPV,
+                                  (acc || kk > 0) ? 1u : 0u);
+                    }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
@@ -616,8 +624,9 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
-    if (a.g.d != 128) return cudaErrorInvalidValue;
-    return launch_fwd_d<128, false, true>(a, stream);
+    if (a.g.d == 128) return launch_fwd_d<128, false, true>(a, stream);
+    if (a.g.d == 64) return launch_fwd_d<64, false, true>(a, stream);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {

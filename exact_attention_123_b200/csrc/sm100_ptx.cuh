@@ -207,6 +207,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
     d |= static_cast<uint64_t>(2) << 61;
     return d;
 }
+// The same for tiles with the 64-byte swizzle (layout code 4): rows of 64 bytes,
+// 8-row groups 512 bytes apart (K-major: SBO = 512; MN-major: one 64-byte atom
+// along N, SBO = 512 between 8-row groups along K).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(4) << 61;
+    return d;
+}
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D:
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),

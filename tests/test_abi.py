@@ -122,15 +122,15 @@ def test_fp8_host_argument_errors(L):
     assert call(scales=(1.0, 0.0, 1.0)) == ea.ATTN_ERR_INVALID_ARG
     assert call(scales=(1.0, 1.0, float("inf"))) == ea.ATTN_ERR_INVALID_ARG
     assert call(scale=-1.0) == ea.ATTN_ERR_INVALID_ARG
-    assert call(d=64) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(d=96) == ea.ATTN_ERR_UNSUPPORTED
     assert call(ptrs=(FAKE, FAKE, FAKE + 4, FAKE, FAKE)) == ea.ATTN_ERR_MISALIGNED
     assert call(ptrs=(FAKE, FAKE, FAKE, FAKE, FAKE + 8)) == ea.ATTN_ERR_MISALIGNED
     assert call(B=0) == ea.ATTN_ERR_INVALID_ARG
-    # packed layout: cu_seqlens is required; masked dense layout: d must still be 128
+    # packed layout: cu_seqlens is required; masked dense layout: d must be 64 or 128
     p5 = [vp(FAKE)] * 3
     assert L.attn_fwd_fp8_varlen(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 2, 100, 64, 1, 128, f(0.1), 1,
                                  None, None, None) == ea.ATTN_ERR_INVALID_ARG
-    assert L.attn_fwd_fp8_masked(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 1, 1, 256, 64, f(0.1), 1,
+    assert L.attn_fwd_fp8_masked(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 1, 1, 256, 96, f(0.1), 1,
                                  vp(FAKE), None) == ea.ATTN_ERR_UNSUPPORTED
 
 

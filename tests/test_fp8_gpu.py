@@ -109,10 +109,11 @@ def check(inp, got_o, got_l, causal, slices=None, key_keep=None):
     return worst
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_ragged_tiles(ea, causal):
+def test_fp8_ragged_tiles(ea, causal, d):
     # 5 query tiles: two full 256-row units and a half one; keys end mid-tile too
-    inp = make_fp8(1, 2, 640 - 37, 128, seed=8200, causal=causal)
+    inp = make_fp8(1, 2, 640 - 37, d, seed=8200 + d, causal=causal)
     o, l = gpu_fp8(ea, inp)
     check(inp, o, l, causal)
 
@@ -130,10 +131,11 @@ def test_fp8_edge_lengths(ea, N):
     check(inp, o, l, True)
 
 
-def test_fp8_wide_scores_exercise_rescaling(ea):
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_wide_scores_exercise_rescaling(ea, d):
     # Q, K ~ N(0, 4^2): scores spread over tens of units, so running maxima move by
     # more than the lazy-rescale threshold and P values reach far below 2^-6
-    inp = make_fp8(1, 2, 512, 128, seed=8220, causal=True, qk_sigma=4.0)
+    inp = make_fp8(1, 2, 512, d, seed=8220 + d, causal=True, qk_sigma=4.0)
     o, l = gpu_fp8(ea, inp)
     check(inp, o, l, True)
 
@@ -204,5 +206,39 @@ def test_fp8_varlen_with_padding_mask(ea, causal):
         st, en = cuv[b], cuv[b + 1]
         for h in range(2):
             check_slice(f"seq {b} head {h}", qd[st:en, h], kd[st:en, h], vd[st:en, h], inp.scale, causal,
+                        o[st:en, h], l[st:en, h], ro[st:en, h], rl[st:en, h], kp[st:en])
+
+
+@pytest.mark.parametrize("N", [1, 129])
+def test_fp8_d64_edge_lengths(ea, N):
+    inp = make_fp8(1, 1, N, 64, seed=8290 + N, causal=True)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, True)
+
+
+def test_fp8_d64_full_size_sampled_slices(ea):
+    # the pages' sequence length at d = 64 (causal, B4 H16 N2048), sampled slices
+    inp = make_fp8(4, 16, 2048, 64, seed=8295, causal=True)
+    o, l = gpu_fp8(ea, inp)
+    check(inp, o, l, True, slices=[0, 37, 63])
+
+
+def test_fp8_d64_varlen_with_padding_mask(ea):
+    from attn_inputs import make_fp8_varlen, padding_key_mask
+    lengths = [300, 1, 517, 129]
+    inp, cu = make_fp8_varlen(lengths, 2, 64, seed=8296, causal=True)
+    keep = padding_key_mask(lengths, seed=8297)
+    o, l = gpu_fp8(ea, inp, key_keep=keep, cu_seqlens=cu)
+    ro, rl = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, inp.v_scale, inp.scale, True,
+                            cu_seqlens=cu, key_keep=keep, N=inp.N)
+    qd = oracle.e4m3_decode(inp.q8, inp.q_scale)
+    kd = oracle.e4m3_decode(inp.k8, inp.k_scale)
+    vd = oracle.e4m3_decode(inp.v8, inp.v_scale)
+    kp = keep.numpy().astype(bool)
+    cuv = cu.tolist()
+    for b in range(len(lengths)):
+        st, en = cuv[b], cuv[b + 1]
+        for h in range(2):
+            check_slice(f"seq {b} head {h}", qd[st:en, h], kd[st:en, h], vd[st:en, h], inp.scale, True,
                         o[st:en, h], l[st:en, h], ro[st:en, h], rl[st:en, h], kp[st:en])
 
