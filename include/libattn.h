@@ -207,7 +207,7 @@ ATTN_API int attn_bwd_blocksparse(const void *q, const void *k, const void *v, c
  *   o        : output (bf16) [B, H, N, d];  lse : output (fp32) [B, H, N], as for
  *              attn_fwd (natural-log logsumexp of the scaled dequantised scores).
  *   scale, is_causal : as for attn_fwd (dense layout, no key mask).
- * d must be 128 (ATTN_ERR_UNSUPPORTED otherwise).  Nothing is allocated and no
+ * d must be 64 or 128 (ATTN_ERR_UNSUPPORTED otherwise).  Nothing is allocated and no
  * workspace is needed.  Rounding beyond attn_fwd's: the probabilities enter P V as
  * e4m3 (half an e4m3 step: 2^-4 relative, or 2^-10 absolute below 2^-6, on the
  * kernel's scale, where the row sum is at least 1), after exponentials accurate to
