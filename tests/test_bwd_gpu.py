@@ -153,6 +153,24 @@ def test_full_size_sampled(ea):
         assert torch.isfinite(t.float()).all()
 
 
+@pytest.mark.parametrize("shape,causal", [((2, 16, 4096, 128), False), ((4, 16, 2048, 64), True),
+                                          ((4, 16, 2048, 64), False)])
+def test_full_size_other_configs_sampled(ea, shape, causal):
+    # the bench shape without the causal mask, and the pages' sequence length at d = 64
+    B, H, N, d = shape
+    inp = make_dense(B, H, N, d, seed=5300 + d + int(causal), causal=causal, with_grad=True)
+    dq, dk, dv = gpu_fwd_bwd(ea, inp, causal)
+    picks = [3, B * H - 2]
+    rq, rk, rv = oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, causal, slices=picks)
+    for s in picks:
+        b, h = divmod(s, H)
+        assert_grad(dq[b, h], rq[b, h], f"dQ slice {s}")
+        assert_grad(dk[b, h], rk[b, h], f"dK slice {s}")
+        assert_grad(dv[b, h], rv[b, h], f"dV slice {s}")
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+
+
 def test_full_size_varlen_sampled(ea):
     inp = make_workload("varlen", with_grad=True)
     dq, dk, dv = gpu_fwd_bwd(ea, inp, True, inp.key_keep)

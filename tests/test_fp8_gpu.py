@@ -167,11 +167,12 @@ def test_fp8_repeat_is_bit_identical(ea):
     check(inp, o1, l1, True)
 
 
-def test_fp8_full_size_sampled_slices(ea):
-    # the benchmark workload (causal, B2 H16 N4096 d128), checked on sampled slices
-    inp = make_fp8(2, 16, 4096, 128, seed=8260, causal=True)
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_full_size_sampled_slices(ea, causal):
+    # the benchmark shape (B2 H16 N4096 d128), checked on sampled slices
+    inp = make_fp8(2, 16, 4096, 128, seed=8260 + int(causal), causal=causal)
     o, l = gpu_fp8(ea, inp)
-    check(inp, o, l, True, slices=[0, 13, 31])
+    check(inp, o, l, causal, slices=[0, 13, 31])
 
 
 def test_fp8_dense_key_mask_with_empty_rows(ea):
