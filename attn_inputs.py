@@ -10,7 +10,11 @@ rounded to bf16, tensors drawn in the order Q, K, V, dO):
 * packed variable-length tensors are token-major ``[total, H, d]`` with
   ``cu_seqlens[B+1]`` (int32) giving each sequence's first token;
 * the key-padding mask ``key_keep`` is uint8, 1 = attend, 0 = masked, shaped
-  ``[B, N]`` (dense) or ``[total]`` (packed).
+  ``[B, N]`` (dense) or ``[total]`` (packed);
+* e4m3 (FP8) inputs are float32 draws for Q, K, V (in that order) quantised per
+  tensor the way a caller prepares them: factor = amax / 448, codes from torch's
+  ``float8_e4m3fn`` rounding (``make_fp8``, ``make_fp8_varlen``);
+* block-sparse tile masks are uint8 ``[H, nb, nb]`` Bernoulli draws (``tile_mask``).
 
 The shapes follow the workloads the attention pages talk about: sequence length
 2048 ("PyTorch Attention 层性能分析与优化" / codechina FlashAttention article §5.2
