@@ -212,6 +212,146 @@ def recorded_traffic(kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+# The backward as timed in the headline step: its kernels launched one by one
+# through attn_bwd_phase so each gets its own CUDA events.  (name, phase, kernel,
+# tensor-core FLOPs of the kernel in units of the forward's count, or None for an
+# HBM-bound kernel.)
+BWD_PHASES = [
+    ("bwd_pre", 0, "attn_bwd_pre_kernel", None),
+    ("bwd_dkdv", 1, "attn_bwd_dkdv_sm100_kernel", 2.0),
+    ("bwd_dq", 2, "attn_bwd_dq_sm100_kernel", 1.5),
+]
+MIN_WARMUP = 10  # warm-up calls before any timing (at least, whatever --warmup says)
+
+
+def _median_ms(fn, flush, stream, reps):
+    """Median over `reps` calls of fn(), CUDA events on the launching stream, L2
+    flushed before each call outside the bracket."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for e in ev:
+        flush.zero_()
+        e[0].record(stream)
+        fn()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+
+
+def _shape_table(ea, dev, stream, flush, peak, reps, with_oracle):
+    """Every workload shape of the pages (sequence length 2048 timing table, codechina
+    article §5.2; N = 4096, d = 128 tiling example, §2.2; variable lengths, §6.2): the
+    median time, TFLOPS and share of the measured peak of each pass, with the
+    oracle's host time on a bounded sample next to it."""
+    import torch
+    from attn_inputs import draw_lengths, make_dense, make_varlen, padding_key_mask
+    out = {}
+    threads = None
+
+    def oracle_time(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    def entry(key, ms, flops, osec=None, ofrac=None):
+        tf = flops / (ms * 1e-3) / 1e12
+        e = {"us": round(ms * 1e3, 1), "tflops": round(tf, 1), "pct": round(100 * tf / peak, 1)}
+        if osec is not None:
+            # oracle on `ofrac` of the work, scaled up to the whole shape
+            e["oracle_s"] = round(osec / ofrac, 2)
+            e["oracle_cores"] = threads
+        out[key] = e
+
+    if with_oracle:
+        import oracle
+        threads = oracle.default_threads()
+    # (name, B, H, N, d, seed, sigma, causal list, with backward)
+    dense = [("c2_n2048_d64", 4, 16, 2048, 64, 2, 1.0, (True, False), True),
+             ("c3_n4096_d128", 2, 16, 4096, 128, 3, 1.0, (False,), True),
+             ("c3s_n4096_d128_sigma4", 2, 16, 4096, 128, 33, 4.0, (True, False), False)]
+    for name, B, H, N, d, seed, sig, causals, with_bwd in dense:
+        inp = make_dense(B, H, N, d, seed=seed, qk_sigma=sig, with_grad=with_bwd)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        do = inp.do.to(dev) if with_bwd else None
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+        ws = ea.workspace_for(q) if with_bwd else None
+        for causal in causals:
+            kw = dict(scale=inp.scale, causal=causal, stream=stream)
+            for _ in range(3):
+                ea.attn_fwd(q, k, v, o, lse, **kw)
+            f_ms = _median_ms(lambda: ea.attn_fwd(q, k, v, o, lse, **kw), flush, stream, reps)
+            ffl = (2.0 if causal else 4.0) * B * H * N * N * d
+            tag = f"{name}_{'causal' if causal else 'noncausal'}"
+            osec = None
+            if with_oracle:
+                osec = oracle_time(lambda: oracle.fwd(inp.q, inp.k, inp.v, inp.scale, causal, slices=[0],
+                                                      nthreads=threads))
+            entry(tag + "_fwd", f_ms, ffl, osec, 1.0 / (B * H))
+            if with_bwd:
+                dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+                for _ in range(3):
+                    ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace=ws, **kw)
+                b_ms = _median_ms(lambda: ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace=ws, **kw),
+                                  flush, stream, reps)
+                osec = None
+                if with_oracle:
+                    osec = oracle_time(lambda: oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, causal,
+                                                          slices=[0], nthreads=threads))
+                entry(tag + "_bwd", b_ms, 2.5 * ffl, osec, 1.0 / (B * H))
+        del q, k, v, o, lse, do, ws
+    # variable-length workload: 8 sequences of U[256, 4096] tokens, H32 d128, causal,
+    # key padding that empties the first 2 % of each sequence's query rows
+    lengths = draw_lengths(8, 256, 4096, 40)
+    keep = padding_key_mask(lengths, 41)
+    vin = make_varlen(lengths, 32, 128, 4, True, keep, with_grad=True)
+    q, k, v, do = (t.to(dev) for t in (vin.q, vin.k, vin.v, vin.do))
+    cu, kk = vin.cu_seqlens.to(dev), keep.to(dev)
+    o, lse = torch.empty_like(q), torch.empty(q.shape[:2], device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = ea.workspace_for(q, cu)
+    kw = dict(scale=vin.scale, causal=True, cu_seqlens=cu, key_keep=kk, max_seqlen=max(lengths), stream=stream)
+    ffl = 2.0 * 32 * 128 * sum(n * n for n in lengths)
+    for _ in range(3):
+        ea.attn_fwd(q, k, v, o, lse, **kw)
+        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace=ws, **kw)
+    f_ms = _median_ms(lambda: ea.attn_fwd(q, k, v, o, lse, **kw), flush, stream, reps)
+    b_ms = _median_ms(lambda: ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace=ws, **kw), flush, stream, reps)
+    osf = osb = None
+    frac = (lengths[0] ** 2) / (32 * sum(n * n for n in lengths))  # sequence 0, head 0
+    if with_oracle:
+        osf = oracle_time(lambda: oracle.fwd(vin.q, vin.k, vin.v, vin.scale, True, cu_seqlens=vin.cu_seqlens,
+                                             key_keep=keep, slices=[0], nthreads=threads))
+        osb = oracle_time(lambda: oracle.bwd(vin.q, vin.k, vin.v, vin.do, vin.scale, True,
+                                             cu_seqlens=vin.cu_seqlens, key_keep=keep, slices=[0],
+                                             nthreads=threads))
+    entry("c4_varlen_8x_h32_d128_causal_fwd", f_ms, ffl, osf, frac)
+    entry("c4_varlen_8x_h32_d128_causal_bwd", b_ms, 2.5 * ffl, osb, frac)
+    st = ea.attn_status(stream)
+    if st != ea.ATTN_OK:
+        raise RuntimeError(f"shape table reported status {st}: {ea.attn_strerror(st)}")
+    return out
+
+
+def launch_plan(gpus: int, env) -> tuple:
+    """How to honour --gpus: ("run", None) when the process layout already matches,
+    ("spawn", argv) to relaunch this script as `gpus` ranks (one process per GPU,
+    torchrun on 127.0.0.1) when started as a single plain process, or ("error", text)
+    when started under a launcher with another world size."""
+    ws = env.get("WORLD_SIZE")
+    if gpus < 1:
+        return "error", f"--gpus must be >= 1, got {gpus}"
+    if ws is None:
+        if gpus == 1:
+            return "run", None
+        argv = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+                "--master-addr=127.0.0.1", "--master-port=29531", os.path.abspath(__file__)] + sys.argv[1:]
+        return "spawn", argv
+    if int(ws) != gpus:
+        return "error", f"--gpus {gpus} but the launcher started WORLD_SIZE={ws} ranks"
+    return "run", None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -219,6 +359,9 @@ def run_ours(args):
     ws, rank, local = dist_env()
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}), flush=True)
+        return 1
+    if ws > torch.cuda.device_count():
+        print(json.dumps({"error": f"{ws} ranks but {torch.cuda.device_count()} visible GPUs"}), flush=True)
         return 1
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -244,25 +387,22 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
     kw = dict(scale=inp.scale, causal=CAUSAL, stream=stream)
+    n_k = 1 + len(BWD_PHASES)  # kernels per step
 
     def step(ev=None):
-        # attn_bwd == phases 0, 1, 2 in order; called one by one here to time each kernel
+        # attn_bwd == its phases in order; launched one by one here to time each kernel
         if ev is not None:
             ev[0].record(stream)
         ea.attn_fwd(q, k, v, o, lse, **kw)
+        for i, (_, ph, _, _) in enumerate(BWD_PHASES):
+            if ev is not None:
+                ev[1 + i].record(stream)
+            ea.attn_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
         if ev is not None:
-            ev[1].record(stream)
-        ea.attn_bwd_phase(0, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
-        if ev is not None:
-            ev[2].record(stream)
-        ea.attn_bwd_phase(1, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
-        if ev is not None:
-            ev[3].record(stream)
-        ea.attn_bwd_phase(2, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
-        if ev is not None:
-            ev[4].record(stream)
+            ev[n_k].record(stream)
 
-    for _ in range(max(3, args.warmup)):
+    n_warm = max(MIN_WARMUP, args.warmup)
+    for _ in range(n_warm):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
@@ -270,7 +410,7 @@ def run_ours(args):
     if st != ea.ATTN_OK:
         raise RuntimeError(f"warm-up reported status {st}: {ea.attn_strerror(st)}")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_k + 1)] for _ in range(args.steps)]
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -287,7 +427,7 @@ def run_ours(args):
     if st != ea.ATTN_OK:
         raise RuntimeError(f"timed steps reported status {st}: {ea.attn_strerror(st)}")
 
-    seg = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in events]  # ms: fwd, pre, dK/dV, dQ
+    seg = [[e[i].elapsed_time(e[i + 1]) for i in range(n_k)] for e in events]  # ms per kernel per step
     step_ms = [sum(x) for x in seg]
     total_ms = sum(step_ms)
     from exact_attention_123_b200.sharding import max_over_ranks
@@ -346,6 +486,10 @@ def run_ours(args):
     if st != ea.ATTN_OK:
         raise RuntimeError(f"end-to-end steps reported status {st}")
 
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks["bf16_tflops"])
+    reps = max(20, args.shape_reps)
+
     # ---- block-sparse variant: the same workload with half of the (query tile, key
     # tile) pairs left out by a seeded per-head tile mask; timed after the headline
     # steps, L2 flushed before each call.  FLOPs are those of the pairs computed
@@ -364,26 +508,17 @@ def run_ours(args):
         for _ in range(3):
             ea.attn_fwd_blocksparse(q, k, v, bmd, o, lse, **kw)
             ea.attn_bwd_blocksparse(q, k, v, o, lse, do, bmd, dq, dk, dv, workspace=wsbuf, **kw)
-        n_bs = 20
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bs)]
-        for e in ev:
-            flush.zero_()
-            e[0].record(stream)
-            ea.attn_fwd_blocksparse(q, k, v, bmd, o, lse, **kw)
-            e[1].record(stream)
-            ea.attn_bwd_blocksparse(q, k, v, o, lse, do, bmd, dq, dk, dv, workspace=wsbuf, **kw)
-            e[2].record(stream)
-        torch.cuda.synchronize(dev)
+        f_ms = _median_ms(lambda: ea.attn_fwd_blocksparse(q, k, v, bmd, o, lse, **kw), flush, stream, reps)
+        b_ms = _median_ms(lambda: ea.attn_bwd_blocksparse(q, k, v, o, lse, do, bmd, dq, dk, dv, workspace=wsbuf, **kw),
+                          flush, stream, reps)
         st = ea.attn_status(stream)
         if st != ea.ATTN_OK:
             raise RuntimeError(f"block-sparse steps reported status {st}")
-        f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-        b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
         dense_units = nbt * (nbt + 1) / 2 - nbt / 2 if CAUSAL else nbt * nbt
-        bsp = {"tile_density": 0.5, "tile_mask_seed": SEED + 7, "pairs_computed_frac_of_dense": pair_units / (H * dense_units),
-               "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": fl_fwd / (f_ms * 1e-3) / 1e12,
-               "bwd_tflops": 2.5 * fl_fwd / (b_ms * 1e-3) / 1e12,
-               "note": "attn_fwd_blocksparse / attn_bwd_blocksparse on the bench workload; FLOPs of the computed tile pairs"}
+        bsp = {"density": 0.5, "seed": SEED + 7, "pairs_frac": round(pair_units / (H * dense_units), 4),
+               "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+               "fwd_tflops": round(fl_fwd / (f_ms * 1e-3) / 1e12, 1),
+               "bwd_tflops": round(2.5 * fl_fwd / (b_ms * 1e-3) / 1e12, 1)}
 
     # ---- FP8 (e4m3) forward on the same workload: q, k, v quantised per tensor
     # (factor = amax / 448) on the device; timed like the block-sparse variant.
@@ -398,48 +533,42 @@ def run_ours(args):
         (q8, qf), (k8, kf), (v8, vf) = q8s
         for _ in range(3):
             ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, **kw)
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
-        for e in ev:
-            flush.zero_()
-            e[0].record(stream)
-            ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, **kw)
-            e[1].record(stream)
-        torch.cuda.synchronize(dev)
+        f8_ms = _median_ms(lambda: ea.attn_fwd_fp8(q8, k8, v8, qf, kf, vf, o, lse, **kw), flush, stream, reps)
         st = ea.attn_status(stream)
         if st != ea.ATTN_OK:
             raise RuntimeError(f"fp8 forward reported status {st}")
-        f8_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
         f8_tf = flops_fwd() / (f8_ms * 1e-3) / 1e12
-        pk8 = 2.0 * float(measured_peaks()[0]["bf16_tflops"])
-        fp8 = {"fwd_ms": f8_ms, "fwd_tflops": f8_tf, "peak_tflops": pk8, "frac_of_peak": f8_tf / pk8,
-               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal e4m3 : bf16 dense ratio)",
-               "note": "attn_fwd_fp8 on the bench workload, e4m3 inputs"}
+        pk8 = 2.0 * peak
+        fp8 = {"fwd_ms": round(f8_ms, 4), "fwd_tflops": round(f8_tf, 1), "pct_of_2x_bf16_peak": round(100 * f8_tf / pk8, 1)}
+
+    shapes = None
+    if not args.no_shapes and ws == 1:
+        shapes = _shape_table(ea, dev, stream, flush, peak, reps, with_oracle=not args.no_cpu_baseline)
 
     step_flops = flops_fwd() + flops_bwd()
     value = step_flops * args.steps * ws / (total_ms_max * 1e-3) / 1e12
     e2e_value = step_flops * e2e_n * ws / (e2e_ms * 1e-3) / 1e12
 
-    peaks, peak_src = measured_peaks()
-    peak = float(peaks["bf16_tflops"])
-    fwd_ms = statistics.mean(x[0] for x in seg)
-    pre_ms = statistics.mean(x[1] for x in seg)
-    dkdv_ms = statistics.mean(x[2] for x in seg)
-    dq_ms = statistics.mean(x[3] for x in seg)
+    # per-kernel medians over the timed steps (the headline value above uses the total)
+    med = [statistics.median(x[i] for x in seg) for i in range(n_k)]
+    fwd_ms = med[0]
+    bwd_ms = sum(med[1:])
     fwd_tf = flops_fwd() / (fwd_ms * 1e-3) / 1e12
-    bwd_tf = flops_bwd() / ((pre_ms + dkdv_ms + dq_ms) * 1e-3) / 1e12
-    # Algorithmic FLOPs per kernel launch, counted as the tensor-core products each
-    # one performs: dK/dV does S^T, dP^T, dV, dK (2x the forward's count); dQ does
-    # S, dP, dQ (1.5x).  (The backward as a whole is credited 2.5x the forward in
-    # the headline value; the recomputed S and dP of the dQ pass are not.)
-    dkdv_tf = 2.0 * flops_fwd() / (dkdv_ms * 1e-3) / 1e12
-    dq_tf = 1.5 * flops_fwd() / (dq_ms * 1e-3) / 1e12
-    # the preprocess kernel is HBM-bound: O and dO read (bf16), lse read, D and lse2 written
-    pre_bytes = B * H * N * (2 * D * 2 + 4 + 8)
-    pre_gbs = pre_bytes / (pre_ms * 1e-3) / 1e9
-    per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf), "attn_bwd_dkdv_sm100_kernel": (dkdv_ms, dkdv_tf),
-                  "attn_bwd_dq_sm100_kernel": (dq_ms, dq_tf)}
+    bwd_tf = flops_bwd() / (bwd_ms * 1e-3) / 1e12
+    per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf)}
+    breakdown = {"fwd": round(fwd_ms * 1e3, 1)}
+    pre = None
+    for (name, _, kname, mult), ms in zip(BWD_PHASES, med[1:]):
+        breakdown[name] = round(ms * 1e3, 1)
+        if mult is None:
+            pre = (kname, ms)
+        else:
+            per_kernel[kname] = (ms, mult * flops_fwd() / (ms * 1e-3) / 1e12)
     dominant = max(per_kernel, key=lambda kname: per_kernel[kname][0])
     dom_tf = per_kernel[dominant][1]
+    # the preprocess kernel is HBM-bound: O and dO read (bf16), lse read, D and lse2 written
+    pre_bytes = B * H * N * (2 * D * 2 + 4 + 8)
+    pre_gbs = pre_bytes / (pre[1] * 1e-3) / 1e9
 
     if ws > 1:
         dist.destroy_process_group()
@@ -452,32 +581,42 @@ def run_ours(args):
         cpu = {"value": cv, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(cdt, 3)}
 
+    ncu = recorded_ncu()
+    if ncu:  # the three headline counters per kernel; the full record is in profiles/
+        ncu = {k: {"tensor_pct": round(e.get("tensor_pipe_active_pct", float("nan")), 1),
+                   "hbm_gbs": round(e.get("hbm_gbs", float("nan"))),
+                   "smem_conflicts": int(e.get("smem_bank_conflicts_ld", 0) + e.get("smem_bank_conflicts_st", 0))}
+               for k, e in ncu.items()}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "causal": CAUSAL, "seed": SEED,
                    "l2": "flushed (256 MiB write) before every timed step, outside the timed bracket",
+                   "warmup_steps_run": n_warm,
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
-        "breakdown_ms": {"fwd": fwd_ms, "bwd_pre": pre_ms, "bwd_dkdv": dkdv_ms, "bwd_dq": dq_ms},
-        "tflops": {"fwd": fwd_tf, "bwd": bwd_tf, "bwd_dkdv_kernel": dkdv_tf, "bwd_dq_kernel": dq_tf},
-        "pct_of_peak": {"fwd": 100 * fwd_tf / peak, "bwd": 100 * bwd_tf / peak, "step": 100 * value / ws / peak,
-                        "peak": f"{peak} TFLOPS bf16 dense ({peak_src}, burst)"},
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "traffic": recorded_traffic(dominant),
                      "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src}, burst)"},
-        "hbm": {"kernel": "attn_bwd_pre_kernel", "achieved": pre_gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                "frac": pre_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": pre_bytes,
-                "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src})"},
-        "ncu_recorded": recorded_ncu(),
+        "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_n, "pipeline": "copy in, kernels, copy out on three streams over two buffer sets"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": n_k * args.steps,
         "clocks": clk.summary(),
-        "wall_s_timed_region": wall,
-        "cpu_baseline": cpu,
+        "wall_s_timed_region": round(wall, 4),
+        "ncu_recorded": ncu,
         "blocksparse": bsp,
         "fp8": fp8,
+        "hbm": {"kernel": pre[0], "achieved": round(pre_gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": round(pre_gbs / float(peaks["hbm_gbs"]), 4), "bytes_per_launch": pre_bytes},
+        "shapes": shapes,
+        # last, so that they survive in any tail of the output
+        "breakdown_us": breakdown,
+        "tflops": {"fwd": round(fwd_tf, 1), "bwd": round(bwd_tf, 1),
+                   **{k: round(v[1], 1) for k, v in per_kernel.items() if k != "attn_fwd_sm100_kernel"}},
+        "pct_of_peak": {"fwd": round(100 * fwd_tf / peak, 2), "bwd": round(100 * bwd_tf / peak, 2),
+                        "step": round(100 * value / ws / peak, 2), "stat": f"median of {args.steps} steps",
+                        "peak": f"{peak} TFLOPS bf16 dense ({peak_src}, burst)"},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -565,7 +704,7 @@ def ncu_summary(report: str, record: bool) -> int:
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -574,6 +713,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward's timing")
+    ap.add_argument("--no-shapes", action="store_true", help="skip the table of the other workload shapes")
+    ap.add_argument("--shape-reps", type=int, default=30, help="timed calls per entry of the shape table (median)")
     ap.add_argument("--ncu-summary", metavar="REPORT",
                     help="print the per-kernel figures of an ncu --set full report (no GPU needed) and exit")
     ap.add_argument("--record", action="store_true",
@@ -581,6 +722,12 @@ def main():
     args = ap.parse_args()
     if args.ncu_summary:
         return ncu_summary(args.ncu_summary, args.record)
+    plan, what = launch_plan(args.gpus, os.environ)
+    if plan == "error":
+        print(json.dumps({"error": what}), flush=True)
+        return 2
+    if plan == "spawn":
+        return subprocess.run(what).returncode
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -6,12 +6,12 @@ current stream.  There is no CPU or library fallback: if ``libattn.so`` is
 missing, importing the entry points raises.
 
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
-``attn_bwd``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
+``attn_bwd``, ``attn_bwd_deterministic``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
 ``attn_fwd_blocksparse``, ``attn_bwd_blocksparse``, ``attn_fwd_fp8``, ``attn_fwd_fp8_masked``,
 ``attn_fwd_fp8_varlen``,
-``attn_bwd_workspace_bytes``,
+``attn_bwd_workspace_bytes``, ``attn_bwd_deterministic_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
-``attn_set_wait_limit_ms``, ``attn_debug_skip_load``.
+``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``.
 """
 from __future__ import annotations
 
@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
     L.attn_bwd_varlen_workspace_bytes.argtypes = [i, i, i]
     L.attn_bwd_varlen_workspace_bytes.restype = sz
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp, sz, vp]
+    L.attn_bwd_deterministic.argtypes = L.attn_bwd.argtypes
+    L.attn_bwd_deterministic_workspace_bytes.argtypes = [i, i, i, i]
+    L.attn_bwd_deterministic_workspace_bytes.restype = sz
     L.attn_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_phase.argtypes = [i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp, vp, sz, vp]
     L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp]
@@ -74,10 +77,12 @@ def lib() -> ctypes.CDLL:
     L.attn_strerror.restype = ctypes.c_char_p
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
-    for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_varlen", "attn_bwd_phase",
+    L.attn_debug_ex2_poly.argtypes = [vp, vp, ctypes.c_longlong, vp]
+    for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_deterministic",
+                 "attn_bwd_varlen", "attn_bwd_phase",
                  "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked",
                  "attn_fwd_fp8_varlen", "attn_status", "attn_set_wait_limit_ms",
-                 "attn_debug_skip_load"):
+                 "attn_debug_skip_load", "attn_debug_ex2_poly"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -194,24 +199,34 @@ def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(lib().attn_bwd_workspace_bytes(B, H, N, d))
 
 
+def attn_bwd_deterministic_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().attn_bwd_deterministic_workspace_bytes(B, H, N, d))
+
+
 def attn_bwd_varlen_workspace_bytes(total: int, H: int, d: int) -> int:
     return int(lib().attn_bwd_varlen_workspace_bytes(total, H, d))
 
 
-def workspace_for(q: torch.Tensor, cu_seqlens=None) -> torch.Tensor:
-    """Allocate (with torch) a backward workspace sized for q's shape."""
+def workspace_for(q: torch.Tensor, cu_seqlens=None, deterministic: bool = False) -> torch.Tensor:
+    """Allocate (with torch) a backward workspace sized for q's shape (the smaller
+    one of the deterministic backward when ``deterministic``)."""
     if cu_seqlens is not None:
-        n = attn_bwd_varlen_workspace_bytes(q.shape[0], q.shape[1], q.shape[2])
+        if deterministic:
+            n = attn_bwd_deterministic_workspace_bytes(1, q.shape[1], q.shape[0], q.shape[2])
+        else:
+            n = attn_bwd_varlen_workspace_bytes(q.shape[0], q.shape[1], q.shape[2])
     else:
         B, H, N, d = q.shape
-        n = attn_bwd_workspace_bytes(B, H, N, d)
+        n = (attn_bwd_deterministic_workspace_bytes if deterministic else attn_bwd_workspace_bytes)(B, H, N, d)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
 
 
 def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[float] = None,
              causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
-             workspace: Optional[torch.Tensor] = None, stream=None):
-    """Backward pass.  Returns (dq, dk, dv)."""
+             workspace: Optional[torch.Tensor] = None, deterministic: bool = False, stream=None):
+    """Backward pass.  Returns (dq, dk, dv).  ``deterministic`` selects the
+    bit-reproducible variant (``attn_bwd_deterministic``; for packed inputs its
+    three phases through ``attn_bwd_phase``)."""
     packed = cu_seqlens is not None
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
@@ -224,9 +239,15 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if workspace is None:
-        workspace = workspace_for(q, cu_seqlens)
+        workspace = workspace_for(q, cu_seqlens, deterministic)
     _need(workspace, torch.uint8, "workspace")
-    if cu_seqlens is not None:
+    if cu_seqlens is not None and deterministic:
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        for ph in range(3):
+            attn_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, workspace=workspace, scale=scale, causal=causal,
+                           cu_seqlens=cu_seqlens, key_keep=key_keep, max_seqlen=max_seqlen, stream=stream)
+    elif cu_seqlens is not None:
         total, H = q.shape[0], q.shape[1]
         B = cu_seqlens.numel() - 1
         if max_seqlen is None:
@@ -238,10 +259,11 @@ def attn_bwd(q, k, v, o, lse, do, dq=None, dk=None, dv=None, *, scale: Optional[
         _check(rc, "attn_bwd_varlen")
     else:
         B, H, N, _ = q.shape
-        rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
-                            B, H, N, d, float(scale), int(causal), None, _ptr(key_keep), _ptr(workspace),
-                            workspace.numel(), _stream(stream))
-        _check(rc, "attn_bwd")
+        name = "attn_bwd_deterministic" if deterministic else "attn_bwd"
+        rc = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), B, H, N, d, float(scale), int(causal), None, _ptr(key_keep),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+        _check(rc, name)
     return dq, dk, dv
 
 
@@ -333,6 +355,11 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None
     return o, lse
 
 
+def attn_bwd_deterministic(q, k, v, o, lse, do, dq=None, dk=None, dv=None, **kw):
+    """attn_bwd with bit-reproducible results (dK/dV and dQ in separate passes)."""
+    return attn_bwd(q, k, v, o, lse, do, dq, dk, dv, deterministic=True, **kw)
+
+
 def attn_bwd_phase(phase: int, q, k, v, o, lse, do, dq, dk, dv, *, workspace, scale: Optional[float] = None,
                    causal: bool = True, cu_seqlens=None, key_keep=None, max_seqlen: Optional[int] = None,
                    stream=None):
@@ -390,3 +417,12 @@ def attn_set_wait_limit_ms(ms: int) -> int:
 
 def attn_debug_skip_load(index: int) -> int:
     return int(lib().attn_debug_skip_load(int(index)))
+
+
+def attn_debug_ex2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The forward kernels' FMA-pipe 2^x on a float32 CUDA tensor of even size
+    (test hook).  Returns y of x's shape."""
+    _need(x, torch.float32, "x")
+    y = torch.empty_like(x)
+    _check(lib().attn_debug_ex2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "attn_debug_ex2_poly")
+    return y

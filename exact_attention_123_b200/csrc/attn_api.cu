@@ -17,6 +17,17 @@ namespace {
 
 __device__ int g_attn_status = 0;
 
+// Test hook kernel: the forward kernels' FMA-pipe exponential on pairs of inputs.
+__global__ void ex2_poly_probe_kernel(const float2 *x, float2 *y, long long pairs) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < pairs;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float2 v = x[i];
+        float a, b;
+        attn::ex2_poly_x2(attn::f2_pack(v.x, v.y), a, b);
+        y[i] = make_float2(a, b);
+    }
+}
+
 constexpr int kMaxDevices = 64;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -333,6 +344,20 @@ size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
     return bwd_ws_bytes(static_cast<long long>(B) * H * N, d);
 }
 
+size_t attn_bwd_deterministic_workspace_bytes(int B, int H, int N, int d) {
+    if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+    return bwd_ws_bytes(static_cast<long long>(B) * H * N, d);
+}
+
+int attn_bwd_deterministic(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                           const void *dout, void *dq, void *dk, void *dv, int B, int H, int N, int d, float scale,
+                           int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
+                    stream);
+}
+
 size_t attn_bwd_varlen_workspace_bytes(int total_tokens, int H, int d) {
     if (total_tokens < 0 || H <= 0 || (d != 64 && d != 128)) return 0;
     return bwd_ws_bytes(static_cast<long long>(total_tokens) * H, d);
@@ -395,6 +420,19 @@ const char *attn_strerror(int code) {
 
 int attn_set_wait_limit_ms(int ms) {
     return g_wait_limit_ms.exchange(ms > 0 ? ms : 4000);
+}
+
+int attn_debug_ex2_poly(const float *x, float *y, long long n, void *stream) {
+    if (!x || !y || n <= 0 || (n & 1)) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return ATTN_ERR_MISALIGNED;
+    DeviceState *ds = nullptr;
+    const int rc = device_state(&ds);
+    if (rc) return rc;
+    const long long pairs = n / 2;
+    const unsigned blocks = static_cast<unsigned>(pairs / 256 + 1 < 4096 ? pairs / 256 + 1 : 4096);
+    ex2_poly_probe_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float2 *>(x), reinterpret_cast<float2 *>(y), pairs);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_debug_skip_load(int load_index) {

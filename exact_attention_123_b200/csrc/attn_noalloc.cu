@@ -42,14 +42,14 @@ extern "C" int attn_bwd_noalloc(const void *q, const void *k, const void *v, con
                                 const void *dout, void *dq, void *dk, void *dv, int B, int H, int N, int d,
                                 float scale, int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
                                 void *stream) {
-    const size_t need = attn_bwd_workspace_bytes(B, H, N, d);
-    if (need == 0)  // invalid sizes: let attn_bwd report the argument error
-        return attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, is_causal, cu_seqlens, key_keep,
-                        nullptr, 0, stream);
+    const size_t need = attn_bwd_deterministic_workspace_bytes(B, H, N, d);
+    if (need == 0)  // invalid sizes: let the backward report the argument error
+        return attn_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, is_causal, cu_seqlens,
+                                      key_keep, nullptr, 0, stream);
     if (need > ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
     void *ws = nullptr;
     const int rc = scratch_address(&ws);
     if (rc != ATTN_OK) return rc;
-    return attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, is_causal, cu_seqlens, key_keep, ws,
-                    ATTN_NOALLOC_SCRATCH_BYTES, stream);
+    return attn_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, is_causal, cu_seqlens,
+                                  key_keep, ws, ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }

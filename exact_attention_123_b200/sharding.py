@@ -1,8 +1,8 @@
 """Head sharding across the GPUs of one node.
 
 Every (sequence, head) slice of exact attention is independent of every other, so
-the heads of a batch can be partitioned across the GPUs of a node ("4.5 注意力优化
-实战：从PyTorch到CUDA的完整流程", §6.3: partition by attention heads, NCCL for the
+the heads of a batch can be partitioned across the GPUs of a node (codechina FlashAttention
+article, §6.3 multi-GPU scaling: partition by attention heads, NCCL for the
 communication between GPUs).  Each rank runs this package's kernels on its own
 contiguous range of heads; the attention itself needs no collective.  Only a caller
 that wants every head's output on every rank gathers the shards (``gather_heads``,
@@ -49,7 +49,7 @@ def attn_fwd_sharded(q, k, v, *, world: int, rank: int, scale: Optional[float] =
 
 
 def attn_bwd_sharded(q, k, v, o_local, lse_local, do, *, world: int, rank: int, scale: Optional[float] = None,
-                     causal: bool = True, stream=None):
+                     causal: bool = True, deterministic: bool = False, stream=None):
     """Backward on this rank's heads (o_local / lse_local from attn_fwd_sharded).
     Returns (dq_local, dk_local, dv_local)."""
     from . import attn_bwd
@@ -58,7 +58,8 @@ def attn_bwd_sharded(q, k, v, o_local, lse_local, do, *, world: int, rank: int, 
         scale = q.shape[-1] ** -0.5
     if ql.shape[1] == 0:
         return torch.empty_like(ql), torch.empty_like(kl), torch.empty_like(vl)
-    return attn_bwd(ql, kl, vl, o_local, lse_local, dol, scale=scale, causal=causal, stream=stream)
+    return attn_bwd(ql, kl, vl, o_local, lse_local, dol, scale=scale, causal=causal, deterministic=deterministic,
+                    stream=stream)
 
 
 def gather_heads(t_local: torch.Tensor, H: int, group=None) -> torch.Tensor:

@@ -112,9 +112,7 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
  *   dq, dk, dv : outputs (bf16, layout of q).
  *   workspace  : caller-owned device memory of at least
  *                attn_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
- *                its contents are scratch (two fp32 terms per query row and
- *                head) and need no initialisation.
- * The result is deterministic: no atomics are used.
+ *                its contents are scratch and need no initialisation.
  * Returns an attn_status_t code.
  */
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -122,6 +120,22 @@ ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o
              int B, int H, int N, int d, float scale, int is_causal,
              const int32_t *cu_seqlens, const uint8_t *key_keep,
              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The same backward computed in an order that does not depend on scheduling, so
+ * that repeated calls on the same inputs give bit-identical dq, dk and dv: dK/dV
+ * in one pass per 128-key tile, dQ in a separate pass per 128-row query tile
+ * ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", 第四步 §2: dQ sweeps all key/value
+ * blocks), with no atomics.  Arguments as attn_bwd; the workspace needs at least
+ * attn_bwd_deterministic_workspace_bytes(B, H, N, d) bytes (two fp32 terms per
+ * query row and head; attn_bwd_workspace_bytes is always enough).
+ */
+ATTN_API size_t attn_bwd_deterministic_workspace_bytes(int B, int H, int N, int d);
+ATTN_API int attn_bwd_deterministic(const void *q, const void *k, const void *v, const void *o,
+                                    const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                                    int B, int H, int N, int d, float scale, int is_causal,
+                                    const int32_t *cu_seqlens, const uint8_t *key_keep,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Packed variable-length forward with an exact token count.
@@ -148,8 +162,9 @@ ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const 
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * One of the backward's three kernels (attn_bwd / attn_bwd_varlen launch all three
- * in this order); lets a caller time or schedule them separately.
+ * One of the three kernels of the deterministic backward (attn_bwd_deterministic
+ * launches all three in this order); lets a caller time or schedule them
+ * separately, and gives the packed layout its deterministic backward.
  *   phase 0 : per-row terms D_i = rowsum(dO o O) and lse2 = lse*log2(e), in
  *             `workspace`
  *   phase 1 : dK and dV (one pass per 128-key tile over the query tiles)
@@ -158,7 +173,9 @@ ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const 
  * they may run in either order (or concurrently on two streams).
  * Phases must run in order on the same workspace and stream.  Other arguments as
  * attn_bwd_varlen; for the dense layout pass cu_seqlens = NULL, num_seqs = B,
- * max_seqlen = N and total_tokens = 0.
+ * max_seqlen = N and total_tokens = 0.  The workspace needs at least
+ * attn_bwd_deterministic_workspace_bytes bytes (for the packed layout with
+ * B = 1, N = total_tokens).
  */
 ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void *v, const void *o,
                             const float *lse, const void *dout, void *dq, void *dk, void *dv,
@@ -167,7 +184,7 @@ ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void 
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Block-sparse attention ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", §7.1,
+ * Block-sparse attention (codechina FlashAttention article, §7.1 variant algorithms,
  * Block-Sparse FlashAttention: only the important pairs are computed, a sparsity
  * pattern combined with the tiling).  Dense layout only, as attn_fwd / attn_bwd
  * with cu_seqlens = NULL and no key mask, plus:
@@ -247,15 +264,16 @@ ATTN_API int attn_fwd_fp8_varlen(const void *q, const void *k, const void *v, fl
  * not allocate once it has started (no counterpart in the attention pages: this
  * is a deployment convenience, not part of the method).
  *
- * The backward's scratch (two fp32 terms per query row and head) lives instead in
- * a fixed array of ATTN_NOALLOC_SCRATCH_BYTES inside the library, one copy per
- * GPU that loads the library, kept until the process exits.  Nothing is
- * allocated per call.  Arguments and layouts are those of attn_bwd (with
- * cu_seqlens != NULL the packed buffers must span B*N token rows).
+ * It runs the deterministic backward (attn_bwd_deterministic), whose scratch (two
+ * fp32 terms per query row and head) lives instead in a fixed array of
+ * ATTN_NOALLOC_SCRATCH_BYTES inside the library, one copy per GPU that loads the
+ * library, kept until the process exits.  Nothing is allocated per call.
+ * Arguments and layouts are those of attn_bwd (with cu_seqlens != NULL the
+ * packed buffers must span B*N token rows).
  *   - The sizes may need at most ATTN_NOALLOC_SCRATCH_BYTES of scratch, i.e.
- *     attn_bwd_workspace_bytes(B, H, N, d) <= ATTN_NOALLOC_SCRATCH_BYTES
- *     (B*H*N <= 1,048,576); larger sizes return ATTN_ERR_WORKSPACE without
- *     launching anything.
+ *     attn_bwd_deterministic_workspace_bytes(B, H, N, d) <=
+ *     ATTN_NOALLOC_SCRATCH_BYTES (B*H*N <= 1,048,576); larger sizes return
+ *     ATTN_ERR_WORKSPACE without launching anything.
  *   - The first call on a device looks up that device's copy of the array (with
  *     the device current); make that first call before any stream capture.
  *   - Every call shares the array, which keeps the last call's contents.  Nothing
@@ -297,6 +315,18 @@ ATTN_API int attn_set_wait_limit_ms(int ms);
  * Returns the previous value.  Nothing faults: all waits are time-limited.
  */
 ATTN_API int attn_debug_skip_load(int load_index);
+
+/*
+ * Test hook for the exponential that the d = 64 and e4m3 forward kernels take from
+ * the FMA pipe for part of their scores (a cubic in f = x - rint(x) on [-1/2, 1/2]
+ * times 2^rint(x), with x clamped to -127 first).  Writes y[i] = that kernel's
+ * 2^x[i] for i < n, on `stream`; x and y are DEVICE float arrays of n elements,
+ * 16-byte aligned.  n must be even and > 0 (the kernels evaluate pairs).  Exposed
+ * so that tests can hold the function to its stated accuracy: relative error
+ * at most 1.02e-4 where 2^x is a normal float, exactly +0 for x <= -127 and for
+ * -inf, exactly 2^x at integer x.  Returns an attn_status_t code.
+ */
+ATTN_API int attn_debug_ex2_poly(const float *x, float *y, long long n, void *stream);
 
 #ifdef __cplusplus
 }

@@ -32,8 +32,8 @@
  *   dQ = scale * dS K,   dK = scale * dS^T Q.
  * The backward recomputes its own float64 P; it never uses a GPU result.
  *
- * The tile mask is the block-sparse variant named in "4.5 注意力优化实战：从
- * PyTorch到CUDA的完整流程", §7.1 (Block-Sparse FlashAttention: compute only the
+ * The tile mask is the block-sparse variant named in the codechina FlashAttention
+ * article, §7.1 (Block-Sparse FlashAttention: compute only the
  * important pairs, combining a sparsity pattern with the tiling): a pair of a
  * block-row query tile and a block-column key tile either takes part or is left
  * out as a whole; left-out pairs behave exactly like masked scores.

@@ -27,6 +27,7 @@ def L():
 def test_header_declares_the_expected_entry_points():
     names = declared_functions()
     for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
+              "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_bytes", "attn_bwd_noalloc",
               "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen", "attn_fwd_blocksparse",
               "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked", "attn_fwd_fp8_varlen"):
         assert n in names
@@ -60,6 +61,25 @@ def test_strerror_and_workspace_sizes(L):
     assert ea.attn_bwd_workspace_bytes(1, 1, 1, 96) == 0
     assert ea.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
     assert ea.attn_bwd_varlen_workspace_bytes(1000, 4, 64) >= 2 * (1000 * 4 * 4)
+    # the deterministic backward needs only the two per-row terms, and never more than attn_bwd
+    assert ea.attn_bwd_deterministic_workspace_bytes(2, 16, 4096, 128) == 2 * (2 * 16 * 4096 * 4)
+    assert ea.attn_bwd_deterministic_workspace_bytes(2, 16, 4096, 128) <= ea.attn_bwd_workspace_bytes(2, 16, 4096, 128)
+    assert ea.attn_bwd_deterministic_workspace_bytes(1, 1, 1, 96) == 0
+
+
+def test_noalloc_size_limit_is_exact(L):
+    # ATTN_NOALLOC_SCRATCH_BYTES = 8 MiB holds the two fp32 terms of exactly 1,048,576
+    # query rows x heads; one more row is refused on the host, before any device work
+    # (so the fake pointers are never read and no GPU is needed).
+    import exact_attention_123_b200 as ea
+    limit = 8 << 20
+    assert ea.attn_bwd_deterministic_workspace_bytes(1, 1, 1048576, 128) <= limit
+    assert ea.attn_bwd_deterministic_workspace_bytes(1, 1, 1048577, 128) > limit
+    assert ea.attn_bwd_deterministic_workspace_bytes(1, 1, 1048577, 64) > limit
+    vp = ctypes.c_void_p
+    for shape in ((1, 1, 1048577, 128), (2, 1, 524289, 64)):
+        rc = L.attn_bwd_noalloc(*[vp(FAKE)] * 9, *shape, ctypes.c_float(0.088), 1, None, None, None)
+        assert rc == ea.ATTN_ERR_WORKSPACE, shape
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails host validation first

@@ -95,3 +95,27 @@ def test_ncu_report_rows(bench):
     assert e["tensor_pipe_active_pct"] == 51.5 and e["smem_per_cta_kb"] == 216.184
     assert e["smem_bank_conflicts_st"] == 7
     assert bench.ncu_kernel_key("void attn::attn_fwd_sm100_kernel<64, 1, 0>(X)") == "attn_fwd_sm100_kernel<64, 1, 0>"
+
+
+def test_launch_plan_honours_gpus(bench):
+    # one plain process and --gpus 1: run here
+    assert bench.launch_plan(1, {}) == ("run", None)
+    # under a launcher whose world size matches: run here
+    assert bench.launch_plan(4, {"WORLD_SIZE": "4"}) == ("run", None)
+    # one plain process asked for N > 1 GPUs: relaunch as N ranks, one per GPU, on 127.0.0.1
+    plan, argv = bench.launch_plan(2, {})
+    assert plan == "spawn"
+    assert "torch.distributed.run" in argv and "--nproc-per-node=2" in argv and "--master-addr=127.0.0.1" in argv
+    assert argv[-1 - len(sys.argv[1:])].endswith("bench.py")
+    # a launcher with another world size: refuse instead of printing the wrong n_gpus
+    plan, why = bench.launch_plan(2, {"WORLD_SIZE": "1"})
+    assert plan == "error" and "WORLD_SIZE=1" in why
+    assert bench.launch_plan(0, {})[0] == "error"
+
+
+def test_gpus_mismatch_exits_nonzero():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "1"],
+                       capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode != 0
+    assert "WORLD_SIZE=1" in json.loads(r.stdout.strip().splitlines()[-1])["error"]

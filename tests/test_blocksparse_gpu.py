@@ -1,4 +1,4 @@
-"""Block-sparse attention ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", §7.1,
+"""Block-sparse attention (codechina FlashAttention article, §7.1 variant algorithms,
 Block-Sparse FlashAttention) through the C ABI, against the float64 oracle with the
 same per-head tile mask: a left-out (query tile, key tile) pair behaves as masked
 scores, a query row left with no key gets O = 0 and lse = -inf.

@@ -6,6 +6,7 @@ short limit set here, every role of the kernel stops cleanly, and the host reads
 ATTN_ERR_TIMEOUT from attn_status().  The context stays usable: the next call
 succeeds and matches the oracle.  Nothing traps, faults or waits forever.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -13,6 +14,11 @@ import oracle
 from attn_inputs import make_dense
 
 pytestmark = pytest.mark.gpu
+
+
+def _within(got, ref, atol, rtol):
+    g = got.double().cpu().numpy()
+    return np.all(np.isfinite(g)) and not (np.abs(g - ref) > atol + rtol * np.abs(ref)).any()
 
 
 @pytest.fixture(scope="module")
@@ -39,9 +45,9 @@ def test_expired_wait_reports_timeout_and_context_survives(ea, skip):
         ea.attn_set_wait_limit_ms(prev_limit)
     o, lse = ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
     assert ea.attn_status() == ea.ATTN_OK
-    ro, _ = oracle.fwd(inp.q, inp.k, inp.v, inp.scale, True)
-    err = (o.double().cpu().numpy() - ro)
-    assert abs(err).max() < 2e-2
+    ro, rl = oracle.fwd(inp.q, inp.k, inp.v, inp.scale, True)
+    assert _within(o, ro, 1e-2, 1e-2)        # the benchmark spec bands
+    assert _within(lse, rl, 1e-3, 0.0)
 
 
 @pytest.mark.parametrize("skip", [0, 2])
@@ -64,5 +70,5 @@ def test_backward_expired_wait_reports_timeout_and_context_survives(ea, skip):
     assert ea.attn_status() == ea.ATTN_OK
     rq, rk, rv = oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, True)
     for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
-        assert abs(got.double().cpu().numpy() - ref).max() < 5e-2
+        assert _within(got, ref, 2e-2, 2e-2)
 

@@ -385,7 +385,7 @@ def test_slice_selection_leaves_others_untouched():
 
 
 # ---------------------------------------------------------------- block-sparse tile mask
-# "4.5 注意力优化实战：从PyTorch到CUDA的完整流程", §7.1 (Block-Sparse FlashAttention):
+# codechina FlashAttention article, §7.1 (Block-Sparse FlashAttention):
 # a (query tile, key tile) pair either takes part as a whole or is left out.
 
 def _tile_mask(H, nb, seed, density=0.6):
