@@ -3,8 +3,8 @@
 
 One step = one forward and one backward pass of causal bf16 attention over one
 batch of B=2, H=16, N=4096, d=128 (Q, K, V, dO ~ N(0,1), seeded), i.e. every
-kernel of the path: the fused forward, the backward's preprocessing, dK/dV and
-dQ kernels.  FLOPs follow the usual convention: forward
+kernel of the path: the fused forward, the backward's preprocessing, its
+single-pass dK/dV/dQ kernel and the dQ conversion.  FLOPs follow the usual convention: forward
 2*B*H*N^2*d for causal (4*B*H*N^2*d non-causal), backward 2.5x the forward.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -173,7 +173,8 @@ def source_digest():
     """Digest of the kernel sources' code: comments and white space are left out, so
     an edit to a comment does not disown counters taken on the same code."""
     h = hashlib.sha256()
-    for f in ("attn_bwd_sm100.cu", "attn_fwd_sm100.cu", "sm100_ptx.cuh", "attn_common.cuh", "attn_api.cu"):
+    for f in ("attn_bwd_sm100.cu", "attn_bwd_fused_sm100.cu", "attn_fwd_sm100.cu", "sm100_ptx.cuh", "attn_common.cuh",
+              "attn_api.cu"):
         with open(os.path.join(HERE, "exact_attention_123_b200", "csrc", f), encoding="utf-8") as fh:
             text = fh.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -217,9 +218,9 @@ def recorded_traffic(kernel: str):
 # tensor-core FLOPs of the kernel in units of the forward's count, or None for an
 # HBM-bound kernel.)
 BWD_PHASES = [
-    ("bwd_pre", 0, "attn_bwd_pre_kernel", None),
-    ("bwd_dkdv", 1, "attn_bwd_dkdv_sm100_kernel", 2.0),
-    ("bwd_dq", 2, "attn_bwd_dq_sm100_kernel", 1.5),
+    ("bwd_pre", 3, "attn_bwd_pre_kernel", None),            # D, lse2, zeroed dQ accumulator
+    ("bwd_main", 4, "attn_bwd_fused_sm100_kernel", 2.5),    # all five products of every tile pair
+    ("bwd_dq_convert", 5, "attn_bwd_dq_convert_kernel", None),
 ]
 MIN_WARMUP = 10  # warm-up calls before any timing (at least, whatever --warmup says)
 
@@ -557,18 +558,22 @@ def run_ours(args):
     bwd_tf = flops_bwd() / (bwd_ms * 1e-3) / 1e12
     per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf)}
     breakdown = {"fwd": round(fwd_ms * 1e3, 1)}
-    pre = None
+    hbm_ms = {}
     for (name, _, kname, mult), ms in zip(BWD_PHASES, med[1:]):
         breakdown[name] = round(ms * 1e3, 1)
         if mult is None:
-            pre = (kname, ms)
+            hbm_ms[kname] = ms
         else:
             per_kernel[kname] = (ms, mult * flops_fwd() / (ms * 1e-3) / 1e12)
     dominant = max(per_kernel, key=lambda kname: per_kernel[kname][0])
     dom_tf = per_kernel[dominant][1]
-    # the preprocess kernel is HBM-bound: O and dO read (bf16), lse read, D and lse2 written
-    pre_bytes = B * H * N * (2 * D * 2 + 4 + 8)
-    pre_gbs = pre_bytes / (pre[1] * 1e-3) / 1e9
+    # HBM-bound kernels, algorithmic bytes per launch: the preprocess reads O and dO
+    # (bf16) and lse, writes D and lse2 and zeroes the fp32 dQ accumulator; the
+    # conversion reads the accumulator and writes dQ (bf16)
+    hbm_bytes = {"attn_bwd_pre_kernel": B * H * N * (2 * D * 2 + 4 + 8 + 4 * D),
+                 "attn_bwd_dq_convert_kernel": B * H * N * (4 * D + 2 * D)}
+    hbm = {k: {"achieved": round(hbm_bytes[k] / (ms * 1e-3) / 1e9, 1), "bytes_per_launch": hbm_bytes[k]}
+           for k, ms in hbm_ms.items() if k in hbm_bytes}
 
     if ws > 1:
         dist.destroy_process_group()
@@ -607,8 +612,8 @@ def run_ours(args):
         "ncu_recorded": ncu,
         "blocksparse": bsp,
         "fp8": fp8,
-        "hbm": {"kernel": pre[0], "achieved": round(pre_gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                "frac": round(pre_gbs / float(peaks["hbm_gbs"]), 4), "bytes_per_launch": pre_bytes},
+        "hbm": {k: dict(e, unit="GB/s", frac=round(e["achieved"] / float(peaks["hbm_gbs"]), 4))
+                for k, e in hbm.items()},
         "shapes": shapes,
         # last, so that they survive in any tail of the output
         "breakdown_us": breakdown,

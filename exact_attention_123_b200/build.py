@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "attn_noalloc.cu"]
+SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "attn_bwd_fused_sm100.cu", "attn_noalloc.cu"]
 HEADERS = ["sm100_ptx.cuh", "attn_common.cuh", "attn_launch.h", "../../include/libattn.h"]
 
 

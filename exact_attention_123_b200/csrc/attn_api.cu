@@ -227,15 +227,22 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
     return attn::launch_fwd_fp8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-size_t bwd_ws_bytes(long long rows_x_heads, int /*d*/) {
-    // D and lse2 (fp32 each, one per query row and head), each region 256-byte aligned
-    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    return 2 * up(static_cast<size_t>(rows_x_heads) * 4);
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Deterministic backward: D and lse2 (fp32 each, one per query row and head), each
+// region 256-byte aligned.
+size_t bwd_ws_bytes(long long rows_x_heads, int /*d*/) { return 2 * up256(static_cast<size_t>(rows_x_heads) * 4); }
+
+// Single-pass backward: the same two terms, then the fp32 dQ accumulator (d per row).
+size_t fused_ws_bytes(long long rows_x_heads, int d) {
+    return bwd_ws_bytes(rows_x_heads, d) + up256(static_cast<size_t>(rows_x_heads) * d * 4);
 }
 
+// phases: 7 = the deterministic backward's three kernels (bits 0-2), 56 = the
+// single-pass backward's three kernels (bits 3-5); one bit = one kernel.
 int bwd_impl(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
              void *dq, void *dk, void *dv, const Shape &s, float scale, int is_causal, const uint8_t *key_keep,
-             void *workspace, size_t workspace_bytes, void *stream, int phases = 7,
+             void *workspace, size_t workspace_bytes, void *stream, int phases,
              const uint8_t *block_mask = nullptr) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
@@ -244,7 +251,8 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return ATTN_ERR_MISALIGNED;
     const long long rows = s.cu ? s.total * s.H : static_cast<long long>(s.B) * s.H * s.N;
-    const size_t need = bwd_ws_bytes(rows, s.d);
+    const bool fused = (phases & 56) != 0;
+    const size_t need = fused ? fused_ws_bytes(rows, s.d) : bwd_ws_bytes(rows, s.d);
     if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
     DeviceState *ds = nullptr;
@@ -255,6 +263,11 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
         (rc = map_for(&a.tm_do, dout, s)) || (rc = map_for(&a.tm_dk_st, dk, s, 32, false, 32)) ||
         (rc = map_for(&a.tm_dv_st, dv, s, 32, false, 32)))
         return rc;
+    char *w = static_cast<char *>(workspace);
+    if (fused) {
+        a.dqacc = reinterpret_cast<float *>(w + bwd_ws_bytes(rows, s.d));
+        if ((rc = map_for(&a.tm_dqacc, a.dqacc, s, 32, true, 32))) return rc;
+    }
     a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);
     a.o = o;
@@ -263,17 +276,20 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    char *w = static_cast<char *>(workspace);
     a.dvec = reinterpret_cast<float *>(w);
-    a.lse2 = reinterpret_cast<float *>(w + up(static_cast<size_t>(rows) * 4));
+    a.lse2 = reinterpret_cast<float *>(w + up256(static_cast<size_t>(rows) * 4));
     a.rows_total = rows;
     a.scale = scale;
     a.causal = is_causal ? 1 : 0;
     a.phases = phases;
     a.num_sms = ds->num_sms > 0 ? ds->num_sms : 1;
-    return attn::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    const cudaError_t e = fused ? attn::launch_bwd_fused(a, static_cast<cudaStream_t>(stream))
+                                : attn::launch_bwd(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+constexpr int kDeterministicPhases = 7;  // preprocess, dK/dV pass, dQ pass
+constexpr int kFusedPhases = 56;         // preprocess + zeroing, single pass, dQ conversion
 
 }  // namespace
 
@@ -336,12 +352,12 @@ int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void
     if (N > 64 * 128) return ATTN_ERR_UNSUPPORTED;
     Shape s{B, H, N, d, 0, nullptr};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, nullptr, workspace, workspace_bytes,
-                    stream, 7, block_mask);
+                    stream, kFusedPhases, block_mask);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
     if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
-    return bwd_ws_bytes(static_cast<long long>(B) * H * N, d);
+    return fused_ws_bytes(static_cast<long long>(B) * H * N, d);
 }
 
 size_t attn_bwd_deterministic_workspace_bytes(int B, int H, int N, int d) {
@@ -355,12 +371,12 @@ int attn_bwd_deterministic(const void *q, const void *k, const void *v, const vo
                            size_t workspace_bytes, void *stream) {
     Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
-                    stream);
+                    stream, kDeterministicPhases);
 }
 
 size_t attn_bwd_varlen_workspace_bytes(int total_tokens, int H, int d) {
     if (total_tokens < 0 || H <= 0 || (d != 64 && d != 128)) return 0;
-    return bwd_ws_bytes(static_cast<long long>(total_tokens) * H, d);
+    return fused_ws_bytes(static_cast<long long>(total_tokens) * H, d);
 }
 
 int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout, void *dq,
@@ -368,7 +384,7 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o, const f
              const uint8_t *key_keep, void *workspace, size_t workspace_bytes, void *stream) {
     Shape s{B, H, N, d, cu_seqlens ? static_cast<long long>(B) * N : 0, cu_seqlens};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
-                    stream);
+                    stream, kFusedPhases);
 }
 
 int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
@@ -378,14 +394,14 @@ int attn_bwd_varlen(const void *q, const void *k, const void *v, const void *o, 
     if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
     Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
-                    stream);
+                    stream, kFusedPhases);
 }
 
 int attn_bwd_phase(int phase, const void *q, const void *k, const void *v, const void *o, const float *lse,
                    const void *dout, void *dq, void *dk, void *dv, int num_seqs, int total_tokens, int max_seqlen,
                    int H, int d, float scale, int is_causal, const int32_t *cu_seqlens, const uint8_t *key_keep,
                    void *workspace, size_t workspace_bytes, void *stream) {
-    if (phase < 0 || phase > 2) return ATTN_ERR_INVALID_ARG;
+    if (phase < 0 || phase > 5) return ATTN_ERR_INVALID_ARG;
     Shape s{num_seqs, H, max_seqlen, d, cu_seqlens ? static_cast<long long>(total_tokens) : 0, cu_seqlens};
     return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, s, scale, is_causal, key_keep, workspace, workspace_bytes,
                     stream, 1 << phase);

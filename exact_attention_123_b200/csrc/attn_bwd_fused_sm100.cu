@@ -1,0 +1,682 @@
+// attn_bwd_fused_sm100.cu -- single-pass exact-attention backward for B200 (sm_100a).
+//
+// The backward recomputes the probabilities from Q, K and the forward's logsumexp
+// ("4.5 注意力优化实战：从PyTorch到CUDA的完整流程", 第四步 §2: the softmax normaliser
+// kept by the forward is reused; dK and dV sweep the query blocks).  With P the
+// probabilities, dO the upstream gradient and D_i = sum_c dO_ic O_ic:
+//   dV = P^T dO,   dS = P o (dO V^T - D),   dK = scale dS^T Q,   dQ = scale dS K.
+//
+// One persistent kernel does all five tensor-core products of a (key tile, query
+// tile) pair once -- the separate dQ pass of the deterministic backward recomputes
+// S and dP, seven products per pair -- and accumulates dQ in fp32 in device memory:
+//   work unit = one 128-key tile K_j, V_j of one (b, h), sweeping the 128-row query
+//   tiles Q_i, dO_i (from the diagonal when causal):
+//     S^T  = K_j Q_i^T            SS, M = 128 keys, N = 128 queries     -> TMEM
+//     dP^T = V_j dO_i^T           SS                                    -> TMEM
+//     P^T  = 2^(S^T scale log2e - lse2)   written back over S^T as bf16 (math warps)
+//     dS   = P o (dP - D)         written to shared memory as bf16, keys x queries
+//     dV  += P^T dO_i             TS: A = P^T from TMEM
+//     dQ_i = dS K_j               SS: A = dS read query-major (the transposed view
+//                                 of the same shared-memory tile), B = K_j
+//     dK  += dS^T Q_i             SS: A = dS as stored
+//   and four "drain" warps move each dQ_i tile out of TMEM, through shared memory,
+//   into an fp32 accumulator with TMA reduce-adds (the add happens in L2).  A small
+//   kernel first zeroes the accumulator (with the per-row D and lse2 terms) and
+//   another one afterwards writes dQ = bf16(scale * accumulator).
+// The fp32 additions from different key tiles land in an order that depends on
+// scheduling, so dQ may differ between runs in its last bits; the deterministic
+// backward (attn_bwd_sm100.cu) avoids that at the price of the two extra products.
+//
+// Warp roles (512 threads, four warpgroups; registers move by whole warpgroups):
+//   warps 0-7   math: warp w owns key rows 32 (w % 4) .. + 31 (its TMEM lane quadrant)
+//               and query columns 64 (w / 4) .. + 63 of each pair
+//   warps 8-11  dQ drain: warp w reads TMEM lanes 32 (w % 4) .. + 31 = query rows
+//   warp 12     TMA loader (K_j, V_j per unit; Q_i, dO_i and the row terms per step)
+//   warp 13     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 14-15 idle (they complete the warpgroup that gives registers away)
+//
+// Tensor memory (512 columns): S^T / P^T [0, 128), dP^T [128, 256), dV, dK after.
+// The dQ_i accumulator needs d more columns: at d = 64 it has [384, 448) to itself;
+// at d = 128 it takes dP^T's columns once the math warps have read dP^T, and the
+// next dP^T is issued only after the drain warps have read dQ_i out.
+//
+// Shared memory (d = 128): K_j, V_j 32 KB each; Q_i and dO_i in a two-stage ring
+// (128 KB); the dS tile (32 KB), which the drain warps reuse as their staging area
+// once both products that read dS are done; the per-row terms of each stage.
+//
+// Every wait is bounded (see attn_common.cuh); an expired wait stops every role,
+// drains the copies in flight and returns with ATTN_ERR_TIMEOUT in the status word.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "attn_common.cuh"
+#include "attn_launch.h"
+
+namespace attn {
+
+namespace {
+
+constexpr float kLog2eF = 1.4426950408889634f;
+
+template <int D>
+struct FusedCfg {
+    static constexpr int kTile = 128 * D * 2;  // K, V, Q or dO tile (bf16)
+    static constexpr int kBoxes = D / 64;      // 64-column TMA boxes per tile
+    static constexpr int kStages = 2;          // Q_i / dO_i ring
+    static constexpr int kThreads = 512;
+    // Launched at 128 registers per thread (the most 512 threads allow); the drain and
+    // control warpgroups give registers back, the two math warpgroups take them.
+    static constexpr int kLaunchRegs = 128, kRegsMath = 160, kRegsDrain = 104, kRegsCtl = 88;
+    static_assert(2 * 128 * kRegsMath + 128 * kRegsDrain + 128 * kRegsCtl <= kThreads * kLaunchRegs,
+                  "register reallocation exceeds the launch pool");
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+    static constexpr bool kDqOverDp = (D == 128);  // the dQ accumulator reuses dP^T's columns
+    static constexpr int kColDQ = kDqOverDp ? kColDP : 256 + 2 * D;
+    static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
+    static constexpr int kOffK = 0, kOffV = kTile;
+    static constexpr int kOffQ = 2 * kTile;                   // + st * kTile
+    static constexpr int kOffDO = kOffQ + kStages * kTile;    // + st * kTile
+    static constexpr int kOffDS = kOffDO + kStages * kTile;   // 128 keys x 128 queries bf16, two 64-query boxes
+    static constexpr int kOffVec = kOffDS + 32768;            // + st * 1024: lse2[128], D[128]
+    static constexpr int kOffBar = kOffVec + kStages * 1024;
+    static constexpr int kBarKVFull = 0;
+    static constexpr int kBarKVEmpty = 1;                 // K_j, V_j no longer read (unit done)
+    static constexpr int kBarQFull = 2;                   // + st
+    static constexpr int kBarQEmpty = 2 + kStages;        // + st
+    static constexpr int kBarSFull = 2 + 2 * kStages;
+    static constexpr int kBarDPFull = kBarSFull + 1;
+    static constexpr int kBarPFull = kBarSFull + 2;       // P^T in TMEM (256 math threads)
+    static constexpr int kBarDSFull = kBarSFull + 3;      // dS in shared memory, dP^T read (256)
+    static constexpr int kBarDQFull = kBarSFull + 4;      // dQ_i product done
+    static constexpr int kBarDSFree = kBarSFull + 5;      // the products reading dS are done
+    static constexpr int kBarDQFree = kBarSFull + 6;      // dQ_i read out of TMEM (128 drain threads)
+    static constexpr int kBarStageFree = kBarSFull + 7;   // the staging reads are done (128)
+    static constexpr int kBarKdv = kBarSFull + 8;         // dV, dK accumulators complete
+    static constexpr int kBarAccFree = kBarSFull + 9;     // dV, dK copied out of TMEM (256)
+    static constexpr int kBarDone = kBarSFull + 10;
+    static constexpr int kNumBars = kBarSFull + 11;
+    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 16;  // from a 1024-byte-aligned base
+    static constexpr int kSmemMax = 232448;
+    // The base of dynamic shared memory is expected to be 1024-byte aligned; the
+    // kernel checks, and where the slack below cannot cover the misalignment it
+    // reports ATTN_ERR_UNSUPPORTED instead of running.
+    static constexpr int kSmemBytes = (kSmemUsed + 1024 <= kSmemMax) ? kSmemUsed + 1024 : kSmemMax;
+    static_assert(kSmemUsed <= kSmemMax, "exceeds the 227 KB per-CTA shared-memory limit");
+    static_assert(kTile % 1024 == 0 && kOffDS % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
+};
+
+struct FusedParams {
+    Geom g;
+    SyncCtl ctl;
+    __nv_bfloat16 *dk, *dv;
+    const float *dvec, *lse2;
+    float scale;
+    float scale_log2;
+    int causal;
+    int n_tiles;  // 128-row tiles per slice
+};
+
+__device__ __forceinline__ uint32_t kstep(int kk) { return (kk >> 2) * 16384 + (kk & 3) * 32; }
+
+// One warp's 32 rows x 32 fp32 columns into a staging box laid out as the 128-byte
+// swizzle of a {32, 32} fp32 TMA box: row r at r * 128, 16-byte chunk c at
+// (c ^ (r % 8)) * 16.  Lane = row.
+__device__ __forceinline__ void stage_rows32_f32(uint32_t box, const uint32_t (&r)[32], int lane) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        st_shared_v4(box + lane * 128 + (((c ^ (lane & 7)) & 7) << 4), r[4 * c], r[4 * c + 1], r[4 * c + 2],
+                     r[4 * c + 3]);
+}
+
+}  // namespace
+
+template <int D, bool SP>
+__global__ void __launch_bounds__(512, 1)
+attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_dqacc, const __grid_constant__ FusedParams p) {
+    using C = FusedCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+    if (sbase - raw_u32 + C::kSmemUsed > static_cast<uint32_t>(C::kSmemBytes)) {  // uniform over the CTA
+        if (threadIdx.x == 0) atomicCAS(p.ctl.status, 0, kStatusUnsupported);
+        return;
+    }
+    uint8_t *sptr = smem_raw + (sbase - raw_u32);
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+    const int BH = p.g.B * p.g.H;
+    const int T = BH * p.n_tiles;
+    // Work unit of rank r (CTA c takes ranks c, 2G-1-c, 2G+c, ...: a snake order over
+    // the units ranked heaviest first): key tile j, slice (b, h); qs = the query tiles
+    // that attend key tile j, nq of them, walked in increasing order.
+    struct Tile {
+        int b, h, j, start, len, kv0, i0, nq;
+        TileSet qs;
+    };
+    auto tile_at = [&](int r, Tile &t) -> bool {
+        t.j = r / BH;
+        const int bh = r - t.j * BH;
+        t.b = bh / p.g.H;
+        t.h = bh - t.b * p.g.H;
+        p.g.slice(t.b, t.start, t.len);
+        t.kv0 = t.j * 128;
+        if (t.kv0 >= t.len) return false;
+        t.i0 = p.causal ? t.j : 0;
+        t.qs = col_tiles<SP>(p.g, t.h, t.j, t.i0, (t.len + 127) / 128);
+        t.nq = t.qs.count();
+        return true;
+    };
+    auto rank_of = [&](int k) { return k * G + ((k & 1) ? (G - 1 - cta) : cta); };
+
+    if (warp == 13) {
+        tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kNumBars; ++i) {
+            uint32_t cnt = 1;
+            if (i == C::kBarPFull || i == C::kBarDSFull || i == C::kBarAccFree) cnt = 256;
+            if (i == C::kBarDQFree || i == C::kBarStageFree) cnt = 128;
+            mbar_init(bar(i), cnt);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    int n_q = 0, n_kv = 0;  // loader: query-tile and K/V loads started (for the abort drain)
+
+    if (warp >= 12) {
+        setmaxnreg_dec<C::kRegsCtl>();
+        if (warp == 12) {
+            // ------------------------------------------------------------ loader
+            if (lane == 0) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                tma_prefetch_desc(&tm_do);
+            }
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int r = rank_of(k);
+                if (r >= T) break;
+                Tile t;
+                if (!tile_at(r, t) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
+                const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
+                const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
+                // K_j, V_j once every product of the previous unit has been issued and done
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKVEmpty), (n_kv & 1) ^ 1, p.ctl, abort_flag));
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(C::kBarKVFull), 2 * C::kTile);
+#pragma unroll
+                    for (int x = 0; x < C::kBoxes; ++x) {
+                        tma_load_3d(sbase + C::kOffK + x * 16384, &tm_k, bar(C::kBarKVFull), x * 64, row0 + t.kv0,
+                                    slab);
+                        tma_load_3d(sbase + C::kOffV + x * 16384, &tm_v, bar(C::kBarKVFull), x * 64, row0 + t.kv0,
+                                    slab);
+                    }
+                }
+                ++n_kv;
+                for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
+                    const int gi = n_q, st = gi % C::kStages;
+                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
+                                                            p.ctl, abort_flag));
+                    if (!ok) break;
+                    const int q0 = i * 128;
+                    float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int q = q0 + u * 32 + lane;
+                        float l2 = INFINITY, dd = 0.f;  // rows past the sequence: P = 0
+                        if (q < t.len) {
+                            l2 = p.lse2[lrow0 + q * lrs];
+                            dd = p.dvec[lrow0 + q * lrs];
+                        }
+                        vec[u * 32 + lane] = l2;
+                        vec[128 + u * 32 + lane] = dd;
+                    }
+                    __syncwarp();
+                    if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
+                        mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x) {
+                            tma_load_3d(sbase + C::kOffQ + st * C::kTile + x * 16384, &tm_q, bar(C::kBarQFull + st),
+                                        x * 64, row0 + q0, slab);
+                            tma_load_3d(sbase + C::kOffDO + st * C::kTile + x * 16384, &tm_do, bar(C::kBarQFull + st),
+                                        x * 64, row0 + q0, slab);
+                        }
+                    }
+                    ++n_q;
+                }
+            }
+        } else if (warp == 13) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+                constexpr uint32_t idKV = idesc_bf16_f32(128, D, 0, 1);   // dV (TS), dK (A = dS as stored)
+                constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 1, 1);   // dQ (A = dS read query-major)
+                const uint32_t ds = sbase + C::kOffDS;
+                // P^T sits in TMEM with queries 0-63 at columns 0-31 and queries 64-127 at
+                // columns 64-95 of the S^T region (each math warp writes only inside the
+                // columns it read).
+                auto acol = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
+                auto issue_s = [&](int gi) {
+                    const uint32_t qs = sbase + C::kOffQ + (gi % C::kStages) * C::kTile;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::kColS, sw128_desc(sbase + C::kOffK + kstep(kk), 16, 1024),
+                               sw128_desc(qs + kstep(kk), 16, 1024), idS, kk > 0);
+                    tc_commit(bar(C::kBarSFull));
+                };
+                auto issue_dp = [&](int gi) {
+                    const uint32_t dos = sbase + C::kOffDO + (gi % C::kStages) * C::kTile;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffV + kstep(kk), 16, 1024),
+                               sw128_desc(dos + kstep(kk), 16, 1024), idS, kk > 0);
+                    tc_commit(bar(C::kBarDPFull));
+                };
+                auto wait_q = [&](int gi) {
+                    return wait_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+                };
+                bool ok = true;
+                int gbase = 0, n_t = 0;
+                for (int k = 0; ok; ++k) {
+                    const int r = rank_of(k);
+                    if (r >= T) break;
+                    Tile t;
+                    if (!tile_at(r, t) || t.nq == 0) continue;
+                    ok = wait_phase(bar(C::kBarKVFull), n_t & 1, p.ctl, abort_flag);
+                    if (ok) ok = wait_q(gbase);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // S^T's columns are free: the previous unit's last dV, which read P^T from
+                    // them, was issued earlier and tensor-core operations complete in order.
+                    issue_s(gbase);
+                    if (C::kDqOverDp && gbase > 0) {  // dP^T's columns held the previous dQ tile
+                        ok = wait_phase(bar(C::kBarDQFree), (gbase - 1) & 1, p.ctl, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    issue_dp(gbase);
+                    for (int it = 0; ok && it < t.nq; ++it) {
+                        const int gi = gbase + it, st = gi % C::kStages;
+                        const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
+                        const uint32_t dos = sbase + C::kOffDO + st * C::kTile;
+                        const bool more = it + 1 < t.nq;
+                        // dV += P^T dO_i   (K = 128 queries: 8 steps)
+                        ok = wait_phase(bar(C::kBarPFull), gi & 1, p.ctl, abort_flag);
+                        if (ok && it == 0 && n_t > 0)  // the previous unit's dV / dK have been copied out
+                            ok = wait_phase(bar(C::kBarAccFree), (n_t - 1) & 1, p.ctl, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ts(tmem + C::kColDV, tmem + C::kColS + acol(kk),
+                                   sw128_desc(dos + kk * 2048, 16384, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                        // S^T_{i+1} may overwrite P^T_i now: dV_i, issued first, completes first
+                        // (the math warps keep their P in registers for dS).
+                        if (more) {
+                            ok = wait_q(gi + 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_s(gi + 1);
+                        }
+                        ok = wait_phase(bar(C::kBarDSFull), gi & 1, p.ctl, abort_flag);
+                        if (ok && !C::kDqOverDp && gi > 0)  // the dQ columns held the previous tile
+                            ok = wait_phase(bar(C::kBarDQFree), (gi - 1) & 1, p.ctl, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        // dQ_i = dS K_j  (K = 128 keys; A = dS with the queries contiguous, B = K_j
+                        // with d contiguous: both read across their 128-byte rows)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(tmem + C::kColDQ, sw128_desc(ds + kk * 2048, 16384, 1024),
+                                   sw128_desc(sbase + C::kOffK + kk * 2048, 16384, 1024), idDQ, kk > 0 ? 1u : 0u);
+                        tc_commit(bar(C::kBarDQFull));
+                        // dK += dS^T Q_i  (K = 128 queries; A = dS as stored, keys x queries)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(tmem + C::kColDK, sw128_desc(ds + kstep(kk), 16, 1024),
+                                   sw128_desc(qs + kk * 2048, 16384, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(bar(C::kBarDSFree));
+                        tc_commit(bar(C::kBarQEmpty + st));  // dK_i was the last reader of Q_i, dV_i of dO_i
+                        if (more) {
+                            if (C::kDqOverDp) {  // dP^T_{i+1} overwrites the dQ_i accumulator
+                                ok = wait_phase(bar(C::kBarDQFree), gi & 1, p.ctl, abort_flag);
+                                if (!ok) break;
+                                tc_fence_after();
+                            }
+                            issue_dp(gi + 1);
+                        }
+                    }
+                    if (!ok) break;
+                    tc_commit(bar(C::kBarKVEmpty));
+                    tc_commit(bar(C::kBarKdv));
+                    gbase += t.nq;
+                    ++n_t;
+                }
+                // Every MMA issued above must have finished before TMEM / smem go away.
+                tc_commit(bar(C::kBarDone));
+                drain_phase(bar(C::kBarDone), 0, p.ctl, abort_flag);
+            }
+        }
+    } else if (warp >= 8) {
+        setmaxnreg_dec<C::kRegsDrain>();
+        // ---------------------------------------------------------------- dQ drain
+        // warp w: query rows 32 (w % 4) .. + 31 of each dQ_i tile; its 8 KB of the dS
+        // area hold two {32 x 32} fp32 boxes.
+        const int q4 = warp & 3;
+        const uint32_t tdq = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kColDQ;
+        const uint32_t box0 = sbase + C::kOffDS + q4 * 8192, box1 = box0 + 4096;
+        bool ok = true;
+        int gbase = 0;
+        for (int k = 0; ok; ++k) {
+            const int r = rank_of(k);
+            if (r >= T) break;
+            Tile t;
+            if (!tile_at(r, t) || t.nq == 0) continue;
+            const int row0 = p.g.tma_row0(t.start) + q4 * 32, slab = p.g.tma_slab(t.b, t.h);
+            for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
+                const int gi = gbase + it;
+                const int row = row0 + i * 128;
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDQFull), gi & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tdq, r0);
+                tmem_ld32(tdq + 32, r1);
+                tmem_wait_ld();
+                if constexpr (!C::kDqOverDp) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarDQFree));
+                }
+                // the dS area is the staging area once dQ_i and dK_i have read dS
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDSFree), gi & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                stage_rows32_f32(box0, r0, lane);
+                stage_rows32_f32(box1, r1, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_3d(&tm_dqacc, box0, 0, row, slab);
+                    tma_reduce_add_3d(&tm_dqacc, box1, 32, row, slab);
+                    bulk_commit();
+                }
+                if constexpr (C::kDqOverDp) {
+                    tmem_ld32(tdq + 64, r0);
+                    tmem_ld32(tdq + 96, r1);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarDQFree));
+                    if (lane == 0) bulk_wait_read0();  // the first two boxes have been read
+                    __syncwarp();
+                    stage_rows32_f32(box0, r0, lane);
+                    stage_rows32_f32(box1, r1, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_3d(&tm_dqacc, box0, 64, row, slab);
+                        tma_reduce_add_3d(&tm_dqacc, box1, 96, row, slab);
+                        bulk_commit();
+                    }
+                }
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+                mbar_arrive(bar(C::kBarStageFree));  // the math warps may write the next dS
+            }
+            if (!ok) break;
+            gbase += t.nq;
+        }
+        if (lane == 0) bulk_wait0();  // every reduce-add of this warp has landed
+    } else {
+        setmaxnreg_inc<C::kRegsMath>();
+        // ---------------------------------------------------------------- P^T and dS (warps 0-7)
+        // warp w: key rows 32 (w % 4) .., query columns 64 (w / 4) .. + 63 of each query tile.
+        const int q4 = warp & 3, hf = warp >> 2;
+        const int kr = q4 * 32 + lane;  // key row within the tile
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::kColS + hf * 64;
+        const uint32_t tDP = tmem + lane_off + C::kColDP + hf * 64;
+        // this thread's row of the dS tile: box hf (queries 64 hf ..), row kr, 128-byte
+        // swizzle (chunk c at (c ^ kr % 8) * 16)
+        const uint32_t dsrow = sbase + C::kOffDS + hf * 16384 + (kr >> 3) * 1024 + (kr & 7) * 128;
+        const float c2 = p.scale_log2;
+        bool ok = true;
+        int gbase = 0, n_t = 0;
+        for (int k = 0; ok; ++k) {
+            const int r = rank_of(k);
+            if (r >= T) break;
+            Tile t;
+            if (!tile_at(r, t)) continue;
+            const int key = t.kv0 + kr;
+            if (t.nq == 0) {
+                // The tile mask leaves key tile j no query tile: dV = dK = 0 for its keys
+                // (warps 0-3 write dV, 4-7 dK), and nothing was computed.
+                if (key < t.len) {
+                    uint4 *dst = reinterpret_cast<uint4 *>((hf == 0 ? p.dv : p.dk) + p.g.base(t.b, t.h, t.start, D) +
+                                                           static_cast<long long>(key) * p.g.row_stride(D));
+#pragma unroll 1
+                    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
+            bool kvalid = key < t.len;
+            if (kvalid && p.g.key_keep) kvalid = p.g.key_keep[p.g.keep_base(t.b, t.start) + key] != 0;
+            for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
+                const int gi = gbase + it, st = gi % C::kStages;
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarSFull), gi & 1, p.ctl, abort_flag));
+                if (ok)
+                    ok = __all_sync(0xffffffffu,
+                                    wait_phase(bar(C::kBarQFull + st), (gi / C::kStages) & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                const float4 *vec = reinterpret_cast<const float4 *>(sptr + C::kOffVec + st * 1024) + hf * 16;
+                uint32_t sr[2][32];
+                tmem_ld32(tS, sr[0]);
+                tmem_ld32(tS + 32, sr[1]);
+                tmem_wait_ld();
+                // P^T = 2^(S^T c - lse2), 0 where the query precedes the key (causal),
+                // for keys outside the sequence or padded, and for rows past the end.
+                const int qb = i * 128 + hf * 64;  // first query column of this warp
+                int lim = p.causal ? key - qb : 0;  // columns c < lim are masked
+                if (!kvalid) lim = 64;
+                float pf[64];
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 l2 = vec[c4];
+                    const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = c4 * 4 + e;
+                        pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2v[e]));
+                    }
+                }
+                if (lim > 0) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < lim) pf[c] = 0.f;
+                }
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pf[x * 32 + 2 * c], pf[x * 32 + 2 * c + 1]);
+                    tmem_st16(tS + x * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::kBarPFull));
+                // dS = P o (dP - D), P taken from registers (fp32), into shared memory
+                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDPFull), gi & 1, p.ctl, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t pk[32];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    uint32_t dr[32];
+                    tmem_ld32(tDP + x * 32, dr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 dd = vec[32 + x * 8 + c4];
+                        const int c = x * 32 + c4 * 4;
+                        pk[x * 16 + 2 * c4] = pack_bf16x2(pf[c] * (__uint_as_float(dr[c4 * 4]) - dd.x),
+                                                          pf[c + 1] * (__uint_as_float(dr[c4 * 4 + 1]) - dd.y));
+                        pk[x * 16 + 2 * c4 + 1] = pack_bf16x2(pf[c + 2] * (__uint_as_float(dr[c4 * 4 + 2]) - dd.z),
+                                                              pf[c + 3] * (__uint_as_float(dr[c4 * 4 + 3]) - dd.w));
+                    }
+                }
+                // the drain warps must have finished with the previous dQ tile's staging
+                if (gi > 0) {
+                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarStageFree), (gi - 1) & 1, p.ctl, abort_flag));
+                    if (!ok) break;
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(dsrow + (((c ^ (kr & 7)) & 7) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                                 pk[4 * c + 3]);
+                fence_proxy_async_smem();  // dS is read by the tensor core (async proxy)
+                tc_fence_before();         // and dP^T's columns have been read (dQ_i may overwrite them)
+                mbar_arrive(bar(C::kBarDSFull));
+            }
+            if (!ok) break;
+            // ---- epilogue: warps 0-3 write dV, warps 4-7 write scale * dK; TMEM is
+            // released (acc free) as soon as the values are in registers
+            ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKdv), n_t & 1, p.ctl, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const bool is_dv = hf == 0;
+            __nv_bfloat16 *out = (is_dv ? p.dv : p.dk) + p.g.base(t.b, t.h, t.start, D) +
+                                 static_cast<long long>(key) * p.g.row_stride(D);
+            const float mul = is_dv ? 1.f : p.scale;
+            const uint32_t col = is_dv ? C::kColDV : C::kColDK;
+            const bool valid = key < t.len;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld32(tmem + lane_off + col + c0, rr);
+                tmem_wait_ld();
+                if (c0 + 32 == D) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::kBarAccFree));
+                }
+                uint32_t o[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    o[c] = pack_bf16x2(__uint_as_float(rr[2 * c]) * mul, __uint_as_float(rr[2 * c + 1]) * mul);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + c0);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                }
+            }
+            gbase += t.nq;
+            ++n_t;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 12 && lane == 0 && *abort_flag) {
+        // After an abort, every copy the loader started must land before the CTA exits.
+        if (n_kv > 0) drain_phase(bar(C::kBarKVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
+            if (gi != p.ctl.inject_skip_load)
+                drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+    }
+    if (warp == 13) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// dQ = bf16(scale * accumulator) over the rows that hold tokens (the flat [rows, d]
+// order of q's layout); 8 elements per thread and iteration.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float *__restrict__ acc,
+                                                                  __nv_bfloat16 *__restrict__ dq, long long rows,
+                                                                  float scale, const int32_t *cu_seqlens, int nseq,
+                                                                  int H) {
+    long long limit = rows;
+    if (cu_seqlens) limit = min(rows, static_cast<long long>(cu_seqlens[nseq]) * H);
+    const long long n8 = limit * (D / 8);
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+        const float4 a = reinterpret_cast<const float4 *>(acc)[2 * i];
+        const float4 b = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+        reinterpret_cast<uint4 *>(dq)[i] =
+            make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                       pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+    }
+}
+
+template <int D, bool SP>
+static cudaError_t launch_fused_d(const BwdLaunch &a, cudaStream_t stream) {
+    using C = FusedCfg<D>;
+    cudaError_t e;
+    if (a.phases & 8) {
+        if ((e = launch_bwd_pre(a, true, stream)) != cudaSuccess) return e;
+    }
+    if (a.phases & 16) {
+        FusedParams p{};
+        p.g = a.g;
+        p.ctl = a.ctl;
+        p.dk = static_cast<__nv_bfloat16 *>(a.dk);
+        p.dv = static_cast<__nv_bfloat16 *>(a.dv);
+        p.dvec = a.dvec;
+        p.lse2 = a.lse2;
+        p.scale = a.scale;
+        p.scale_log2 = a.scale * kLog2eF;
+        p.causal = a.causal;
+        p.n_tiles = (a.g.N + 127) / 128;
+        e = cudaFuncSetAttribute(attn_bwd_fused_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        // The in-kernel register reallocation assumes the launch register count it was
+        // sized for; with fewer, an increase could never be satisfied, so refuse.
+        static const cudaError_t regs_ok = [] {
+            cudaFuncAttributes fa{};
+            const cudaError_t r = cudaFuncGetAttributes(&fa, attn_bwd_fused_sm100_kernel<D, SP>);
+            if (r != cudaSuccess) return r;
+            return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
+        }();
+        if (regs_ok != cudaSuccess) return regs_ok;
+        const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_tiles;
+        const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
+        attn_bwd_fused_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v,
+                                                                                         a.tm_do, a.tm_dqacc, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (a.phases & 32) {
+        const long long n8 = a.rows_total * (D / 8);
+        const long long want = (n8 + 255) / 256;
+        const unsigned blocks = static_cast<unsigned>(want < 148LL * 16 ? (want > 0 ? want : 1) : 148LL * 16);
+        attn_bwd_dq_convert_kernel<D><<<blocks, 256, 0, stream>>>(a.dqacc, static_cast<__nv_bfloat16 *>(a.dq),
+                                                                  a.rows_total, a.scale,
+                                                                  a.g.varlen ? a.g.cu_seqlens : nullptr, a.g.B, a.g.H);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_bwd_fused(const BwdLaunch &a, cudaStream_t stream) {
+    const bool sp = a.g.block_mask != nullptr;
+    if (a.g.d == 128) return sp ? launch_fused_d<128, true>(a, stream) : launch_fused_d<128, false>(a, stream);
+    return sp ? launch_fused_d<64, true>(a, stream) : launch_fused_d<64, false>(a, stream);
+}
+
+}  // namespace attn

@@ -57,12 +57,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 // kernel is HBM-bound).  Rows are in the lse layout order, which is
 // also the row order of the flat [rows, d] view of O and dO.
 constexpr int kPrePasses = 4;
+// With a non-null dqacc (the single-pass backward) the kernel also zeroes the fp32 dQ
+// accumulator's rows (same flat [rows, d] order), which the fused kernel then adds into.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *__restrict__ o,
                                                           const __nv_bfloat16 *__restrict__ dout,
                                                           const float *__restrict__ lse, float *__restrict__ dvec,
-                                                          float *__restrict__ lse2, long long rows,
-                                                          const int32_t *cu_seqlens, int nseq, int H) {
+                                                          float *__restrict__ lse2, float *__restrict__ dqacc,
+                                                          long long rows, const int32_t *cu_seqlens, int nseq, int H) {
     constexpr int TPR = D / 8;          // threads per row
     constexpr int RPP = 256 / TPR;      // rows per pass
     long long limit = rows;
@@ -99,6 +101,11 @@ __global__ void __launch_bounds__(256) attn_bwd_pre_kernel(const __nv_bfloat16 *
             dvec[row] = acc;
             const float L = lse[row];
             lse2[row] = (L == -INFINITY) ? INFINITY : L * kLog2e;
+        }
+        if (dqacc != nullptr && row < limit) {
+            float4 *z = reinterpret_cast<float4 *>(dqacc + row * D + part * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = z[0];
         }
     }
 }
@@ -928,10 +935,25 @@ attn_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_
 }
 
 // ============================================================================ launch
+cudaError_t launch_bwd_pre(const BwdLaunch &a, bool zero_dqacc, cudaStream_t stream) {
+    const int *cu = a.g.varlen ? a.g.cu_seqlens : nullptr;
+    const int D = a.g.d;
+    const long long rows_per_cta = (256 / (D / 8)) * kPrePasses;
+    const unsigned blocks = static_cast<unsigned>((a.rows_total + rows_per_cta - 1) / rows_per_cta);
+    float *z = zero_dqacc ? a.dqacc : nullptr;
+    const auto *o = static_cast<const __nv_bfloat16 *>(a.o);
+    const auto *dout = static_cast<const __nv_bfloat16 *>(a.dout);
+    if (D == 128)
+        attn_bwd_pre_kernel<128><<<blocks, 256, 0, stream>>>(o, dout, a.lse, a.dvec, a.lse2, z, a.rows_total, cu,
+                                                             a.g.B, a.g.H);
+    else
+        attn_bwd_pre_kernel<64><<<blocks, 256, 0, stream>>>(o, dout, a.lse, a.dvec, a.lse2, z, a.rows_total, cu,
+                                                            a.g.B, a.g.H);
+    return cudaGetLastError();
+}
+
 template <int D, bool SP>
 static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
-    const int nseq = a.g.B;
-    const int *cu = a.g.varlen ? a.g.cu_seqlens : nullptr;
     BwdParams p{};
     p.g = a.g;
     p.ctl = a.ctl;
@@ -945,12 +967,7 @@ static cudaError_t launch_bwd_d(const BwdLaunch &a, cudaStream_t stream) {
     p.causal = a.causal;
     p.n_tiles = (a.g.N + 127) / 128;
     if (a.phases & 1) {
-        const long long rows_per_cta = (256 / (D / 8)) * kPrePasses;
-        const unsigned blocks = static_cast<unsigned>((a.rows_total + rows_per_cta - 1) / rows_per_cta);
-        attn_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(a.o),
-                                                           static_cast<const __nv_bfloat16 *>(a.dout), a.lse, a.dvec,
-                                                           a.lse2, a.rows_total, cu, nseq, a.g.H);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_bwd_pre(a, false, stream);
         if (e != cudaSuccess) return e;
     }
     // dK/dV then dQ, as two launches: one grid holding both kinds of CTA measured

@@ -11,7 +11,8 @@
 namespace attn {
 
 constexpr int kStatusOk = 0;
-constexpr int kStatusTimeout = 6;  // ATTN_ERR_TIMEOUT
+constexpr int kStatusUnsupported = 2;  // ATTN_ERR_UNSUPPORTED (a launch that cannot run as configured)
+constexpr int kStatusTimeout = 6;      // ATTN_ERR_TIMEOUT
 
 // Geometry of one (sequence, head) slice, common to dense and packed layouts.
 // A tensor element (row r, column c) of slice (b, h) sits at

@@ -76,6 +76,11 @@ struct FwdCfg {
     static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
                   "register reallocation exceeds the launch pool");
     static constexpr int kTmemCols = 512;
+    // column pairs c (of each 32-pair half row) whose exponentials come from the FMA
+    // pipe: bit (c % 8) set.  Measured best: one pair in eight with e4m3 operands and
+    // with bf16 at d = 64 (where the exponentials outweigh the products), none at
+    // bf16 d = 128.
+    static constexpr uint32_t kPolyPairs = (F8 || D == 64) ? 0x80u : 0u;
     static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
     // barrier indices
     static constexpr int kBarQ = 0;
@@ -376,6 +381,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const TileSet ts = t ? u.ts1 : u.ts0;  // the key tiles this tile attends
         bool first_step = true;
         for (int j = ts.next(0); j < ts.hi; j = ts.next(j + 1), ++gs) {
+            const int kbase = j * 128;
+            // the key-padding flags of this key tile (128 bytes, at most two cache lines)
+            // are brought into L1 before waiting for S, so that reading them below does
+            // not add a trip to L2 to the softmax chain
+            if (keep != nullptr && lane < 2) prefetch_l1(keep + kbase + lane * 127);
             ok = wait_phase(bar(C::kBarS + t), gs & 1, p.ctl, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -388,7 +398,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
 
             // ---- masking: keys outside the sequence, above the diagonal, or padded
-            const int kbase = j * 128;
             int limit = len - kbase;
             if (p.causal) limit = min(limit, row - kbase + 1);
             if (limit < 128) {
@@ -443,10 +452,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int c = 0; c < 32; ++c) {
                     const uint64_t x2 = f2_fma(f2_pack(s[half * 64 + 2 * c], s[half * 64 + 2 * c + 1]), c2x2, negm2);
                     float p0, p1;
-                    if ((F8 || D == 64) && (c & 7) == 7) {
+                    if ((C::kPolyPairs >> (c & 7)) & 1u) {
                         // Where the products take half the time of the exponentials (e4m3
                         // operands at d = 128, bf16 at d = 64) the MUFU unit sets the pace, so
-                        // one pair in eight goes to the FMA pipe
+                        // some column pairs go to the FMA pipe
                         ex2_poly_x2(x2, p0, p1);
                     } else {
                         float x0, x1;

@@ -24,6 +24,7 @@ struct FwdLaunch {
 struct BwdLaunch {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;  // same map shape as the forward (128-row boxes)
     CUtensorMap tm_dk_st, tm_dv_st;       // dK, dV stores: 32 x 32 boxes, 64-byte swizzle
+    CUtensorMap tm_dqacc;                 // fp32 dQ accumulator reduce-adds: 32 x 32 boxes, 128-byte swizzle
     Geom g;
     SyncCtl ctl;
     const void *o, *dout;
@@ -31,15 +32,21 @@ struct BwdLaunch {
     void *dq, *dk, *dv;
     float *dvec;       // fp32 D_i = rowsum(dO o O), lse layout (workspace)
     float *lse2;       // fp32 lse * log2(e), +inf for empty rows, lse layout (workspace)
+    float *dqacc;      // fp32 dQ accumulator, q's layout (workspace; single-pass backward only)
     long long rows_total;  // token rows (packed) or B*H*N (dense) of the lse layout
     float scale;
     int causal;
-    int phases;        // bit 0: preprocess, bit 1: dK/dV kernel, bit 2: dQ kernel
+    int phases;        // deterministic: bit 0 preprocess, bit 1 dK/dV kernel, bit 2 dQ kernel;
+                       // single pass: bit 3 preprocess + zero dQ accumulator, bit 4 fused
+                       // dK/dV/dQ kernel, bit 5 dQ accumulator -> bf16
     int num_sms;       // persistent grid size
 };
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream);
 cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream);  // tm_q/tm_k/tm_v: e4m3 maps
 cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream);
+// the backward's per-row terms D and lse2 (and, with zero_dqacc, zeroes a.dqacc)
+cudaError_t launch_bwd_pre(const BwdLaunch &a, bool zero_dqacc, cudaStream_t stream);
+cudaError_t launch_bwd_fused(const BwdLaunch &a, cudaStream_t stream);  // phases bits 3-5
 
 }  // namespace attn

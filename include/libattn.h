@@ -97,8 +97,9 @@ ATTN_API int attn_fwd_masked(const void *q, const void *k, const void *v, void *
 
 /*
  * Bytes of device workspace attn_bwd needs for these sizes (for packed inputs,
- * pass the same B and N as to attn_bwd; the bound B*N >= total is used).
- * Returns 0 for invalid sizes.
+ * pass the same B and N as to attn_bwd; the bound B*N >= total is used): two
+ * fp32 terms per query row and head, plus the fp32 dQ accumulator (d per query
+ * row and head).  Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -113,6 +114,11 @@ ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
  *   workspace  : caller-owned device memory of at least
  *                attn_bwd_workspace_bytes(B, H, N, d) bytes, 256-byte aligned;
  *                its contents are scratch and need no initialisation.
+ * One pass per 128-key tile computes every product of the method once; the
+ * contributions of the key tiles to dQ are summed in an fp32 accumulator in the
+ * workspace (fp32 accumulation, "4.5 注意力优化实战" 第四步 §2 backward).  Their
+ * order of arrival depends on scheduling, so dq may differ between calls in its
+ * last bits; attn_bwd_deterministic gives bit-identical results.
  * Returns an attn_status_t code.
  */
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -162,20 +168,26 @@ ATTN_API int attn_bwd_varlen(const void *q, const void *k, const void *v, const 
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * One of the three kernels of the deterministic backward (attn_bwd_deterministic
- * launches all three in this order); lets a caller time or schedule them
- * separately, and gives the packed layout its deterministic backward.
+ * One kernel of one of the two backward algorithms; lets a caller time or schedule
+ * them separately, and gives the packed layout its deterministic backward.
+ * Deterministic backward (attn_bwd_deterministic launches phases 0, 1, 2 in order):
  *   phase 0 : per-row terms D_i = rowsum(dO o O) and lse2 = lse*log2(e), in
  *             `workspace`
  *   phase 1 : dK and dV (one pass per 128-key tile over the query tiles)
  *   phase 2 : dQ (one pass per 128-row query tile over the key tiles)
- * Phases 1 and 2 both read only the inputs and phase 0's terms, so after phase 0
- * they may run in either order (or concurrently on two streams).
+ *   Phases 1 and 2 both read only the inputs and phase 0's terms, so after phase 0
+ *   they may run in either order (or concurrently on two streams).  The workspace
+ *   needs at least attn_bwd_deterministic_workspace_bytes bytes (for the packed
+ *   layout with B = 1, N = total_tokens).
+ * Single-pass backward (attn_bwd / attn_bwd_varlen launch phases 3, 4, 5 in order):
+ *   phase 3 : the terms of phase 0, and zeroes the fp32 dQ accumulator
+ *   phase 4 : dK, dV and the dQ accumulator (one pass per 128-key tile)
+ *   phase 5 : dq = bf16(scale * accumulator)
+ *   The workspace needs at least attn_bwd_workspace_bytes (dense) or
+ *   attn_bwd_varlen_workspace_bytes (packed) bytes.
  * Phases must run in order on the same workspace and stream.  Other arguments as
  * attn_bwd_varlen; for the dense layout pass cu_seqlens = NULL, num_seqs = B,
- * max_seqlen = N and total_tokens = 0.  The workspace needs at least
- * attn_bwd_deterministic_workspace_bytes bytes (for the packed layout with
- * B = 1, N = total_tokens).
+ * max_seqlen = N and total_tokens = 0.
  */
 ATTN_API int attn_bwd_phase(int phase, const void *q, const void *k, const void *v, const void *o,
                             const float *lse, const void *dout, void *dq, void *dk, void *dv,
@@ -289,7 +301,9 @@ ATTN_API int attn_bwd_noalloc(const void *q, const void *k, const void *v, const
 /*
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait
- * expired since the last call, or ATTN_ERR_CUDA if synchronisation failed.
+ * expired since the last call, ATTN_ERR_UNSUPPORTED if a kernel found its shared
+ * memory laid out in a way it cannot run with (and did nothing), or ATTN_ERR_CUDA
+ * if synchronisation failed.
  */
 ATTN_API int attn_status(void *stream);
 
