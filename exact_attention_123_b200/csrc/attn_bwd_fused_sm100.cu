@@ -40,9 +40,13 @@
 // at d = 128 it takes dP^T's columns once the math warps have read dP^T, and the
 // next dP^T is issued only after the drain warps have read dQ_i out.
 //
-// Shared memory (d = 128): K_j, V_j 32 KB each; Q_i and dO_i in a two-stage ring
-// (128 KB); the dS tile (32 KB), which the drain warps reuse as their staging area
-// once both products that read dS are done; the per-row terms of each stage.
+// Shared memory (d = 128): K_j, V_j 32 KB each; Q_i in a two-stage ring with its
+// per-row terms; dO_i in one buffer (it is free again once dV_i is done, well
+// before dP^T_{i+1} is issued); the dS tile (32 KB); the drain warps' staging area
+// (32 KB: two 4 KB boxes per warp, reused as soon as the TMA has read them).
+// The next dS is written only after dP^T_{i+1} is complete, which (tensor-core
+// operations completing in issue order) implies dQ_i and dK_i, the products that
+// read dS, are done.
 //
 // Every wait is bounded (see attn_common.cuh); an expired wait stops every role,
 // drains the copies in flight and returns with ATTN_ERR_TIMEOUT in the status word.
@@ -64,11 +68,12 @@ template <int D>
 struct FusedCfg {
     static constexpr int kTile = 128 * D * 2;  // K, V, Q or dO tile (bf16)
     static constexpr int kBoxes = D / 64;      // 64-column TMA boxes per tile
-    static constexpr int kStages = 2;          // Q_i / dO_i ring
+    static constexpr int kStages = 2;                      // Q_i ring (and its per-row terms)
+    static constexpr int kDoStages = (D == 128) ? 1 : 2;   // dO_i buffers
     static constexpr int kThreads = 512;
     // Launched at 128 registers per thread (the most 512 threads allow); the drain and
     // control warpgroups give registers back, the two math warpgroups take them.
-    static constexpr int kLaunchRegs = 128, kRegsMath = 160, kRegsDrain = 104, kRegsCtl = 88;
+    static constexpr int kLaunchRegs = 128, kRegsMath = 160, kRegsDrain = 96, kRegsCtl = 96;
     static_assert(2 * 128 * kRegsMath + 128 * kRegsDrain + 128 * kRegsCtl <= kThreads * kLaunchRegs,
                   "register reallocation exceeds the launch pool");
     static constexpr int kTmemCols = 512;
@@ -78,26 +83,27 @@ struct FusedCfg {
     static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
     static constexpr int kOffK = 0, kOffV = kTile;
     static constexpr int kOffQ = 2 * kTile;                   // + st * kTile
-    static constexpr int kOffDO = kOffQ + kStages * kTile;    // + st * kTile
-    static constexpr int kOffDS = kOffDO + kStages * kTile;   // 128 keys x 128 queries bf16, two 64-query boxes
-    static constexpr int kOffVec = kOffDS + 32768;            // + st * 1024: lse2[128], D[128]
+    static constexpr int kOffDO = kOffQ + kStages * kTile;     // + buffer * kTile
+    static constexpr int kOffDS = kOffDO + kDoStages * kTile;  // 128 keys x 128 queries bf16, two 64-query boxes
+    static constexpr int kOffStage = kOffDS + 32768;           // + warp * 8192: two {32 x 32} fp32 boxes
+    static constexpr int kOffVec = kOffStage + 32768;          // + st * 1024: lse2[128], D[128]
     static constexpr int kOffBar = kOffVec + kStages * 1024;
     static constexpr int kBarKVFull = 0;
-    static constexpr int kBarKVEmpty = 1;                 // K_j, V_j no longer read (unit done)
-    static constexpr int kBarQFull = 2;                   // + st
-    static constexpr int kBarQEmpty = 2 + kStages;        // + st
-    static constexpr int kBarSFull = 2 + 2 * kStages;
+    static constexpr int kBarKVEmpty = 1;                      // K_j, V_j no longer read (unit done)
+    static constexpr int kBarQFull = 2;                        // + st
+    static constexpr int kBarQEmpty = kBarQFull + kStages;     // + st
+    static constexpr int kBarDOFull = kBarQEmpty + kStages;    // + buffer
+    static constexpr int kBarDOEmpty = kBarDOFull + kDoStages; // + buffer
+    static constexpr int kBarSFull = kBarDOEmpty + kDoStages;
     static constexpr int kBarDPFull = kBarSFull + 1;
     static constexpr int kBarPFull = kBarSFull + 2;       // P^T in TMEM (256 math threads)
     static constexpr int kBarDSFull = kBarSFull + 3;      // dS in shared memory, dP^T read (256)
     static constexpr int kBarDQFull = kBarSFull + 4;      // dQ_i product done
-    static constexpr int kBarDSFree = kBarSFull + 5;      // the products reading dS are done
-    static constexpr int kBarDQFree = kBarSFull + 6;      // dQ_i read out of TMEM (128 drain threads)
-    static constexpr int kBarStageFree = kBarSFull + 7;   // the staging reads are done (128)
-    static constexpr int kBarKdv = kBarSFull + 8;         // dV, dK accumulators complete
-    static constexpr int kBarAccFree = kBarSFull + 9;     // dV, dK copied out of TMEM (256)
-    static constexpr int kBarDone = kBarSFull + 10;
-    static constexpr int kNumBars = kBarSFull + 11;
+    static constexpr int kBarDQFree = kBarSFull + 5;      // dQ_i read out of TMEM (128 drain threads)
+    static constexpr int kBarKdv = kBarSFull + 6;         // dV, dK accumulators complete
+    static constexpr int kBarAccFree = kBarSFull + 7;     // dV, dK copied out of TMEM (256)
+    static constexpr int kBarDone = kBarSFull + 8;
+    static constexpr int kNumBars = kBarSFull + 9;
     static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 16;  // from a 1024-byte-aligned base
     static constexpr int kSmemMax = 232448;
     // The base of dynamic shared memory is expected to be 1024-byte aligned; the
@@ -105,7 +111,8 @@ struct FusedCfg {
     // reports ATTN_ERR_UNSUPPORTED instead of running.
     static constexpr int kSmemBytes = (kSmemUsed + 1024 <= kSmemMax) ? kSmemUsed + 1024 : kSmemMax;
     static_assert(kSmemUsed <= kSmemMax, "exceeds the 227 KB per-CTA shared-memory limit");
-    static_assert(kTile % 1024 == 0 && kOffDS % 1024 == 0, "swizzled tiles must be 1024-byte aligned");
+    static_assert(kTile % 1024 == 0 && kOffDS % 1024 == 0 && kOffStage % 1024 == 0,
+                  "swizzled tiles must be 1024-byte aligned");
 };
 
 struct FusedParams {
@@ -185,7 +192,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         for (int i = 0; i < C::kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i == C::kBarPFull || i == C::kBarDSFull || i == C::kBarAccFree) cnt = 256;
-            if (i == C::kBarDQFree || i == C::kBarStageFree) cnt = 128;
+            if (i == C::kBarDQFree) cnt = 128;
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
@@ -195,7 +202,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    int n_q = 0, n_kv = 0;  // loader: query-tile and K/V loads started (for the abort drain)
+    int n_q = 0, n_do = 0, n_kv = 0;  // loader: Q, dO and K/V loads started (for the abort drain)
 
     if (warp >= 12) {
         setmaxnreg_dec<C::kRegsCtl>();
@@ -249,16 +256,26 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     }
                     __syncwarp();
                     if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
-                        mbar_arrive_expect_tx(bar(C::kBarQFull + st), 2 * C::kTile);
+                        mbar_arrive_expect_tx(bar(C::kBarQFull + st), C::kTile);
 #pragma unroll
-                        for (int x = 0; x < C::kBoxes; ++x) {
+                        for (int x = 0; x < C::kBoxes; ++x)
                             tma_load_3d(sbase + C::kOffQ + st * C::kTile + x * 16384, &tm_q, bar(C::kBarQFull + st),
                                         x * 64, row0 + q0, slab);
-                            tma_load_3d(sbase + C::kOffDO + st * C::kTile + x * 16384, &tm_do, bar(C::kBarQFull + st),
-                                        x * 64, row0 + q0, slab);
-                        }
                     }
                     ++n_q;
+                    // dO_i once dV of the step that last used its buffer is done
+                    const int db = gi % C::kDoStages;
+                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDOEmpty + db), ((gi / C::kDoStages) & 1) ^ 1,
+                                                            p.ctl, abort_flag));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(C::kBarDOFull + db), C::kTile);
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            tma_load_3d(sbase + C::kOffDO + db * C::kTile + x * 16384, &tm_do, bar(C::kBarDOFull + db),
+                                        x * 64, row0 + q0, slab);
+                    }
+                    ++n_do;
                 }
             }
         } else if (warp == 13) {
@@ -281,7 +298,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     tc_commit(bar(C::kBarSFull));
                 };
                 auto issue_dp = [&](int gi) {
-                    const uint32_t dos = sbase + C::kOffDO + (gi % C::kStages) * C::kTile;
+                    const uint32_t dos = sbase + C::kOffDO + (gi % C::kDoStages) * C::kTile;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
                         mma_ss(tmem + C::kColDP, sw128_desc(sbase + C::kOffV + kstep(kk), 16, 1024),
@@ -290,6 +307,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 };
                 auto wait_q = [&](int gi) {
                     return wait_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+                };
+                auto wait_do = [&](int gi) {
+                    return wait_phase(bar(C::kBarDOFull + gi % C::kDoStages), (gi / C::kDoStages) & 1, p.ctl,
+                                      abort_flag);
                 };
                 bool ok = true;
                 int gbase = 0, n_t = 0;
@@ -305,16 +326,16 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     // S^T's columns are free: the previous unit's last dV, which read P^T from
                     // them, was issued earlier and tensor-core operations complete in order.
                     issue_s(gbase);
-                    if (C::kDqOverDp && gbase > 0) {  // dP^T's columns held the previous dQ tile
+                    if (C::kDqOverDp && gbase > 0)  // dP^T's columns held the previous dQ tile
                         ok = wait_phase(bar(C::kBarDQFree), (gbase - 1) & 1, p.ctl, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
+                    if (ok) ok = wait_do(gbase);
+                    if (!ok) break;
+                    tc_fence_after();
                     issue_dp(gbase);
                     for (int it = 0; ok && it < t.nq; ++it) {
                         const int gi = gbase + it, st = gi % C::kStages;
                         const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
-                        const uint32_t dos = sbase + C::kOffDO + st * C::kTile;
+                        const uint32_t dos = sbase + C::kOffDO + (gi % C::kDoStages) * C::kTile;
                         const bool more = it + 1 < t.nq;
                         // dV += P^T dO_i   (K = 128 queries: 8 steps)
                         ok = wait_phase(bar(C::kBarPFull), gi & 1, p.ctl, abort_flag);
@@ -326,6 +347,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ts(tmem + C::kColDV, tmem + C::kColS + acol(kk),
                                    sw128_desc(dos + kk * 2048, 16384, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(bar(C::kBarDOEmpty + gi % C::kDoStages));  // dV_i was the last reader of dO_i
                         // S^T_{i+1} may overwrite P^T_i now: dV_i, issued first, completes first
                         // (the math warps keep their P in registers for dS).
                         if (more) {
@@ -351,14 +373,15 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ss(tmem + C::kColDK, sw128_desc(ds + kstep(kk), 16, 1024),
                                    sw128_desc(qs + kk * 2048, 16384, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
-                        tc_commit(bar(C::kBarDSFree));
-                        tc_commit(bar(C::kBarQEmpty + st));  // dK_i was the last reader of Q_i, dV_i of dO_i
+                        tc_commit(bar(C::kBarQEmpty + st));  // dK_i was the last reader of Q_i
                         if (more) {
-                            if (C::kDqOverDp) {  // dP^T_{i+1} overwrites the dQ_i accumulator
+                            if (C::kDqOverDp)  // dP^T_{i+1} overwrites the dQ_i accumulator
                                 ok = wait_phase(bar(C::kBarDQFree), gi & 1, p.ctl, abort_flag);
-                                if (!ok) break;
-                                tc_fence_after();
-                            }
+                            if (ok) ok = wait_do(gi + 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            // (dS_{i+1} is written after this product completes, hence after
+                            // dQ_i and dK_i, issued earlier, have read dS_i)
                             issue_dp(gi + 1);
                         }
                     }
@@ -376,11 +399,24 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     } else if (warp >= 8) {
         setmaxnreg_dec<C::kRegsDrain>();
         // ---------------------------------------------------------------- dQ drain
-        // warp w: query rows 32 (w % 4) .. + 31 of each dQ_i tile; its 8 KB of the dS
-        // area hold two {32 x 32} fp32 boxes.
+        // warp w: query rows 32 (w % 4) .. + 31 of each dQ_i tile, staged 32 columns at a
+        // time in two {32 x 32} fp32 boxes of its own; each box is a bulk group of its
+        // own, so a box is rewritten as soon as the reduce-add issued two boxes earlier
+        // has read it.
         const int q4 = warp & 3;
         const uint32_t tdq = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::kColDQ;
-        const uint32_t box0 = sbase + C::kOffDS + q4 * 8192, box1 = box0 + 4096;
+        const uint32_t box[2] = {sbase + C::kOffStage + q4 * 8192, sbase + C::kOffStage + q4 * 8192 + 4096};
+        auto put = [&](int b, const uint32_t (&r)[32], int col, int row, int slab) {
+            if (lane == 0) bulk_wait_read1();  // the group issued before the last one read box b
+            __syncwarp();
+            stage_rows32_f32(box[b], r, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_reduce_add_3d(&tm_dqacc, box[b], col, row, slab);
+                bulk_commit();
+            }
+        };
         bool ok = true;
         int gbase = 0;
         for (int k = 0; ok; ++k) {
@@ -403,39 +439,17 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     tc_fence_before();
                     mbar_arrive(bar(C::kBarDQFree));
                 }
-                // the dS area is the staging area once dQ_i and dK_i have read dS
-                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDSFree), gi & 1, p.ctl, abort_flag));
-                if (!ok) break;
-                stage_rows32_f32(box0, r0, lane);
-                stage_rows32_f32(box1, r1, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_reduce_add_3d(&tm_dqacc, box0, 0, row, slab);
-                    tma_reduce_add_3d(&tm_dqacc, box1, 32, row, slab);
-                    bulk_commit();
-                }
+                put(0, r0, 0, row, slab);
+                put(1, r1, 32, row, slab);
                 if constexpr (C::kDqOverDp) {
                     tmem_ld32(tdq + 64, r0);
                     tmem_ld32(tdq + 96, r1);
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(bar(C::kBarDQFree));
-                    if (lane == 0) bulk_wait_read0();  // the first two boxes have been read
-                    __syncwarp();
-                    stage_rows32_f32(box0, r0, lane);
-                    stage_rows32_f32(box1, r1, lane);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_reduce_add_3d(&tm_dqacc, box0, 64, row, slab);
-                        tma_reduce_add_3d(&tm_dqacc, box1, 96, row, slab);
-                        bulk_commit();
-                    }
+                    put(0, r0, 64, row, slab);
+                    put(1, r1, 96, row, slab);
                 }
-                if (lane == 0) bulk_wait_read0();
-                __syncwarp();
-                mbar_arrive(bar(C::kBarStageFree));  // the math warps may write the next dS
             }
             if (!ok) break;
             gbase += t.nq;
@@ -539,11 +553,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                                                               pf[c + 3] * (__uint_as_float(dr[c4 * 4 + 3]) - dd.w));
                     }
                 }
-                // the drain warps must have finished with the previous dQ tile's staging
-                if (gi > 0) {
-                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarStageFree), (gi - 1) & 1, p.ctl, abort_flag));
-                    if (!ok) break;
-                }
+                // (dQ_{i-1} and dK_{i-1}, which read the previous dS, are complete: they were
+                // issued before dP^T_i, whose completion was just waited for)
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     st_shared_v4(dsrow + (((c ^ (kr & 7)) & 7) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
@@ -597,6 +608,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
             if (gi != p.ctl.inject_skip_load)
                 drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
+        for (int gi = max(0, n_do - C::kDoStages); gi < n_do; ++gi)
+            drain_phase(bar(C::kBarDOFull + gi % C::kDoStages), (gi / C::kDoStages) & 1, p.ctl, abort_flag);
     }
     if (warp == 13) {
         tc_fence_after();

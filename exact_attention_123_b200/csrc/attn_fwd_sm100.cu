@@ -225,22 +225,55 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * (128 / C::kEsz),
                                     row0 + u.m0 + 128 * t, slab);
                 ++n_qload;
-                for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
+                if constexpr (!SP) {
+                    for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
 #pragma unroll
-                    for (int kv = 0; kv < 2; ++kv, ++idx) {
-                        const int s = idx % C::kStages;
-                        if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
-                            ok = false;
-                            break;
+                        for (int kv = 0; kv < 2; ++kv, ++idx) {
+                            const int s = idx % C::kStages;
+                            if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
+                            mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
+#pragma unroll
+                            for (int x = 0; x < C::kBoxes; ++x)
+                                tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s),
+                                            x * (128 / C::kEsz), row0 + 128 * j, slab);
+                            n_issued = idx + 1;
                         }
-                        if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
+                    }
+                    continue;
+                }
+                // one ring load (K or V tile j) at position idx; false once the wait gave up
+                auto load = [&](bool is_v, int j) -> bool {
+                    const int s = idx % C::kStages;
+                    if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag))
+                        return false;
+                    if (idx != p.ctl.inject_skip_load) {  // (test hook: this slot never fills)
                         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x)
-                            tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s),
+                            tma_load_3d(slot(s) + x * 16384, is_v ? &tm_v : &tm_k, bar(C::kBarFull + s),
                                         x * (128 / C::kEsz), row0 + 128 * j, slab);
                         n_issued = idx + 1;
                     }
+                    ++idx;
+                    return true;
+                };
+                // With a tile mask each query tile sweeps its own key tiles: step s pairs the
+                // s-th key tile of Q0 with the s-th of Q1 and loads K then V of both (once
+                // when they coincide), so a step never idles one of the tiles.
+                int j0 = u.ts0.next(0), j1 = u.ts1.next(0);
+                while (ok && (j0 < u.ts0.hi || j1 < u.ts1.hi)) {
+                    const bool a0 = j0 < u.ts0.hi;
+                    const bool a1 = j1 < u.ts1.hi && !(a0 && j1 == j0);
+                    for (int kv = 0; kv < 2 && ok; ++kv) {
+                        if (a0) ok = load(kv != 0, j0);
+                        if (ok && a1) ok = load(kv != 0, j1);
+                    }
+                    if (j0 < u.ts0.hi) j0 = u.ts0.next(j0 + 1);
+                    if (j1 < u.ts1.hi) j1 = u.ts1.next(j1 + 1);
                 }
             }
         }
@@ -296,8 +329,88 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             int base = 0;          // ring position of the unit's K_0
             int n_u = 0;           // units started
             int gs[2] = {0, 0};    // S_t products issued (all units): phase counters
+            auto wait_full = [&](int pos) {
+                return wait_phase(bar(C::kBarFull + pos % C::kStages), (pos / C::kStages) & 1, p.ctl, abort_flag);
+            };
             FOR_EACH_UNIT(u) {
                 if (!ok) break;
+                if constexpr (SP) {
+                    // Independent sweeps (see the producer): the ring positions of step s's
+                    // K and V tiles for Q0 and Q1; a tile is active while its key tiles last.
+                    struct StepPos {
+                        bool a0, a1, dup;
+                        int k0, k1, v0, v1, next;
+                    };
+                    auto step_pos = [&](int j0, int j1, int pos) {
+                        StepPos r;
+                        r.a0 = j0 < u.ts0.hi;
+                        r.a1 = j1 < u.ts1.hi;
+                        r.dup = r.a0 && r.a1 && j0 == j1;
+                        const int nk = static_cast<int>(r.a0) + static_cast<int>(r.a1) - static_cast<int>(r.dup);
+                        r.k0 = pos;
+                        r.k1 = r.dup ? pos : pos + static_cast<int>(r.a0);
+                        r.v0 = pos + nk;
+                        r.v1 = r.dup ? r.v0 : r.v0 + static_cast<int>(r.a0);
+                        r.next = pos + 2 * nk;
+                        return r;
+                    };
+                    int j0 = u.ts0.next(0), j1 = u.ts1.next(0);
+                    StepPos cs = step_pos(j0, j1, base);
+                    if (!cs.a0 && !cs.a1) continue;  // no tile pair to compute
+                    ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
+                    if (ok && cs.a0) ok = wait_full(cs.k0);
+                    if (ok && cs.a1 && !cs.dup) ok = wait_full(cs.k1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (cs.a0) issue_S(0, cs.k0);
+                    if (cs.a1) issue_S(1, cs.k1);
+                    if (cs.a0) tc_commit(bar(C::kBarEmpty + cs.k0 % C::kStages));
+                    if (cs.a1 && !cs.dup) tc_commit(bar(C::kBarEmpty + cs.k1 % C::kStages));
+                    if (cs.a0) j0 = u.ts0.next(j0 + 1);
+                    if (cs.a1) j1 = u.ts1.next(j1 + 1);
+                    StepPos ns = step_pos(j0, j1, cs.next);
+                    if (!ns.a0 && !ns.a1) tc_commit(bar(C::kBarQEmpty));
+                    bool started[2] = {false, false};
+                    while (ok) {
+                        if (cs.a0) ok = wait_full(cs.v0);
+                        if (ok && cs.a1 && !cs.dup) ok = wait_full(cs.v1);
+                        if (!ok) break;
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (t ? cs.a1 : cs.a0) {
+                                ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
+                                if (!ok) break;
+                                ++gs[t];
+                                tc_fence_after();
+                                issue_PV(t, t ? cs.v1 : cs.v0, started[t]);
+                                started[t] = true;
+                                if (!(t ? ns.a1 : ns.a0)) tc_commit(bar(C::kBarO + t));  // the tile's last P V
+                            }
+                            if (t ? ns.a1 : ns.a0) {
+                                if (!(t == 1 && ns.dup)) {  // (a shared K tile was waited for by Q0)
+                                    ok = wait_full(t ? ns.k1 : ns.k0);
+                                    if (!ok) break;
+                                    tc_fence_after();
+                                }
+                                issue_S(t, t ? ns.k1 : ns.k0);
+                            }
+                        }
+                        if (!ok) break;
+                        if (cs.a0) tc_commit(bar(C::kBarEmpty + cs.v0 % C::kStages));
+                        if (cs.a1 && !cs.dup) tc_commit(bar(C::kBarEmpty + cs.v1 % C::kStages));
+                        if (ns.a0) tc_commit(bar(C::kBarEmpty + ns.k0 % C::kStages));
+                        if (ns.a1 && !ns.dup) tc_commit(bar(C::kBarEmpty + ns.k1 % C::kStages));
+                        if (!ns.a0 && !ns.a1) break;
+                        cs = ns;
+                        if (cs.a0) j0 = u.ts0.next(j0 + 1);
+                        if (cs.a1) j1 = u.ts1.next(j1 + 1);
+                        ns = step_pos(j0, j1, cs.next);
+                        if (!ns.a0 && !ns.a1) tc_commit(bar(C::kBarQEmpty));  // the S products just issued were the unit's last
+                    }
+                    if (!ok) break;
+                    base = cs.next;
+                    ++n_u;
+                    continue;
+                }
                 const int hi = u.nkv_max();
                 int j = u.unext(0);  // the unit's key tiles are j, unext(j + 1), ... (< hi)
                 if (j >= hi) continue;  // no tile pair to compute (tile mask)
