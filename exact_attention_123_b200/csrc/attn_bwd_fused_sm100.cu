@@ -19,10 +19,11 @@
 //     dQ_i = dS K_j               SS: A = dS read query-major (the transposed view
 //                                 of the same shared-memory tile), B = K_j
 //     dK  += dS^T Q_i             SS: A = dS as stored
-//   and four "drain" warps move each dQ_i tile out of TMEM, through shared memory,
-//   into an fp32 accumulator with TMA reduce-adds (the add happens in L2).  A small
-//   kernel first zeroes the accumulator (with the per-row D and lse2 terms) and
-//   another one afterwards writes dQ = bf16(scale * accumulator).
+//   and four "drain" warps move each dQ_i tile out of TMEM, through a shared-memory
+//   staging area of their own, into an fp32 accumulator with TMA reduce-adds (the
+//   add happens in L2).  A small kernel first zeroes the accumulator (with the
+//   per-row D and lse2 terms) and another one afterwards writes
+//   dQ = bf16(scale * accumulator).
 // The fp32 additions from different key tiles land in an order that depends on
 // scheduling, so dQ may differ between runs in its last bits; the deterministic
 // backward (attn_bwd_sm100.cu) avoids that at the price of the two extra products.
@@ -46,7 +47,9 @@
 // (32 KB: two 4 KB boxes per warp, reused as soon as the TMA has read them).
 // The next dS is written only after dP^T_{i+1} is complete, which (tensor-core
 // operations completing in issue order) implies dQ_i and dK_i, the products that
-// read dS, are done.
+// read dS, are done.  At a unit's end V_j is reloaded once its last dP^T is done and
+// K_j once its last dQ is, and the following unit's K/V tiles are prefetched into L2
+// meanwhile.
 //
 // Every wait is bounded (see attn_common.cuh); an expired wait stops every role,
 // drains the copies in flight and returns with ATTN_ERR_TIMEOUT in the status word.
@@ -88,9 +91,11 @@ struct FusedCfg {
     static constexpr int kOffStage = kOffDS + 32768;           // + warp * 8192: two {32 x 32} fp32 boxes
     static constexpr int kOffVec = kOffStage + 32768;          // + st * 1024: lse2[128], D[128]
     static constexpr int kOffBar = kOffVec + kStages * 1024;
-    static constexpr int kBarKVFull = 0;
-    static constexpr int kBarKVEmpty = 1;                      // K_j, V_j no longer read (unit done)
-    static constexpr int kBarQFull = 2;                        // + st
+    static constexpr int kBarKFull = 0;
+    static constexpr int kBarKEmpty = 1;                       // K_j no longer read (the unit's last dQ done)
+    static constexpr int kBarVFull = 2;
+    static constexpr int kBarVEmpty = 3;                       // V_j no longer read (the unit's last dP^T done)
+    static constexpr int kBarQFull = 4;                        // + st
     static constexpr int kBarQEmpty = kBarQFull + kStages;     // + st
     static constexpr int kBarDOFull = kBarQEmpty + kStages;    // + buffer
     static constexpr int kBarDOEmpty = kBarDOFull + kDoStages; // + buffer
@@ -222,37 +227,61 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 if (!tile_at(r, t) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
                 const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
-                // K_j, V_j once every product of the previous unit has been issued and done
-                ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarKVEmpty), (n_kv & 1) ^ 1, p.ctl, abort_flag));
-                if (!ok) break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(C::kBarKVFull), 2 * C::kTile);
+                // V_j once the previous unit's last dP^T is done, K_j once its last dQ is
 #pragma unroll
-                    for (int x = 0; x < C::kBoxes; ++x) {
-                        tma_load_3d(sbase + C::kOffK + x * 16384, &tm_k, bar(C::kBarKVFull), x * 64, row0 + t.kv0,
-                                    slab);
-                        tma_load_3d(sbase + C::kOffV + x * 16384, &tm_v, bar(C::kBarKVFull), x * 64, row0 + t.kv0,
-                                    slab);
+                for (int kv = 1; kv >= 0; --kv) {
+                    const int full = kv ? C::kBarVFull : C::kBarKFull, empty = kv ? C::kBarVEmpty : C::kBarKEmpty;
+                    ok = __all_sync(0xffffffffu, wait_phase(bar(empty), (n_kv & 1) ^ 1, p.ctl, abort_flag));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(full), C::kTile);
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            tma_load_3d(sbase + (kv ? C::kOffV : C::kOffK) + x * 16384, kv ? &tm_v : &tm_k, bar(full),
+                                        x * 64, row0 + t.kv0, slab);
                     }
                 }
+                if (!ok) break;
                 ++n_kv;
+                // the next unit's K and V tiles into L2 while this unit runs
+                if (lane == 0) {
+                    for (int k2 = k + 1;; ++k2) {
+                        const int r2 = rank_of(k2);
+                        if (r2 >= T) break;
+                        Tile t2;
+                        if (!tile_at(r2, t2) || t2.nq == 0) continue;
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x) {
+                            tma_prefetch_l2_3d(&tm_k, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
+                            tma_prefetch_l2_3d(&tm_v, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
+                        }
+                        break;
+                    }
+                }
                 for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
                     const int gi = n_q, st = gi % C::kStages;
-                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
-                                                            p.ctl, abort_flag));
-                    if (!ok) break;
                     const int q0 = i * 128;
-                    float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
+                    // the step's row terms, read before waiting for the stage so that their
+                    // global-memory latency overlaps the wait
+                    float l2[4], dd[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int q = q0 + u * 32 + lane;
-                        float l2 = INFINITY, dd = 0.f;  // rows past the sequence: P = 0
+                        l2[u] = INFINITY;  // rows past the sequence: P = 0
+                        dd[u] = 0.f;
                         if (q < t.len) {
-                            l2 = p.lse2[lrow0 + q * lrs];
-                            dd = p.dvec[lrow0 + q * lrs];
+                            l2[u] = p.lse2[lrow0 + q * lrs];
+                            dd[u] = p.dvec[lrow0 + q * lrs];
                         }
-                        vec[u * 32 + lane] = l2;
-                        vec[128 + u * 32 + lane] = dd;
+                    }
+                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
+                                                            p.ctl, abort_flag));
+                    if (!ok) break;
+                    float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        vec[u * 32 + lane] = l2[u];
+                        vec[128 + u * 32 + lane] = dd[u];
                     }
                     __syncwarp();
                     if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
@@ -319,7 +348,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     if (r >= T) break;
                     Tile t;
                     if (!tile_at(r, t) || t.nq == 0) continue;
-                    ok = wait_phase(bar(C::kBarKVFull), n_t & 1, p.ctl, abort_flag);
+                    ok = wait_phase(bar(C::kBarKFull), n_t & 1, p.ctl, abort_flag);
                     if (ok) ok = wait_q(gbase);
                     if (!ok) break;
                     tc_fence_after();
@@ -328,10 +357,12 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     issue_s(gbase);
                     if (C::kDqOverDp && gbase > 0)  // dP^T's columns held the previous dQ tile
                         ok = wait_phase(bar(C::kBarDQFree), (gbase - 1) & 1, p.ctl, abort_flag);
+                    if (ok) ok = wait_phase(bar(C::kBarVFull), n_t & 1, p.ctl, abort_flag);
                     if (ok) ok = wait_do(gbase);
                     if (!ok) break;
                     tc_fence_after();
                     issue_dp(gbase);
+                    if (t.nq == 1) tc_commit(bar(C::kBarVEmpty));  // the unit's last dP^T
                     for (int it = 0; ok && it < t.nq; ++it) {
                         const int gi = gbase + it, st = gi % C::kStages;
                         const uint32_t qs = sbase + C::kOffQ + st * C::kTile;
@@ -368,6 +399,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                             mma_ss(tmem + C::kColDQ, sw128_desc(ds + kk * 2048, 16384, 1024),
                                    sw128_desc(sbase + C::kOffK + kk * 2048, 16384, 1024), idDQ, kk > 0 ? 1u : 0u);
                         tc_commit(bar(C::kBarDQFull));
+                        if (!more) tc_commit(bar(C::kBarKEmpty));  // the unit's last reader of K_j
                         // dK += dS^T Q_i  (K = 128 queries; A = dS as stored, keys x queries)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
@@ -383,10 +415,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                             // (dS_{i+1} is written after this product completes, hence after
                             // dQ_i and dK_i, issued earlier, have read dS_i)
                             issue_dp(gi + 1);
+                            if (it + 2 == t.nq) tc_commit(bar(C::kBarVEmpty));  // the unit's last dP^T
                         }
                     }
                     if (!ok) break;
-                    tc_commit(bar(C::kBarKVEmpty));
                     tc_commit(bar(C::kBarKdv));
                     gbase += t.nq;
                     ++n_t;
@@ -604,7 +636,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     __syncthreads();
     if (warp == 12 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        if (n_kv > 0) drain_phase(bar(C::kBarKVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        if (n_kv > 0) {
+            drain_phase(bar(C::kBarKFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+            drain_phase(bar(C::kBarVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        }
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
             if (gi != p.ctl.inject_skip_load)
                 drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);

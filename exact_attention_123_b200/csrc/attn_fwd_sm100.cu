@@ -225,8 +225,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * (128 / C::kEsz),
                                     row0 + u.m0 + 128 * t, slab);
                 ++n_qload;
+                // the key-padding flags of the unit (if any) are brought into L1 with the
+                // K/V tiles, so that the softmax warps' reads of them hit L1
+                const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(u.b, u.start) : nullptr;
                 if constexpr (!SP) {
                     for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
+                        if (keep != nullptr) {
+                            prefetch_l1(keep + 128 * j);
+                            prefetch_l1(keep + 128 * j + 127);
+                        }
 #pragma unroll
                         for (int kv = 0; kv < 2; ++kv, ++idx) {
                             const int s = idx % C::kStages;
@@ -495,10 +502,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         bool first_step = true;
         for (int j = ts.next(0); j < ts.hi; j = ts.next(j + 1), ++gs) {
             const int kbase = j * 128;
-            // the key-padding flags of this key tile (128 bytes, at most two cache lines)
-            // are brought into L1 before waiting for S, so that reading them below does
-            // not add a trip to L2 to the softmax chain
-            if (keep != nullptr && lane < 2) prefetch_l1(keep + kbase + lane * 127);
             ok = wait_phase(bar(C::kBarS + t), gs & 1, p.ctl, abort_flag);
             if (!ok) break;
             tc_fence_after();
