@@ -602,7 +602,9 @@ def run_ours(args):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "traffic": recorded_traffic(dominant),
-                     "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src}, burst)"},
+                     "peak_source": ("MEASURED_PEAKS.json bf16_tflops (burst)" if peak_src == "measured" else
+                                     "fallback: 1590 TFLOPS measured earlier on this pool "
+                                     "(no MEASURED_PEAKS.json beside bench.py)")},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_n, "pipeline": "copy in, kernels, copy out on three streams over two buffer sets"},
