@@ -132,7 +132,8 @@ struct FwdUnit {
     }
 };
 
-template <bool SP>
+// Sets: also build the tile sets (the epilogue needs only the unit's position).
+template <bool SP, bool Sets = true>
 __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int G, FwdUnit &u) {
     const int BH = p.g.B * p.g.H;
     const int r = k * G + ((k & 1) ? (G - 1 - cta) : cta);
@@ -147,8 +148,10 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int
     const int r1 = u.m0 + 128;
     u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
     u.nkv1 = (r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
-    u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
-    u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
+    if constexpr (Sets) {
+        u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
+        u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
+    }
     return true;
 }
 
@@ -379,18 +382,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     if (!ns.a0 && !ns.a1) tc_commit(bar(C::kBarQEmpty));
                     bool started[2] = {false, false};
                     while (ok) {
-                        if (cs.a0) ok = wait_full(cs.v0);
-                        if (ok && cs.a1 && !cs.dup) ok = wait_full(cs.v1);
-                        if (!ok) break;
                         for (int t = 0; t < 2 && ok; ++t) {
                             if (t ? cs.a1 : cs.a0) {
-                                ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
+                                // this tile's V (a shared one was waited for by Q0)
+                                if (!(t == 1 && cs.dup)) ok = wait_full(t ? cs.v1 : cs.v0);
+                                if (ok) ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
                                 if (!ok) break;
                                 ++gs[t];
                                 tc_fence_after();
                                 issue_PV(t, t ? cs.v1 : cs.v0, started[t]);
                                 started[t] = true;
                                 if (!(t ? ns.a1 : ns.a0)) tc_commit(bar(C::kBarO + t));  // the tile's last P V
+                                // The tile's V slot is free once its P V is done (a V tile the two
+                                // share, once Q1's is): with up to four ring loads per step the next
+                                // step's V loads must not wait for the S products issued after it.
+                                if (t == 1 || !cs.dup) tc_commit(bar(C::kBarEmpty + (t ? cs.v1 : cs.v0) % C::kStages));
                             }
                             if (t ? ns.a1 : ns.a0) {
                                 if (!(t == 1 && ns.dup)) {  // (a shared K tile was waited for by Q0)
@@ -402,8 +408,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             }
                         }
                         if (!ok) break;
-                        if (cs.a0) tc_commit(bar(C::kBarEmpty + cs.v0 % C::kStages));
-                        if (cs.a1 && !cs.dup) tc_commit(bar(C::kBarEmpty + cs.v1 % C::kStages));
                         if (ns.a0) tc_commit(bar(C::kBarEmpty + ns.k0 % C::kStages));
                         if (ns.a1 && !ns.dup) tc_commit(bar(C::kBarEmpty + ns.k1 % C::kStages));
                         if (!ns.a0 && !ns.a1) break;
@@ -632,7 +636,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // The tile mask leaves this tile no key tile: O = 0 and lse = -inf, like any
             // row that sees no key; nothing was computed for it.
             FwdUnit e;
-            fwd_unit<SP>(p, k_, cta, G, e);
+            fwd_unit<SP, false>(p, k_, cta, G, e);
             if (row < len) {
                 const long long r = static_cast<long long>(row);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + p.g.base(e.b, e.h, e.start, D) + r * p.g.row_stride(D));
@@ -650,7 +654,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float inv = (l > 0.f) ? p.o_scale / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
-            fwd_unit<SP>(p, k_, cta, G, e);
+            fwd_unit<SP, false>(p, k_, cta, G, e);
             __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
             // A warp's full 32-row block goes out by TMA store from its stage (laid out
             // as the 64-byte swizzle of a 32 x 32 box), so the warp moves on to the next
