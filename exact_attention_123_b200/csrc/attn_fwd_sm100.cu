@@ -42,6 +42,13 @@
 // A row that sees no key keeps m = -inf and l = 0 and writes O = 0, lse = -inf
 // (the _safe_softmax rule of "Profiling in PyTorch (part 3)", math backend).
 //
+// With a tile mask (block-sparse) the kernel runs with one query tile per CTA and two
+// CTAs per SM (NT = 1; 256 threads: softmax warps 0-3, producer warp 4, issuer warp 5,
+// 256 TMEM columns: S0 = [0,128), O0 = [128, 128+d)): each CTA sweeps only the key
+// tiles its own tile attends, with a K/V ring of its own, so a tile never waits for
+// the other tile of a pair (whose key tiles differ) and one CTA's unit change
+// overlaps the other CTA's work.
+//
 // With e4m3 operands (F8, the FP8 direction of the codechina article's §9) both
 // products are kind::f8f6f4 with fp32 accumulation; P is rounded to e4m3 and
 // written to a swizzled shared-memory tile (the A operand of P V) instead of TMEM,
@@ -49,6 +56,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 
 #include "attn_common.cuh"
@@ -58,7 +66,12 @@ namespace attn {
 
 // F8: Q, K and V in e4m3 (V, keys x d, is the MN-major B operand of P V as in the
 // bf16 path), P rounded to e4m3 in shared memory, fp32 accumulation.
-template <int D, bool F8 = false>
+// NT: 128-row query tiles per CTA.  NT = 2: one CTA per SM, its two tiles share every
+// K/V tile and take turns on the tensor core.  NT = 1 (tile masks, where the query
+// tiles of a pair attend different key tiles): two CTAs per SM, each sweeping the key
+// tiles of its own query tile with a ring of its own, so neither waits for the other
+// at the end of a unit and neither loads a K/V tile for the other.
+template <int D, bool F8 = false, int NT = 2>
 struct FwdCfg {
     static constexpr int kEsz = F8 ? 1 : 2;                // bytes per Q/K/V element
     static constexpr int kTileBytes = 128 * D * kEsz;      // one 128-row tile
@@ -66,22 +79,31 @@ struct FwdCfg {
     // d bytes per row (128-byte swizzle at d = 128, 64-byte swizzle at d = 64)
     static constexpr int kBoxes = F8 ? 1 : D / 64;
     static constexpr int kKSteps = D * kEsz / 32;          // 32-byte K steps of S = Q K^T
-    static constexpr int kStages = F8 ? (D == 128 ? 8 : 16) : (D == 128) ? 4 : 8;
-    // 3 warpgroups: two softmax groups, and one with the TMA producer, the MMA issuer
-    // and two idle warps (registers move by whole warpgroups).  Launched at 168
-    // registers per thread (the most 384 threads allow), the control group gives
-    // registers back and the softmax groups take them: 2*128*200 + 128*104 = 384*168.
-    static constexpr int kThreads = 384;
-    static constexpr int kLaunchRegs = 168, kRegsSoftmax = 200, kRegsControl = 104;
-    static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
+    static_assert(NT == 2 || (NT == 1 && !F8), "one tile per CTA: bf16 only");
+    // K/V ring: at NT = 1 what half an SM's shared memory leaves after Q and the stage
+    static constexpr int kStages = NT == 1 ? (D == 128 ? 2 : 5) : F8 ? (D == 128 ? 8 : 16) : (D == 128) ? 4 : 8;
+    // NT + 1 warpgroups: NT softmax groups, and one with the TMA producer, the MMA
+    // issuer and two idle warps (registers move by whole warpgroups).  Launched at the
+    // most registers per thread the CTAs of one SM allow (NT = 2: 384 threads, 168;
+    // NT = 1: two CTAs of 256, 128), the control group gives registers back and the
+    // softmax groups take them: 2*128*200 + 128*104 = 384*168; at NT = 1
+    // 128*184 + 128*72 (d = 128) or 128*200 + 128*56 (d = 64) = 256*128, the faster
+    // split of each (same-box timings).
+    static constexpr int kThreads = 128 * (NT + 1);
+    static constexpr int kCtasPerSm = NT == 1 ? 2 : 1;
+    static constexpr int kLaunchRegs = NT == 1 ? 128 : 168;
+    static constexpr int kRegsSoftmax = (NT == 1 && D == 128) ? 184 : 200;
+    static constexpr int kRegsControl = NT == 1 ? 256 - kRegsSoftmax : 104;
+    static_assert(NT * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
                   "register reallocation exceeds the launch pool");
-    static constexpr int kTmemCols = 512;
+    static constexpr int kProducerWarp = 4 * NT, kIssuerWarp = 4 * NT + 1;
+    static constexpr int kTmemCols = NT == 1 ? 256 : 512;
     // column pairs c (of each 32-pair half row) whose exponentials come from the FMA
     // pipe: bit (c % 8) set.  Measured best: one pair in eight with e4m3 operands and
     // with bf16 at d = 64 (where the exponentials outweigh the products), none at
     // bf16 d = 128.
     static constexpr uint32_t kPolyPairs = (F8 || D == 64) ? 0x80u : 0u;
-    static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+    static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 128 * NT, kColO1 = 128 * NT + D;
     // barrier indices
     static constexpr int kBarQ = 0;
     static constexpr int kBarFull = 1;                       // + slot
@@ -91,14 +113,18 @@ struct FwdCfg {
     static constexpr int kBarO = 5 + 2 * kStages;            // + tile
     static constexpr int kBarDone = 7 + 2 * kStages;
     static constexpr int kBarQEmpty = 8 + 2 * kStages;       // the unit's last S products are done
-    static constexpr int kNumBars = 9 + 2 * kStages;
-    static constexpr int kSmemTiles = (2 + kStages) * kTileBytes;
+    static constexpr int kBarUFull = 9 + 2 * kStages;        // + entry: a claimed unit rank is published
+    static constexpr int kBarUEmpty = 13 + 2 * kStages;      // + entry: every role has read it
+    static constexpr int kNumBars = 17 + 2 * kStages;
+    static constexpr int kSmemTiles = (NT + kStages) * kTileBytes;
     static constexpr int kOffP = kSmemTiles;                   // e4m3 P_0, P_1: 128 x 128 bytes each
-    static constexpr int kOffStage = kOffP + (F8 ? 2 * 16384 : 0);  // 8 softmax warps x 2 KB output stage
-    static constexpr int kOffBar = kOffStage + 8 * 2048;
-    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 16;
+    static constexpr int kOffStage = kOffP + (F8 ? 2 * 16384 : 0);  // 2 KB output stage per softmax warp
+    static constexpr int kOffBar = kOffStage + 4 * NT * 2048;
+    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed unit ranks
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 32;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
-    static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared-memory limit");
+    // 227 KB per CTA; two CTAs share an SM's 228 KB less 1 KB reserved per CTA
+    static_assert(kSmemBytes <= (NT == 1 ? 115712 : 232448), "exceeds the per-CTA shared-memory limit");
 };
 
 struct FwdParams {
@@ -109,15 +135,18 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e) (e4m3: times the Q and K dequantisation scales)
     float o_scale;     // 1, or the V dequantisation scale (e4m3)
     int causal;
-    int n_pairs;       // 256-row query blocks per slice
+    int n_units;       // (128 NT)-row query blocks per slice
+    unsigned int *sched;  // dynamic deal: {units claimed, CTAs finished} of this launch (else null)
 };
 
-// Unit r of the persistent schedule: k = r / (B*H) counts down the 256-row blocks
-// from the last one, so ranks are ordered heaviest first for causal masking.
-// CTA c of G takes ranks c, 2G-1-c, 2G+c, 4G-1-c, ... (snake order).
+// Unit r of the persistent schedule: k = r / (B*H) counts down the (128 NT)-row
+// blocks from the last one, so ranks are ordered heaviest first for causal masking.
+// CTA c of G takes ranks c, 2G-1-c, 2G+c, 4G-1-c, ... (snake order), or, with a
+// tile mask (whose rows make the units' costs uneven), the next unclaimed rank each
+// time it starts a unit (a global counter: the CTAs that draw light units draw more).
 struct FwdUnit {
     int b, h, start, len, m0;
-    int nkv0, nkv1;  // key tiles in reach of Q0 and Q1 (0: the tile lies past the sequence)
+    int nkv0, nkv1;  // key tiles in reach of Q0 and Q1 (0: the tile lies past the sequence or NT = 1)
     TileSet ts0, ts1;  // the key tiles Q0 / Q1 actually attend (all of them without a tile mask)
     __device__ __forceinline__ int nkv(int t) const { return t ? nkv1 : nkv0; }
     __device__ __forceinline__ int nkv_max() const { return max(nkv0, nkv1); }
@@ -132,22 +161,22 @@ struct FwdUnit {
     }
 };
 
-// Sets: also build the tile sets (the epilogue needs only the unit's position).
-template <bool SP, bool Sets = true>
-__device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int G, FwdUnit &u) {
+// The unit of rank r.  Sets: also build the tile sets (the epilogue needs only the
+// unit's position).
+template <bool SP, int NT, bool Sets = true>
+__device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u) {
     const int BH = p.g.B * p.g.H;
-    const int r = k * G + ((k & 1) ? (G - 1 - cta) : cta);
     const int kk = r / BH;
     const int bh = r - kk * BH;
     u.b = bh / p.g.H;
     u.h = bh - u.b * p.g.H;
     p.g.slice(u.b, u.start, u.len);
-    u.m0 = (p.n_pairs - 1 - kk) * 256;
+    u.m0 = (p.n_units - 1 - kk) * 128 * NT;
     if (u.m0 >= u.len) return false;
     const int nkv_all = (u.len + 127) / 128;
     const int r1 = u.m0 + 128;
     u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
-    u.nkv1 = (r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
+    u.nkv1 = (NT == 1 || r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
     if constexpr (Sets) {
         u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
         u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
@@ -158,33 +187,64 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int k, int cta, int
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-// SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs.
-template <int D, bool SP, bool F8>
-__global__ void __launch_bounds__(384, 1)
+// SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs.  NT: query
+// tiles per CTA (see FwdCfg).
+template <int D, bool SP, bool F8, int NT>
+__global__ void __launch_bounds__(FwdCfg<D, F8, NT>::kThreads, FwdCfg<D, F8, NT>::kCtasPerSm)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o_st,
                       const __grid_constant__ FwdParams p) {
-    using C = FwdCfg<D, F8>;
+    using C = FwdCfg<D, F8, NT>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
     uint8_t *sptr = smem_raw + (sbase - raw_u32);
     const uint32_t bars = sbase + C::kOffBar;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
-    auto slot = [&](int s) -> uint32_t { return sbase + static_cast<uint32_t>(2 + s) * C::kTileBytes; };
+    auto slot = [&](int s) -> uint32_t { return sbase + static_cast<uint32_t>(NT + s) * C::kTileBytes; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
-    const int n_ranks = p.g.B * p.g.H * p.n_pairs;
-    // walks this CTA's units in order; every role uses the same walk
-#define FOR_EACH_UNIT(u)                                                        \
-    for (int k_ = 0; k_ * G < n_ranks; ++k_)                                     \
-        if (FwdUnit u; (k_ * G + ((k_ & 1) ? (G - 1 - cta) : cta)) < n_ranks && \
-                       fwd_unit<SP>(p, k_, cta, G, u))
+    const int n_ranks = p.g.B * p.g.H * p.n_units;
+    // Dynamic deal (tile masks): the producer claims each unit rank and publishes it
+    // to the other roles through a 4-entry ring; n_ranks ends the walk.
+    constexpr bool kDyn = SP && NT == 1;
+    volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_holder + 2);
+    auto claim_rank = [&](int k) -> int {  // producer
+        int r = n_ranks;
+        if (!*abort_flag) r = min(static_cast<int>(atomicAdd(p.sched, 1u)), n_ranks);
+        if (!wait_phase(bar(C::kBarUEmpty + (k & 3)), ((k >> 2) & 1) ^ 1, p.ctl, abort_flag)) return n_ranks;
+        unit_ring[k & 3] = r;
+        mbar_arrive(bar(C::kBarUFull + (k & 3)));
+        return r;
+    };
+    auto take_rank = [&](int k) -> int {  // issuer and softmax threads
+        if (!wait_phase(bar(C::kBarUFull + (k & 3)), (k >> 2) & 1, p.ctl, abort_flag)) return n_ranks;
+        const int r = unit_ring[k & 3];
+        mbar_arrive(bar(C::kBarUEmpty + (k & 3)));
+        return r;
+    };
+    auto static_rank = [&](int k) -> int { return k * G + ((k & 1) ? (G - 1 - cta) : cta); };
+    // walks this CTA's units in order (RANK(k): the role's way to get its k-th rank;
+    // the static deal's last round can hold ranks past the end); every role sees the
+    // same ranks
+#define FOR_EACH_UNIT(u, RANK)                                   \
+    for (int k_ = 0; kDyn || k_ * G < n_ranks; ++k_)             \
+        if (const int r_ = (RANK)(k_); kDyn && r_ >= n_ranks)    \
+            break;                                               \
+        else if (FwdUnit u; r_ < n_ranks && fwd_unit<SP, NT>(p, r_, u))
+    auto producer_rank = [&](int k) -> int {
+        if constexpr (kDyn) return claim_rank(k);
+        else return static_rank(k);
+    };
+    auto consumer_rank = [&](int k) -> int {
+        if constexpr (kDyn) return take_rank(k);
+        else return static_rank(k);
+    };
 
-    if (warp == 9) {
+    if (warp == C::kIssuerWarp) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
         tmem_relinquish();
     }
@@ -192,6 +252,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         for (int i = 0; i < C::kNumBars; ++i) {
             uint32_t cnt = 1;
             if (i == C::kBarP || i == C::kBarP + 1) cnt = 128;
+            if (i >= C::kBarUEmpty && i < C::kBarUEmpty + 4) cnt = 1 + 128 * NT;  // issuer + softmax threads
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
@@ -203,9 +264,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t tmem = *tmem_holder;
     int n_issued = 0;  // producer: ring loads 0 .. n_issued-1 were started (except a skipped one)
     int n_qload = 0;   // producer: Q pairs whose load was started
-    if (warp >= 8) {
+    if (warp >= 4 * NT) {
     setmaxnreg_dec<C::kRegsControl>();
-    if (warp == 8) {
+    if (warp == C::kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
@@ -213,16 +274,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tma_prefetch_desc(&tm_v);
             bool ok = true;
             int idx = 0;  // ring position, continuing across units
-            FOR_EACH_UNIT(u) {
+            FOR_EACH_UNIT(u, producer_rank) {
                 if (!ok) break;
                 const int nkv_max = u.nkv_max();
                 if (u.unext(0) >= nkv_max) continue;  // no tile pair to compute (tile mask)
                 const int row0 = p.g.tma_row0(u.start), slab = p.g.tma_slab(u.b, u.h);
-                // Q0/Q1 once the previous unit's last S products have read theirs
+                // the unit's Q tiles once the previous unit's last S products have read theirs
                 if (!wait_phase(bar(C::kBarQEmpty), (n_qload & 1) ^ 1, p.ctl, abort_flag)) break;
-                mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTileBytes);
+                mbar_arrive_expect_tx(bar(C::kBarQ), NT * C::kTileBytes);
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
+                for (int t = 0; t < NT; ++t)
 #pragma unroll
                     for (int x = 0; x < C::kBoxes; ++x)
                         tma_load_3d(sbase + t * C::kTileBytes + x * 16384, &tm_q, bar(C::kBarQ), x * (128 / C::kEsz),
@@ -231,63 +292,32 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // the key-padding flags of the unit (if any) are brought into L1 with the
                 // K/V tiles, so that the softmax warps' reads of them hit L1
                 const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(u.b, u.start) : nullptr;
-                if constexpr (!SP) {
-                    for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
-                        if (keep != nullptr) {
-                            prefetch_l1(keep + 128 * j);
-                            prefetch_l1(keep + 128 * j + 127);
-                        }
-#pragma unroll
-                        for (int kv = 0; kv < 2; ++kv, ++idx) {
-                            const int s = idx % C::kStages;
-                            if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
-                            mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
-#pragma unroll
-                            for (int x = 0; x < C::kBoxes; ++x)
-                                tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s),
-                                            x * (128 / C::kEsz), row0 + 128 * j, slab);
-                            n_issued = idx + 1;
-                        }
+                // the key tiles either query tile attends (with a tile mask, NT = 1: those of
+                // the CTA's one tile)
+                for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
+                    if (keep != nullptr) {
+                        prefetch_l1(keep + 128 * j);
+                        prefetch_l1(keep + 128 * j + 127);
                     }
-                    continue;
-                }
-                // one ring load (K or V tile j) at position idx; false once the wait gave up
-                auto load = [&](bool is_v, int j) -> bool {
-                    const int s = idx % C::kStages;
-                    if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag))
-                        return false;
-                    if (idx != p.ctl.inject_skip_load) {  // (test hook: this slot never fills)
+#pragma unroll
+                    for (int kv = 0; kv < 2; ++kv, ++idx) {
+                        const int s = idx % C::kStages;
+                        if (!wait_phase(bar(C::kBarEmpty + s), ((idx / C::kStages) & 1) ^ 1, p.ctl, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
                         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x)
-                            tma_load_3d(slot(s) + x * 16384, is_v ? &tm_v : &tm_k, bar(C::kBarFull + s),
+                            tma_load_3d(slot(s) + x * 16384, kv ? &tm_v : &tm_k, bar(C::kBarFull + s),
                                         x * (128 / C::kEsz), row0 + 128 * j, slab);
                         n_issued = idx + 1;
                     }
-                    ++idx;
-                    return true;
-                };
-                // With a tile mask each query tile sweeps its own key tiles: step s pairs the
-                // s-th key tile of Q0 with the s-th of Q1 and loads K then V of both (once
-                // when they coincide), so a step never idles one of the tiles.
-                int j0 = u.ts0.next(0), j1 = u.ts1.next(0);
-                while (ok && (j0 < u.ts0.hi || j1 < u.ts1.hi)) {
-                    const bool a0 = j0 < u.ts0.hi;
-                    const bool a1 = j1 < u.ts1.hi && !(a0 && j1 == j0);
-                    for (int kv = 0; kv < 2 && ok; ++kv) {
-                        if (a0) ok = load(kv != 0, j0);
-                        if (ok && a1) ok = load(kv != 0, j1);
-                    }
-                    if (j0 < u.ts0.hi) j0 = u.ts0.next(j0 + 1);
-                    if (j1 < u.ts1.hi) j1 = u.ts1.next(j1 + 1);
                 }
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == C::kIssuerWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, 0) : idesc_bf16_f32(128, 128, 0, 0);
@@ -339,89 +369,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             int base = 0;          // ring position of the unit's K_0
             int n_u = 0;           // units started
             int gs[2] = {0, 0};    // S_t products issued (all units): phase counters
-            auto wait_full = [&](int pos) {
-                return wait_phase(bar(C::kBarFull + pos % C::kStages), (pos / C::kStages) & 1, p.ctl, abort_flag);
-            };
-            FOR_EACH_UNIT(u) {
+            FOR_EACH_UNIT(u, consumer_rank) {
                 if (!ok) break;
-                if constexpr (SP) {
-                    // Independent sweeps (see the producer): the ring positions of step s's
-                    // K and V tiles for Q0 and Q1; a tile is active while its key tiles last.
-                    struct StepPos {
-                        bool a0, a1, dup;
-                        int k0, k1, v0, v1, next;
-                    };
-                    auto step_pos = [&](int j0, int j1, int pos) {
-                        StepPos r;
-                        r.a0 = j0 < u.ts0.hi;
-                        r.a1 = j1 < u.ts1.hi;
-                        r.dup = r.a0 && r.a1 && j0 == j1;
-                        const int nk = static_cast<int>(r.a0) + static_cast<int>(r.a1) - static_cast<int>(r.dup);
-                        r.k0 = pos;
-                        r.k1 = r.dup ? pos : pos + static_cast<int>(r.a0);
-                        r.v0 = pos + nk;
-                        r.v1 = r.dup ? r.v0 : r.v0 + static_cast<int>(r.a0);
-                        r.next = pos + 2 * nk;
-                        return r;
-                    };
-                    int j0 = u.ts0.next(0), j1 = u.ts1.next(0);
-                    StepPos cs = step_pos(j0, j1, base);
-                    if (!cs.a0 && !cs.a1) continue;  // no tile pair to compute
-                    ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
-                    if (ok && cs.a0) ok = wait_full(cs.k0);
-                    if (ok && cs.a1 && !cs.dup) ok = wait_full(cs.k1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (cs.a0) issue_S(0, cs.k0);
-                    if (cs.a1) issue_S(1, cs.k1);
-                    if (cs.a0) tc_commit(bar(C::kBarEmpty + cs.k0 % C::kStages));
-                    if (cs.a1 && !cs.dup) tc_commit(bar(C::kBarEmpty + cs.k1 % C::kStages));
-                    if (cs.a0) j0 = u.ts0.next(j0 + 1);
-                    if (cs.a1) j1 = u.ts1.next(j1 + 1);
-                    StepPos ns = step_pos(j0, j1, cs.next);
-                    if (!ns.a0 && !ns.a1) tc_commit(bar(C::kBarQEmpty));
-                    bool started[2] = {false, false};
-                    while (ok) {
-                        for (int t = 0; t < 2 && ok; ++t) {
-                            if (t ? cs.a1 : cs.a0) {
-                                // this tile's V (a shared one was waited for by Q0)
-                                if (!(t == 1 && cs.dup)) ok = wait_full(t ? cs.v1 : cs.v0);
-                                if (ok) ok = wait_phase(bar(C::kBarP + t), gs[t] & 1, p.ctl, abort_flag);
-                                if (!ok) break;
-                                ++gs[t];
-                                tc_fence_after();
-                                issue_PV(t, t ? cs.v1 : cs.v0, started[t]);
-                                started[t] = true;
-                                if (!(t ? ns.a1 : ns.a0)) tc_commit(bar(C::kBarO + t));  // the tile's last P V
-                                // The tile's V slot is free once its P V is done (a V tile the two
-                                // share, once Q1's is): with up to four ring loads per step the next
-                                // step's V loads must not wait for the S products issued after it.
-                                if (t == 1 || !cs.dup) tc_commit(bar(C::kBarEmpty + (t ? cs.v1 : cs.v0) % C::kStages));
-                            }
-                            if (t ? ns.a1 : ns.a0) {
-                                if (!(t == 1 && ns.dup)) {  // (a shared K tile was waited for by Q0)
-                                    ok = wait_full(t ? ns.k1 : ns.k0);
-                                    if (!ok) break;
-                                    tc_fence_after();
-                                }
-                                issue_S(t, t ? ns.k1 : ns.k0);
-                            }
-                        }
-                        if (!ok) break;
-                        if (ns.a0) tc_commit(bar(C::kBarEmpty + ns.k0 % C::kStages));
-                        if (ns.a1 && !ns.dup) tc_commit(bar(C::kBarEmpty + ns.k1 % C::kStages));
-                        if (!ns.a0 && !ns.a1) break;
-                        cs = ns;
-                        if (cs.a0) j0 = u.ts0.next(j0 + 1);
-                        if (cs.a1) j1 = u.ts1.next(j1 + 1);
-                        ns = step_pos(j0, j1, cs.next);
-                        if (!ns.a0 && !ns.a1) tc_commit(bar(C::kBarQEmpty));  // the S products just issued were the unit's last
-                    }
-                    if (!ok) break;
-                    base = cs.next;
-                    ++n_u;
-                    continue;
-                }
                 const int hi = u.nkv_max();
                 int j = u.unext(0);  // the unit's key tiles are j, unext(j + 1), ... (< hi)
                 if (j >= hi) continue;  // no tile pair to compute (tile mask)
@@ -494,7 +443,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         bool ok = true;
         int gs = 0;  // S_t phases consumed (all units)
         int go = 0;  // units in which this tile was active
-        FOR_EACH_UNIT(u) {
+        FOR_EACH_UNIT(u, consumer_rank) {
         if (!ok) break;
         // only what this tile needs is kept from the unit (registers)
         const int len = u.len;
@@ -636,7 +585,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // The tile mask leaves this tile no key tile: O = 0 and lse = -inf, like any
             // row that sees no key; nothing was computed for it.
             FwdUnit e;
-            fwd_unit<SP, false>(p, k_, cta, G, e);
+            fwd_unit<SP, NT, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
             if (row < len) {
                 const long long r = static_cast<long long>(row);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + p.g.base(e.b, e.h, e.start, D) + r * p.g.row_stride(D));
@@ -654,7 +603,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float inv = (l > 0.f) ? p.o_scale / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
-            fwd_unit<SP, false>(p, k_, cta, G, e);
+            fwd_unit<SP, NT, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
             __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
             // A warp's full 32-row block goes out by TMA store from its stage (laid out
             // as the 64-byte swizzle of a 32 x 32 box), so the warp moves on to the next
@@ -702,7 +651,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncwarp();  // reconverge the single-lane roles before the CTA barrier
     tc_fence_before();
     __syncthreads();
-    if (warp == 8 && lane == 0 && *abort_flag) {
+    if (warp == C::kProducerWarp && lane == 0 && *abort_flag) {
         // After an abort, every copy the producer started must land before the CTA
         // exits (the flag is final here: every role has finished).
         for (int s = 0; s < C::kStages; ++s) {
@@ -712,15 +661,47 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (n_qload > 0) drain_phase(bar(C::kBarQ), (n_qload - 1) & 1, p.ctl, abort_flag);
     }
-    if (warp == 9) {
+    if (warp == C::kIssuerWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+    if constexpr (kDyn) {
+        // the last CTA to finish returns the counters to zero for the slot's next launch
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+                atomicExch(p.sched, 0u);
+                atomicExch(p.sched + 1, 0u);
+            }
+        }
+    }
 }
 
-template <int D, bool SP, bool F8 = false>
+// Counter pairs of the dynamic deal, one per launch in flight: a launch takes the next
+// pair round-robin and its last CTA returns the pair to zero.  Launches reuse a pair
+// only 1024 launches later; a device runs at most 128 kernels at once, and launches of
+// one CUDA graph run in order, so two launches never hold the same pair together.
+constexpr int kSchedSlots = 1024;
+__device__ unsigned int g_fwd_sched[kSchedSlots][2];
+
+static unsigned int *next_sched_slot() {
+    static std::atomic<unsigned int> cursor{0};
+    static std::atomic<unsigned int *> base[64];  // per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    unsigned int *b = base[dev].load();
+    if (b == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_fwd_sched) != cudaSuccess) return nullptr;
+        b = static_cast<unsigned int *>(ptr);
+        base[dev].store(b);
+    }
+    return b + 2 * (cursor.fetch_add(1u) % kSchedSlots);
+}
+
+template <int D, bool SP, bool F8 = false, int NT = 2>
 static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
-    using C = FwdCfg<D, F8>;
+    using C = FwdCfg<D, F8, NT>;
     FwdParams p{};
     p.g = a.g;
     p.ctl = a.ctl;
@@ -733,22 +714,29 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
         p.o_scale = a.v_scale;
     }
     p.causal = a.causal;
-    p.n_pairs = (a.g.N + 255) / 256;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    p.n_units = (a.g.N + 128 * NT - 1) / (128 * NT);
+    p.sched = nullptr;
+    if constexpr (SP && NT == 1) {
+        p.sched = next_sched_slot();
+        if (p.sched == nullptr) return cudaErrorInvalidSymbol;
+    }
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP, F8, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The in-kernel register reallocation assumes the launch register count it was
     // sized for; with fewer, an increase could never be satisfied, so refuse.
     static const cudaError_t regs_ok = [] {
         cudaFuncAttributes fa{};
-        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP, F8>);
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP, F8, NT>);
         if (r != cudaSuccess) return r;
         return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
     }();
     if (regs_ok != cudaSuccess) return regs_ok;
-    const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_pairs;
-    const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-    attn_fwd_sm100_kernel<D, SP, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st, p);
+    const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_units;
+    const long long slots = static_cast<long long>(a.num_sms) * C::kCtasPerSm;
+    const dim3 grid(static_cast<unsigned>(units < slots ? units : slots));
+    attn_fwd_sm100_kernel<D, SP, F8, NT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st,
+                                                                                    p);
     return cudaGetLastError();
 }
 
@@ -760,8 +748,9 @@ cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {
     const bool sp = a.g.block_mask != nullptr;
-    if (a.g.d == 128) return sp ? launch_fwd_d<128, true>(a, stream) : launch_fwd_d<128, false>(a, stream);
-    return sp ? launch_fwd_d<64, true>(a, stream) : launch_fwd_d<64, false>(a, stream);
+    // a tile mask: one query tile per CTA, two CTAs per SM
+    if (a.g.d == 128) return sp ? launch_fwd_d<128, true, false, 1>(a, stream) : launch_fwd_d<128, false>(a, stream);
+    return sp ? launch_fwd_d<64, true, false, 1>(a, stream) : launch_fwd_d<64, false>(a, stream);
 }
 
 }  // namespace attn
