@@ -129,6 +129,7 @@ struct FusedParams {
     float scale_log2;
     int causal;
     int n_tiles;  // 128-row tiles per slice
+    int band;     // slices per band of the rank order (rank_to_unit)
 };
 
 __device__ __forceinline__ uint32_t kstep(int kk) { return (kk >> 2) * 16384 + (kk & 3) * 32; }
@@ -145,7 +146,9 @@ __device__ __forceinline__ void stage_rows32_f32(uint32_t box, const uint32_t (&
 
 }  // namespace
 
-template <int D, bool SP>
+// BANDED: ranks walk the slices in bands (rank_to_unit) -- only when the slices' Q, dO
+// and dQ far exceed the L2 cache; otherwise unit index first over all slices.
+template <int D, bool SP, bool BANDED>
 __global__ void __launch_bounds__(512, 1)
 attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -168,15 +171,21 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     const int BH = p.g.B * p.g.H;
     const int T = BH * p.n_tiles;
     // Work unit of rank r (CTA c takes ranks c, 2G-1-c, 2G+c, ...: a snake order over
-    // the units ranked heaviest first): key tile j, slice (b, h); qs = the query tiles
-    // that attend key tile j, nq of them, walked in increasing order.
+    // the units ranked heaviest first, within bands of slices when BANDED): key tile j,
+    // slice (b, h); qs = the query tiles that attend key tile j, nq of them, walked in
+    // increasing order.
     struct Tile {
         int b, h, j, start, len, kv0, i0, nq;
         TileSet qs;
     };
     auto tile_at = [&](int r, Tile &t) -> bool {
-        t.j = r / BH;
-        const int bh = r - t.j * BH;
+        int bh;
+        if constexpr (BANDED) {
+            rank_to_unit(r, p.n_tiles, BH, p.band, t.j, bh);
+        } else {
+            t.j = r / BH;
+            bh = r - t.j * BH;
+        }
         t.b = bh / p.g.H;
         t.h = bh - t.b * p.g.H;
         p.g.slice(t.b, t.start, t.len);
@@ -672,6 +681,28 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float *_
     }
 }
 
+template <int D, bool SP, bool BANDED>
+static cudaError_t launch_fused_kernel(const BwdLaunch &a, const FusedParams &p, cudaStream_t stream) {
+    using C = FusedCfg<D>;
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_fused_sm100_kernel<D, SP, BANDED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    // The in-kernel register reallocation assumes the launch register count it was
+    // sized for; with fewer, an increase could never be satisfied, so refuse.
+    static const cudaError_t regs_ok = [] {
+        cudaFuncAttributes fa{};
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_bwd_fused_sm100_kernel<D, SP, BANDED>);
+        if (r != cudaSuccess) return r;
+        return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
+    }();
+    if (regs_ok != cudaSuccess) return regs_ok;
+    const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_tiles;
+    const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
+    attn_bwd_fused_sm100_kernel<D, SP, BANDED><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v,
+                                                                                             a.tm_do, a.tm_dqacc, p);
+    return cudaGetLastError();
+}
+
 template <int D, bool SP>
 static cudaError_t launch_fused_d(const BwdLaunch &a, cudaStream_t stream) {
     using C = FusedCfg<D>;
@@ -691,23 +722,11 @@ static cudaError_t launch_fused_d(const BwdLaunch &a, cudaStream_t stream) {
         p.scale_log2 = a.scale * kLog2eF;
         p.causal = a.causal;
         p.n_tiles = (a.g.N + 127) / 128;
-        e = cudaFuncSetAttribute(attn_bwd_fused_sm100_kernel<D, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes);
+        // per slice the pairs stream Q, dO (bf16), the fp32 dQ accumulator and the row terms
+        p.band = l2_band(a.g.B * a.g.H, static_cast<double>(a.g.N) * (8.0 * a.g.d + 8.0));
+        e = p.band < a.g.B * a.g.H ? launch_fused_kernel<D, SP, true>(a, p, stream)
+                                   : launch_fused_kernel<D, SP, false>(a, p, stream);
         if (e != cudaSuccess) return e;
-        // The in-kernel register reallocation assumes the launch register count it was
-        // sized for; with fewer, an increase could never be satisfied, so refuse.
-        static const cudaError_t regs_ok = [] {
-            cudaFuncAttributes fa{};
-            const cudaError_t r = cudaFuncGetAttributes(&fa, attn_bwd_fused_sm100_kernel<D, SP>);
-            if (r != cudaSuccess) return r;
-            return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
-        }();
-        if (regs_ok != cudaSuccess) return regs_ok;
-        const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_tiles;
-        const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-        attn_bwd_fused_sm100_kernel<D, SP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v,
-                                                                                         a.tm_do, a.tm_dqacc, p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.phases & 32) {
         const long long n8 = a.rows_total * (D / 8);

@@ -98,6 +98,37 @@ __device__ __forceinline__ TileSet col_tiles(const Geom &g, int h, int kt, int l
     return t;
 }
 
+// Rank r of a persistent schedule over `units` work units per (sequence, head) slice
+// and BH slices, as (unit index k, slice bh).  The slices are taken in bands of
+// `band` (the last band may be smaller) and, inside a band, unit index first: ranks
+// 0, 1, ... are the first units of every slice of band 0, then their second units,
+// and so on.  With unit index 0 the heaviest, this is heaviest first within a band,
+// while the CTAs running at any one time share the data of one or two bands (their
+// K/V, or Q/dO/dQ), which the host sizes to fit the L2 cache.  band = BH: unit index
+// first over all slices.
+__device__ __forceinline__ void rank_to_unit(int r, int units, int BH, int band, int &k, int &bh) {
+    const int per_band = band * units;
+    const int bnd = r / per_band;
+    const int rr = r - bnd * per_band;
+    const int nb = min(band, BH - bnd * band);
+    k = rr / nb;
+    bh = bnd * band + (rr - k * nb);
+}
+
+// Slices per band for rank_to_unit: all of them unless their data exceeds four times
+// the L2 cache, then as many as fill about half of it (at least one).  Measured: with
+// the backward's Q/dO/dQ at 830 MB (8 packed sequences of up to 3,141 tokens, 32
+// heads) bands of 19 slices cut the time by 19 %; at 68-135 MB (B4 H16 N2048 d64,
+// B2 H16 N4096 d128) banding only unbalanced the last band (+15 %), and the forward,
+// whose two query tiles share each K/V load, lost 22 % at 410 MB.
+__host__ __forceinline__ int l2_band(int BH, double bytes_per_slice) {
+    constexpr double kBudget = 64.0 * 1024 * 1024;      // about half of the 126 MB L2
+    constexpr double kBandAbove = 512.0 * 1024 * 1024;  // about four times the L2
+    if (BH * bytes_per_slice <= kBandAbove) return BH;
+    const int b = static_cast<int>(kBudget / bytes_per_slice);
+    return b < 1 ? 1 : (b > BH ? BH : b);
+}
+
 struct SyncCtl {
     int *status;             // device status word (first error wins)
     unsigned long long wait_limit_ns;
