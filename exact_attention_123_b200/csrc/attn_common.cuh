@@ -121,10 +121,9 @@ __device__ __forceinline__ void rank_to_unit(int r, int units, int BH, int band,
 // heads) bands of 19 slices cut the time by 19 %; at 68-135 MB (B4 H16 N2048 d64,
 // B2 H16 N4096 d128) banding only unbalanced the last band (+15 %), and the forward,
 // whose two query tiles share each K/V load, lost 22 % at 410 MB.
-__host__ __forceinline__ int l2_band(int BH, double bytes_per_slice) {
-    constexpr double kBudget = 64.0 * 1024 * 1024;      // about half of the 126 MB L2
-    constexpr double kBandAbove = 512.0 * 1024 * 1024;  // about four times the L2
-    if (BH * bytes_per_slice <= kBandAbove) return BH;
+__host__ __forceinline__ int l2_band(int BH, double bytes_per_slice, double band_above = 512.0 * 1024 * 1024) {
+    constexpr double kBudget = 64.0 * 1024 * 1024;  // about half of the 126 MB L2
+    if (BH * bytes_per_slice <= band_above) return BH;
     const int b = static_cast<int>(kBudget / bytes_per_slice);
     return b < 1 ? 1 : (b > BH ? BH : b);
 }

@@ -136,6 +136,7 @@ struct FwdParams {
     float o_scale;     // 1, or the V dequantisation scale (e4m3)
     int causal;
     int n_units;       // (128 NT)-row query blocks per slice
+    int band;          // slices per band of the rank order (rank_to_unit; DYN only)
     unsigned int *sched;  // dynamic deal: {units claimed, CTAs finished} of this launch (else null)
 };
 
@@ -162,12 +163,17 @@ struct FwdUnit {
 };
 
 // The unit of rank r.  Sets: also build the tile sets (the epilogue needs only the
-// unit's position).
-template <bool SP, int NT, bool Sets = true>
+// unit's position).  BANDED: ranks walk bands of slices (rank_to_unit).
+template <bool SP, int NT, bool BANDED, bool Sets = true>
 __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u) {
     const int BH = p.g.B * p.g.H;
-    const int kk = r / BH;
-    const int bh = r - kk * BH;
+    int kk, bh;
+    if constexpr (BANDED) {
+        rank_to_unit(r, p.n_units, BH, p.band, kk, bh);
+    } else {
+        kk = r / BH;
+        bh = r - kk * BH;
+    }
     u.b = bh / p.g.H;
     u.h = bh - u.b * p.g.H;
     p.g.slice(u.b, u.start, u.len);
@@ -188,8 +194,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 // SP: a tile mask (block-sparse attention) is given.  F8: e4m3 inputs.  NT: query
-// tiles per CTA (see FwdCfg).
-template <int D, bool SP, bool F8, int NT>
+// tiles per CTA (see FwdCfg).  DYN: units are claimed at run time (a global counter)
+// instead of dealt, in rank order over bands of slices (rank_to_unit): tile masks and
+// packed sequences, whose units' costs are uneven.
+template <int D, bool SP, bool F8, int NT, bool DYN>
 __global__ void __launch_bounds__(FwdCfg<D, F8, NT>::kThreads, FwdCfg<D, F8, NT>::kCtasPerSm)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o_st,
@@ -210,7 +218,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int n_ranks = p.g.B * p.g.H * p.n_units;
     // Dynamic deal (tile masks): the producer claims each unit rank and publishes it
     // to the other roles through a 4-entry ring; n_ranks ends the walk.
-    constexpr bool kDyn = SP && NT == 1;
+    constexpr bool kDyn = DYN;
     volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_holder + 2);
     auto claim_rank = [&](int k) -> int {  // producer
         int r = n_ranks;
@@ -234,7 +242,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int k_ = 0; kDyn || k_ * G < n_ranks; ++k_)             \
         if (const int r_ = (RANK)(k_); kDyn && r_ >= n_ranks)    \
             break;                                               \
-        else if (FwdUnit u; r_ < n_ranks && fwd_unit<SP, NT>(p, r_, u))
+        else if (FwdUnit u; r_ < n_ranks && fwd_unit<SP, NT, DYN>(p, r_, u))
     auto producer_rank = [&](int k) -> int {
         if constexpr (kDyn) return claim_rank(k);
         else return static_rank(k);
@@ -585,7 +593,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // The tile mask leaves this tile no key tile: O = 0 and lse = -inf, like any
             // row that sees no key; nothing was computed for it.
             FwdUnit e;
-            fwd_unit<SP, NT, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
+            fwd_unit<SP, NT, DYN, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
             if (row < len) {
                 const long long r = static_cast<long long>(row);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + p.g.base(e.b, e.h, e.start, D) + r * p.g.row_stride(D));
@@ -603,7 +611,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float inv = (l > 0.f) ? p.o_scale / l : 0.f;
             const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
             FwdUnit e;  // the unit again, from the loop counter (fewer registers live in the key loop)
-            fwd_unit<SP, NT, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
+            fwd_unit<SP, NT, DYN, false>(p, kDyn ? r_ : static_rank(k_), e);  // (static: recomputed, not kept live)
             __nv_bfloat16 *orow = p.o + p.g.base(e.b, e.h, e.start, D) + static_cast<long long>(row) * p.g.row_stride(D);
             // A warp's full 32-row block goes out by TMA store from its stage (laid out
             // as the 64-byte swizzle of a 32 x 32 box), so the warp moves on to the next
@@ -699,7 +707,7 @@ static unsigned int *next_sched_slot() {
     return b + 2 * (cursor.fetch_add(1u) % kSchedSlots);
 }
 
-template <int D, bool SP, bool F8 = false, int NT = 2>
+template <int D, bool SP, bool F8 = false, int NT = 2, bool DYN = false>
 static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     using C = FwdCfg<D, F8, NT>;
     FwdParams p{};
@@ -716,18 +724,20 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     p.causal = a.causal;
     p.n_units = (a.g.N + 128 * NT - 1) / (128 * NT);
     p.sched = nullptr;
-    if constexpr (SP && NT == 1) {
+    // K and V of a slice; banded only beyond about twice the L2 cache
+    p.band = l2_band(a.g.B * a.g.H, 2.0 * a.g.N * a.g.d * C::kEsz, 256.0 * 1024 * 1024);
+    if constexpr (DYN) {
         p.sched = next_sched_slot();
         if (p.sched == nullptr) return cudaErrorInvalidSymbol;
     }
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP, F8, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, SP, F8, NT, DYN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The in-kernel register reallocation assumes the launch register count it was
     // sized for; with fewer, an increase could never be satisfied, so refuse.
     static const cudaError_t regs_ok = [] {
         cudaFuncAttributes fa{};
-        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP, F8, NT>);
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_sm100_kernel<D, SP, F8, NT, DYN>);
         if (r != cudaSuccess) return r;
         return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
     }();
@@ -735,22 +745,28 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_units;
     const long long slots = static_cast<long long>(a.num_sms) * C::kCtasPerSm;
     const dim3 grid(static_cast<unsigned>(units < slots ? units : slots));
-    attn_fwd_sm100_kernel<D, SP, F8, NT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st,
+    attn_fwd_sm100_kernel<D, SP, F8, NT, DYN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_o_st,
                                                                                     p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
-    if (a.g.d == 128) return launch_fwd_d<128, false, true>(a, stream);
-    if (a.g.d == 64) return launch_fwd_d<64, false, true>(a, stream);
+    const bool dyn = a.g.varlen != 0;  // packed sequences: uneven units, claimed at run time
+    if (a.g.d == 128) return dyn ? launch_fwd_d<128, false, true, 2, true>(a, stream) : launch_fwd_d<128, false, true>(a, stream);
+    if (a.g.d == 64) return dyn ? launch_fwd_d<64, false, true, 2, true>(a, stream) : launch_fwd_d<64, false, true>(a, stream);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd(const FwdLaunch &a, cudaStream_t stream) {
     const bool sp = a.g.block_mask != nullptr;
     // a tile mask: one query tile per CTA, two CTAs per SM
-    if (a.g.d == 128) return sp ? launch_fwd_d<128, true, false, 1>(a, stream) : launch_fwd_d<128, false>(a, stream);
-    return sp ? launch_fwd_d<64, true, false, 1>(a, stream) : launch_fwd_d<64, false>(a, stream);
+    const bool dyn = a.g.varlen != 0;  // packed sequences: uneven units, claimed at run time
+    if (a.g.d == 128) {
+        if (sp) return launch_fwd_d<128, true, false, 1, true>(a, stream);
+        return dyn ? launch_fwd_d<128, false, false, 2, true>(a, stream) : launch_fwd_d<128, false>(a, stream);
+    }
+    if (sp) return launch_fwd_d<64, true, false, 1, true>(a, stream);
+    return dyn ? launch_fwd_d<64, false, false, 2, true>(a, stream) : launch_fwd_d<64, false>(a, stream);
 }
 
 }  // namespace attn
