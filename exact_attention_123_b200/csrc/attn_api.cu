@@ -291,7 +291,29 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *o, const f
 constexpr int kDeterministicPhases = 7;  // preprocess, dK/dV pass, dQ pass
 constexpr int kFusedPhases = 56;         // preprocess + zeroing, single pass, dQ conversion
 
+// Counter pairs of the dynamic unit deals, one per launch in flight: a launch takes the
+// next pair round-robin and its last CTA returns the pair to zero.  A pair is reused
+// only 1024 launches later; a device runs at most 128 kernels at once, and launches of
+// one CUDA graph run in order, so two launches never hold the same pair together.
+constexpr int kSchedSlots = 1024;
+__device__ unsigned int g_sched_pool[kSchedSlots][2];
+
 }  // namespace
+
+unsigned int *attn::next_sched_slot() {
+    static std::atomic<unsigned int> cursor{0};
+    static std::atomic<unsigned int *> base[64];  // per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    unsigned int *b = base[dev].load();
+    if (b == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_sched_pool) != cudaSuccess) return nullptr;
+        b = static_cast<unsigned int *>(ptr);
+        base[dev].store(b);
+    }
+    return b + 2 * (cursor.fetch_add(1u) % kSchedSlots);
+}
 
 extern "C" {
 

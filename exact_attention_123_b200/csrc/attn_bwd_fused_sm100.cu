@@ -108,8 +108,11 @@ struct FusedCfg {
     static constexpr int kBarKdv = kBarSFull + 6;         // dV, dK accumulators complete
     static constexpr int kBarAccFree = kBarSFull + 7;     // dV, dK copied out of TMEM (256)
     static constexpr int kBarDone = kBarSFull + 8;
-    static constexpr int kNumBars = kBarSFull + 9;
-    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 16;  // from a 1024-byte-aligned base
+    static constexpr int kBarUFull = kBarSFull + 9;       // + entry: a claimed unit rank is published
+    static constexpr int kBarUEmpty = kBarSFull + 13;     // + entry: every role has read it (385)
+    static constexpr int kNumBars = kBarSFull + 17;
+    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed unit ranks
+    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 32;  // from a 1024-byte-aligned base
     static constexpr int kSmemMax = 232448;
     // The base of dynamic shared memory is expected to be 1024-byte aligned; the
     // kernel checks, and where the slack below cannot cover the misalignment it
@@ -130,6 +133,7 @@ struct FusedParams {
     int causal;
     int n_tiles;  // 128-row tiles per slice
     int band;     // slices per band of the rank order (rank_to_unit)
+    unsigned int *sched;  // claimed deal: {units claimed, CTAs finished} of this launch (else null)
 };
 
 __device__ __forceinline__ uint32_t kstep(int kk) { return (kk >> 2) * 16384 + (kk & 3) * 32; }
@@ -146,9 +150,12 @@ __device__ __forceinline__ void stage_rows32_f32(uint32_t box, const uint32_t (&
 
 }  // namespace
 
-// BANDED: ranks walk the slices in bands (rank_to_unit) -- only when the slices' Q, dO
-// and dQ far exceed the L2 cache; otherwise unit index first over all slices.
-template <int D, bool SP, bool BANDED>
+// SCHED: how the CTAs get their units.  0: dealt (a snake order over the ranks, unit
+// index first over all slices).  1: claimed at run time from a global counter, in rank
+// order (tile masks, whose units' costs are uneven).  2: claimed, and the ranks walk
+// the slices in bands (rank_to_unit) -- when the slices' Q, dO and dQ far exceed the
+// L2 cache.
+template <int D, bool SP, int SCHED>
 __global__ void __launch_bounds__(512, 1)
 attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -170,17 +177,18 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
     const int BH = p.g.B * p.g.H;
     const int T = BH * p.n_tiles;
-    // Work unit of rank r (CTA c takes ranks c, 2G-1-c, 2G+c, ...: a snake order over
-    // the units ranked heaviest first, within bands of slices when BANDED): key tile j,
-    // slice (b, h); qs = the query tiles that attend key tile j, nq of them, walked in
-    // increasing order.
+    // Work unit of rank r (SCHED 0: CTA c takes ranks c, 2G-1-c, 2G+c, ..., a snake
+    // order over the units ranked heaviest first; else the ranks it claims, in order,
+    // within bands of slices when SCHED = 2): key tile j, slice (b, h); qs = the query
+    // tiles that attend key tile j, nq of them, walked in increasing order.
+    constexpr bool kDyn = SCHED != 0;
     struct Tile {
         int b, h, j, start, len, kv0, i0, nq;
         TileSet qs;
     };
     auto tile_at = [&](int r, Tile &t) -> bool {
         int bh;
-        if constexpr (BANDED) {
+        if constexpr (SCHED == 2) {
             rank_to_unit(r, p.n_tiles, BH, p.band, t.j, bh);
         } else {
             t.j = r / BH;
@@ -197,6 +205,27 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         return true;
     };
     auto rank_of = [&](int k) { return k * G + ((k & 1) ? (G - 1 - cta) : cta); };
+    // Claimed deal: the loader claims each rank and publishes it to the issuer, the drain
+    // and the math warps through a 4-entry ring; T ends the walk.
+    volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_holder + 2);
+    auto publish_rank = [&](int k) -> int {  // loader, lane 0
+        int r = T;
+        if (!*abort_flag) r = min(static_cast<int>(atomicAdd(p.sched, 1u)), T);
+        if (!wait_phase(bar(C::kBarUEmpty + (k & 3)), ((k >> 2) & 1) ^ 1, p.ctl, abort_flag)) return T;
+        unit_ring[k & 3] = r;
+        mbar_arrive(bar(C::kBarUFull + (k & 3)));
+        return r;
+    };
+    auto consumer_rank = [&](int k) -> int {  // issuer, drain and math threads
+        if constexpr (kDyn) {
+            if (!wait_phase(bar(C::kBarUFull + (k & 3)), (k >> 2) & 1, p.ctl, abort_flag)) return T;
+            const int r = unit_ring[k & 3];
+            mbar_arrive(bar(C::kBarUEmpty + (k & 3)));
+            return r;
+        } else {
+            return rank_of(k);
+        }
+    };
 
     if (warp == 13) {
         tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -207,6 +236,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             uint32_t cnt = 1;
             if (i == C::kBarPFull || i == C::kBarDSFull || i == C::kBarAccFree) cnt = 256;
             if (i == C::kBarDQFree) cnt = 128;
+            if (i >= C::kBarUEmpty && i < C::kBarUEmpty + 4) cnt = 1 + 128 + 256;  // issuer, drain, math
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
@@ -229,9 +259,22 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 tma_prefetch_desc(&tm_do);
             }
             bool ok = true;
+            int r_next = 0;  // claimed deal: the next unit, claimed one unit ahead (its L2 prefetch)
+            if constexpr (kDyn) {
+                if (lane == 0) r_next = publish_rank(0);
+                r_next = __shfl_sync(0xffffffffu, r_next, 0);
+            }
             for (int k = 0; ok; ++k) {
-                const int r = rank_of(k);
-                if (r >= T) break;
+                int r;
+                if constexpr (kDyn) {
+                    r = r_next;
+                    if (r >= T) break;
+                    if (lane == 0) r_next = publish_rank(k + 1);
+                    r_next = __shfl_sync(0xffffffffu, r_next, 0);
+                } else {
+                    r = rank_of(k);
+                    if (r >= T) break;
+                }
                 Tile t;
                 if (!tile_at(r, t) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
@@ -253,7 +296,17 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 if (!ok) break;
                 ++n_kv;
                 // the next unit's K and V tiles into L2 while this unit runs
-                if (lane == 0) {
+                if (kDyn && lane == 0) {
+                    Tile t2;
+                    if (r_next < T && tile_at(r_next, t2) && t2.nq > 0) {
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x) {
+                            tma_prefetch_l2_3d(&tm_k, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
+                            tma_prefetch_l2_3d(&tm_v, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
+                        }
+                    }
+                }
+                if (!kDyn && lane == 0) {
                     for (int k2 = k + 1;; ++k2) {
                         const int r2 = rank_of(k2);
                         if (r2 >= T) break;
@@ -353,7 +406,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 bool ok = true;
                 int gbase = 0, n_t = 0;
                 for (int k = 0; ok; ++k) {
-                    const int r = rank_of(k);
+                    const int r = consumer_rank(k);
                     if (r >= T) break;
                     Tile t;
                     if (!tile_at(r, t) || t.nq == 0) continue;
@@ -461,7 +514,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         bool ok = true;
         int gbase = 0;
         for (int k = 0; ok; ++k) {
-            const int r = rank_of(k);
+            const int r = consumer_rank(k);
             if (r >= T) break;
             Tile t;
             if (!tile_at(r, t) || t.nq == 0) continue;
@@ -512,7 +565,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         bool ok = true;
         int gbase = 0, n_t = 0;
         for (int k = 0; ok; ++k) {
-            const int r = rank_of(k);
+            const int r = consumer_rank(k);
             if (r >= T) break;
             Tile t;
             if (!tile_at(r, t)) continue;
@@ -659,6 +712,16 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+    if constexpr (kDyn) {
+        // the last CTA to finish returns the counters to zero for the pair's next launch
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+                atomicExch(p.sched, 0u);
+                atomicExch(p.sched + 1, 0u);
+            }
+        }
+    }
 }
 
 // dQ = bf16(scale * accumulator) over the rows that hold tokens (the flat [rows, d]
@@ -681,24 +744,24 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float *_
     }
 }
 
-template <int D, bool SP, bool BANDED>
+template <int D, bool SP, int SCHED>
 static cudaError_t launch_fused_kernel(const BwdLaunch &a, const FusedParams &p, cudaStream_t stream) {
     using C = FusedCfg<D>;
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_fused_sm100_kernel<D, SP, BANDED>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_fused_sm100_kernel<D, SP, SCHED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // The in-kernel register reallocation assumes the launch register count it was
     // sized for; with fewer, an increase could never be satisfied, so refuse.
     static const cudaError_t regs_ok = [] {
         cudaFuncAttributes fa{};
-        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_bwd_fused_sm100_kernel<D, SP, BANDED>);
+        const cudaError_t r = cudaFuncGetAttributes(&fa, attn_bwd_fused_sm100_kernel<D, SP, SCHED>);
         if (r != cudaSuccess) return r;
         return fa.numRegs == C::kLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
     }();
     if (regs_ok != cudaSuccess) return regs_ok;
     const long long units = static_cast<long long>(a.g.B) * a.g.H * p.n_tiles;
     const dim3 grid(static_cast<unsigned>(units < a.num_sms ? units : a.num_sms));
-    attn_bwd_fused_sm100_kernel<D, SP, BANDED><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v,
+    attn_bwd_fused_sm100_kernel<D, SP, SCHED><<<grid, C::kThreads, C::kSmemBytes, stream>>>(a.tm_q, a.tm_k, a.tm_v,
                                                                                              a.tm_do, a.tm_dqacc, p);
     return cudaGetLastError();
 }
@@ -724,8 +787,17 @@ static cudaError_t launch_fused_d(const BwdLaunch &a, cudaStream_t stream) {
         p.n_tiles = (a.g.N + 127) / 128;
         // per slice the pairs stream Q, dO (bf16), the fp32 dQ accumulator and the row terms
         p.band = l2_band(a.g.B * a.g.H, static_cast<double>(a.g.N) * (8.0 * a.g.d + 8.0));
-        e = p.band < a.g.B * a.g.H ? launch_fused_kernel<D, SP, true>(a, p, stream)
-                                   : launch_fused_kernel<D, SP, false>(a, p, stream);
+        // tile masks: claimed units; banded rank order: claimed too (the static deal of a
+        // banded order balances badly); otherwise dealt
+        p.sched = nullptr;
+        const bool banded = p.band < a.g.B * a.g.H;
+        if (SP || banded) {
+            p.sched = next_sched_slot();
+            if (p.sched == nullptr) return cudaErrorInvalidSymbol;
+        }
+        if (banded) e = launch_fused_kernel<D, SP, 2>(a, p, stream);
+        else if constexpr (SP) e = launch_fused_kernel<D, SP, 1>(a, p, stream);
+        else e = launch_fused_kernel<D, SP, 0>(a, p, stream);
         if (e != cudaSuccess) return e;
     }
     if (a.phases & 32) {

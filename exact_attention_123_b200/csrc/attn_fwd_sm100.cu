@@ -56,7 +56,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cmath>
 
 #include "attn_common.cuh"
@@ -683,28 +682,6 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
     }
-}
-
-// Counter pairs of the dynamic deal, one per launch in flight: a launch takes the next
-// pair round-robin and its last CTA returns the pair to zero.  Launches reuse a pair
-// only 1024 launches later; a device runs at most 128 kernels at once, and launches of
-// one CUDA graph run in order, so two launches never hold the same pair together.
-constexpr int kSchedSlots = 1024;
-__device__ unsigned int g_fwd_sched[kSchedSlots][2];
-
-static unsigned int *next_sched_slot() {
-    static std::atomic<unsigned int> cursor{0};
-    static std::atomic<unsigned int *> base[64];  // per device
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    unsigned int *b = base[dev].load();
-    if (b == nullptr) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_fwd_sched) != cudaSuccess) return nullptr;
-        b = static_cast<unsigned int *>(ptr);
-        base[dev].store(b);
-    }
-    return b + 2 * (cursor.fetch_add(1u) % kSchedSlots);
 }
 
 template <int D, bool SP, bool F8 = false, int NT = 2, bool DYN = false>

@@ -48,5 +48,8 @@ cudaError_t launch_bwd(const BwdLaunch &a, cudaStream_t stream);
 // the backward's per-row terms D and lse2 (and, with zero_dqacc, zeroes a.dqacc)
 cudaError_t launch_bwd_pre(const BwdLaunch &a, bool zero_dqacc, cudaStream_t stream);
 cudaError_t launch_bwd_fused(const BwdLaunch &a, cudaStream_t stream);  // phases bits 3-5
+// A zeroed {units claimed, CTAs finished} counter pair in device memory for one launch
+// of a kernel with a dynamic unit deal (null if the device's pool cannot be reached).
+unsigned int *next_sched_slot();
 
 }  // namespace attn
