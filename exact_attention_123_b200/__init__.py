@@ -11,7 +11,7 @@ The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen
 ``attn_fwd_fp8_varlen``,
 ``attn_bwd_workspace_bytes``, ``attn_bwd_deterministic_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
-``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``.
+``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``, ``attn_debug_force_band``.
 """
 from __future__ import annotations
 
@@ -77,12 +77,13 @@ def lib() -> ctypes.CDLL:
     L.attn_strerror.restype = ctypes.c_char_p
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
+    L.attn_debug_force_band.argtypes = [i]
     L.attn_debug_ex2_poly.argtypes = [vp, vp, ctypes.c_longlong, vp]
     for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_deterministic",
                  "attn_bwd_varlen", "attn_bwd_phase",
                  "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked",
                  "attn_fwd_fp8_varlen", "attn_status", "attn_set_wait_limit_ms",
-                 "attn_debug_skip_load", "attn_debug_ex2_poly"):
+                 "attn_debug_skip_load", "attn_debug_ex2_poly", "attn_debug_force_band"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -417,6 +418,12 @@ def attn_set_wait_limit_ms(ms: int) -> int:
 
 def attn_debug_skip_load(index: int) -> int:
     return int(lib().attn_debug_skip_load(int(index)))
+
+
+def attn_debug_force_band(slices: int) -> int:
+    """Test hook: force bands of `slices` slices in the banded unit order (0: automatic).
+    Returns the previous value."""
+    return int(lib().attn_debug_force_band(int(slices)))
 
 
 def attn_debug_ex2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:

@@ -36,6 +36,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
 
 std::atomic<int> g_wait_limit_ms{4000};
 std::atomic<int> g_skip_load{-1};
+std::atomic<int> g_force_band{0};  // test hook: slices per band forced (0: automatic)
 
 struct DeviceState {
     std::once_flag once;
@@ -300,6 +301,8 @@ __device__ unsigned int g_sched_pool[kSchedSlots][2];
 
 }  // namespace
 
+int attn::forced_band() { return g_force_band.load(); }
+
 unsigned int *attn::next_sched_slot() {
     static std::atomic<unsigned int> cursor{0};
     static std::atomic<unsigned int *> base[64];  // per device
@@ -476,5 +479,7 @@ int attn_debug_ex2_poly(const float *x, float *y, long long n, void *stream) {
 int attn_debug_skip_load(int load_index) {
     return g_skip_load.exchange(load_index < 0 ? -1 : load_index);
 }
+
+int attn_debug_force_band(int slices) { return g_force_band.exchange(slices > 0 ? slices : 0); }
 
 }  // extern "C"

@@ -787,6 +787,7 @@ static cudaError_t launch_fused_d(const BwdLaunch &a, cudaStream_t stream) {
         p.n_tiles = (a.g.N + 127) / 128;
         // per slice the pairs stream Q, dO (bf16), the fp32 dQ accumulator and the row terms
         p.band = l2_band(a.g.B * a.g.H, static_cast<double>(a.g.N) * (8.0 * a.g.d + 8.0));
+        if (forced_band() > 0) p.band = min(forced_band(), a.g.B * a.g.H);  // (test hook)
         // tile masks: claimed units; banded rank order: claimed too (the static deal of a
         // banded order balances badly); otherwise dealt
         p.sched = nullptr;

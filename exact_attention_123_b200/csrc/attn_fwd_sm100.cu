@@ -703,6 +703,7 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
     p.sched = nullptr;
     // K and V of a slice; banded only beyond about twice the L2 cache
     p.band = l2_band(a.g.B * a.g.H, 2.0 * a.g.N * a.g.d * C::kEsz, 256.0 * 1024 * 1024);
+    if (forced_band() > 0) p.band = min(forced_band(), a.g.B * a.g.H);  // (test hook; DYN kernels only)
     if constexpr (DYN) {
         p.sched = next_sched_slot();
         if (p.sched == nullptr) return cudaErrorInvalidSymbol;

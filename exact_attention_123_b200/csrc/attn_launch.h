@@ -51,5 +51,7 @@ cudaError_t launch_bwd_fused(const BwdLaunch &a, cudaStream_t stream);  // phase
 // A zeroed {units claimed, CTAs finished} counter pair in device memory for one launch
 // of a kernel with a dynamic unit deal (null if the device's pool cannot be reached).
 unsigned int *next_sched_slot();
+// Slices per band forced by attn_debug_force_band (0: the launchers choose).
+int forced_band();
 
 }  // namespace attn

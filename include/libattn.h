@@ -342,6 +342,19 @@ ATTN_API int attn_debug_skip_load(int load_index);
  */
 ATTN_API int attn_debug_ex2_poly(const float *x, float *y, long long n, void *stream);
 
+/*
+ * Test hook for the banded unit order.  When the data of the (sequence, head) slices
+ * far exceeds the L2 cache, the single-pass backward (Q, dO and the fp32 dQ
+ * accumulator beyond 512 MB) and the packed and block-sparse forwards (K and V
+ * beyond 256 MB) walk their units in bands of slices that fit about half of the L2
+ * cache, claiming units at run time.  For later launches from this process,
+ * slices > 0 forces bands of that many slices (at most B*H) at any size, so that
+ * tests can run those kernels on small problems; 0 (the default) restores the
+ * automatic choice.  The results do not depend on the order (the backward's dQ up
+ * to the order of its fp32 additions).  Returns the previous value.
+ */
+ATTN_API int attn_debug_force_band(int slices);
+
 #ifdef __cplusplus
 }
 #endif

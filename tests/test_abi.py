@@ -160,6 +160,9 @@ def test_wait_limit_and_fault_hook_setters(L):
     assert ea.attn_set_wait_limit_ms(prev) == 1234
     assert ea.attn_debug_skip_load(5) == -1
     assert ea.attn_debug_skip_load(-1) == 5
+    assert ea.attn_debug_force_band(3) == 0
+    assert ea.attn_debug_force_band(-2) == 3  # (non-positive: automatic)
+    assert ea.attn_debug_force_band(0) == 0
 
 
 def test_product_package_never_touches_the_oracle():
