@@ -655,7 +655,7 @@ def ncu_kernel_key(name: str) -> str:
     the bench times, the name with its template arguments otherwise."""
     base = name.split("(")[0].replace("void ", "").replace("attn::", "").strip()
     short, _, args = base.partition("<")
-    return short if args.rstrip(">") in ("128, 0", "128, 0, 0") else base
+    return short if args.rstrip(">") in ("128, 0", "128, 0, 0", "128, 0, 0, 2, 0") else base
 
 
 def ncu_rows(csv_text: str):
