@@ -119,8 +119,9 @@ struct FwdCfg {
     static constexpr int kOffP = kSmemTiles;                   // e4m3 P_0, P_1: 128 x 128 bytes each
     static constexpr int kOffStage = kOffP + (F8 ? 2 * 16384 : 0);  // 2 KB output stage per softmax warp
     static constexpr int kOffBar = kOffStage + 4 * NT * 2048;
-    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed unit ranks
-    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 32;
+    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
+    // ({rank, key-tile bits}, 16 bytes each)
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 96;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
     // 227 KB per CTA; two CTAs share an SM's 228 KB less 1 KB reserved per CTA
     static_assert(kSmemBytes <= (NT == 1 ? 115712 : 232448), "exceeds the per-CTA shared-memory limit");
@@ -162,9 +163,11 @@ struct FwdUnit {
 };
 
 // The unit of rank r.  Sets: also build the tile sets (the epilogue needs only the
-// unit's position).  BANDED: ranks walk bands of slices (rank_to_unit).
+// unit's position), from the mask or, if `bits` is given, from Q0's key-tile bits
+// read by another role (one query tile per CTA, or no mask).  BANDED: ranks walk
+// bands of slices (rank_to_unit).
 template <bool SP, int NT, bool BANDED, bool Sets = true>
-__device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u) {
+__device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u, const uint64_t *bits = nullptr) {
     const int BH = p.g.B * p.g.H;
     int kk, bh;
     if constexpr (BANDED) {
@@ -183,8 +186,13 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u) 
     u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
     u.nkv1 = (NT == 1 || r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
     if constexpr (Sets) {
-        u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
-        u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
+        if (bits != nullptr) {
+            u.ts0 = TileSet{*bits, 0, u.nkv0, SP};
+            u.ts1 = TileSet{0ull, 0, u.nkv1, SP};
+        } else {
+            u.ts0 = row_tiles<SP>(p.g, u.h, u.m0 / 128, u.nkv0);
+            u.ts1 = row_tiles<SP>(p.g, u.h, u.m0 / 128 + 1, u.nkv1);
+        }
     }
     return true;
 }
@@ -215,21 +223,27 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
     const int n_ranks = p.g.B * p.g.H * p.n_units;
-    // Dynamic deal (tile masks): the producer claims each unit rank and publishes it
-    // to the other roles through a 4-entry ring; n_ranks ends the walk.
+    // Dynamic deal: the producer claims each unit rank, reads the unit's mask row and
+    // publishes {rank, Q0's key-tile bits} to the other roles through a 4-entry ring (so
+    // only the producer reads the mask); n_ranks ends the walk.
     constexpr bool kDyn = DYN;
-    volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_holder + 2);
+    volatile uint64_t *unit_ring = reinterpret_cast<volatile uint64_t *>(tmem_holder + 2);  // 8-byte aligned
+    uint64_t unit_bits = 0;  // key-tile bits of the unit of the role's last rank (dynamic deal)
     auto claim_rank = [&](int k) -> int {  // producer
         int r = n_ranks;
         if (!*abort_flag) r = min(static_cast<int>(atomicAdd(p.sched, 1u)), n_ranks);
+        unit_bits = 0;
+        if (FwdUnit un; r < n_ranks && fwd_unit<SP, NT, DYN>(p, r, un)) unit_bits = un.ts0.bits;
         if (!wait_phase(bar(C::kBarUEmpty + (k & 3)), ((k >> 2) & 1) ^ 1, p.ctl, abort_flag)) return n_ranks;
-        unit_ring[k & 3] = r;
+        unit_ring[2 * (k & 3)] = static_cast<uint64_t>(r);
+        unit_ring[2 * (k & 3) + 1] = unit_bits;
         mbar_arrive(bar(C::kBarUFull + (k & 3)));
         return r;
     };
     auto take_rank = [&](int k) -> int {  // issuer and softmax threads
         if (!wait_phase(bar(C::kBarUFull + (k & 3)), (k >> 2) & 1, p.ctl, abort_flag)) return n_ranks;
-        const int r = unit_ring[k & 3];
+        const int r = static_cast<int>(unit_ring[2 * (k & 3)]);
+        unit_bits = unit_ring[2 * (k & 3) + 1];
         mbar_arrive(bar(C::kBarUEmpty + (k & 3)));
         return r;
     };
@@ -241,7 +255,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int k_ = 0; kDyn || k_ * G < n_ranks; ++k_)             \
         if (const int r_ = (RANK)(k_); kDyn && r_ >= n_ranks)    \
             break;                                               \
-        else if (FwdUnit u; r_ < n_ranks && fwd_unit<SP, NT, DYN>(p, r_, u))
+        else if (FwdUnit u; r_ < n_ranks && fwd_unit<SP, NT, DYN>(p, r_, u, kDyn ? &unit_bits : nullptr))
     auto producer_rank = [&](int k) -> int {
         if constexpr (kDyn) return claim_rank(k);
         else return static_rank(k);
