@@ -111,8 +111,9 @@ struct FusedCfg {
     static constexpr int kBarUFull = kBarSFull + 9;       // + entry: a claimed unit rank is published
     static constexpr int kBarUEmpty = kBarSFull + 13;     // + entry: every role has read it (385)
     static constexpr int kNumBars = kBarSFull + 17;
-    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed unit ranks
-    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 32;  // from a 1024-byte-aligned base
+    // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
+    // ({rank, query-tile bits}, 16 bytes each)
+    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 80;  // from a 1024-byte-aligned base
     static constexpr int kSmemMax = 232448;
     // The base of dynamic shared memory is expected to be 1024-byte aligned; the
     // kernel checks, and where the slack below cannot cover the misalignment it
@@ -186,7 +187,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         int b, h, j, start, len, kv0, i0, nq;
         TileSet qs;
     };
-    auto tile_at = [&](int r, Tile &t) -> bool {
+    // (bits: the unit's query-tile bits as another role read them from the mask)
+    auto tile_at = [&](int r, Tile &t, const uint64_t *bits = nullptr) -> bool {
         int bh;
         if constexpr (SCHED == 2) {
             rank_to_unit(r, p.n_tiles, BH, p.band, t.j, bh);
@@ -200,26 +202,33 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         t.kv0 = t.j * 128;
         if (t.kv0 >= t.len) return false;
         t.i0 = p.causal ? t.j : 0;
-        t.qs = col_tiles<SP>(p.g, t.h, t.j, t.i0, (t.len + 127) / 128);
+        t.qs = bits ? TileSet{*bits, t.i0, (t.len + 127) / 128, SP} : col_tiles<SP>(p.g, t.h, t.j, t.i0, (t.len + 127) / 128);
         t.nq = t.qs.count();
         return true;
     };
     auto rank_of = [&](int k) { return k * G + ((k & 1) ? (G - 1 - cta) : cta); };
-    // Claimed deal: the loader claims each rank and publishes it to the issuer, the drain
-    // and the math warps through a 4-entry ring; T ends the walk.
-    volatile int *unit_ring = reinterpret_cast<volatile int *>(tmem_holder + 2);
-    auto publish_rank = [&](int k) -> int {  // loader, lane 0
+    // Claimed deal: the loader claims each rank, reads the unit's column of the tile
+    // mask and publishes {rank, query-tile bits} to the issuer, the drain and the math
+    // warps through a 4-entry ring (so only the loader reads the mask); T ends the walk.
+    volatile uint64_t *unit_ring = reinterpret_cast<volatile uint64_t *>(tmem_holder + 2);  // 8-byte aligned
+    uint64_t unit_bits = 0;  // the query-tile bits of the unit of the role's last rank
+    const uint64_t *ubits = kDyn ? &unit_bits : nullptr;
+    auto publish_rank = [&](int k, uint64_t &bits) -> int {  // loader, lane 0
         int r = T;
         if (!*abort_flag) r = min(static_cast<int>(atomicAdd(p.sched, 1u)), T);
+        bits = 0;
+        if (Tile tn; r < T && tile_at(r, tn)) bits = tn.qs.bits;
         if (!wait_phase(bar(C::kBarUEmpty + (k & 3)), ((k >> 2) & 1) ^ 1, p.ctl, abort_flag)) return T;
-        unit_ring[k & 3] = r;
+        unit_ring[2 * (k & 3)] = static_cast<uint64_t>(r);
+        unit_ring[2 * (k & 3) + 1] = bits;
         mbar_arrive(bar(C::kBarUFull + (k & 3)));
         return r;
     };
     auto consumer_rank = [&](int k) -> int {  // issuer, drain and math threads
         if constexpr (kDyn) {
             if (!wait_phase(bar(C::kBarUFull + (k & 3)), (k >> 2) & 1, p.ctl, abort_flag)) return T;
-            const int r = unit_ring[k & 3];
+            const int r = static_cast<int>(unit_ring[2 * (k & 3)]);
+            unit_bits = unit_ring[2 * (k & 3) + 1];
             mbar_arrive(bar(C::kBarUEmpty + (k & 3)));
             return r;
         } else {
@@ -260,23 +269,27 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             }
             bool ok = true;
             int r_next = 0;  // claimed deal: the next unit, claimed one unit ahead (its L2 prefetch)
+            uint64_t bits_next = 0;
             if constexpr (kDyn) {
-                if (lane == 0) r_next = publish_rank(0);
+                if (lane == 0) r_next = publish_rank(0, bits_next);
                 r_next = __shfl_sync(0xffffffffu, r_next, 0);
+                bits_next = __shfl_sync(0xffffffffu, bits_next, 0);
             }
             for (int k = 0; ok; ++k) {
                 int r;
                 if constexpr (kDyn) {
                     r = r_next;
+                    unit_bits = bits_next;
                     if (r >= T) break;
-                    if (lane == 0) r_next = publish_rank(k + 1);
+                    if (lane == 0) r_next = publish_rank(k + 1, bits_next);
                     r_next = __shfl_sync(0xffffffffu, r_next, 0);
+                    bits_next = __shfl_sync(0xffffffffu, bits_next, 0);
                 } else {
                     r = rank_of(k);
                     if (r >= T) break;
                 }
                 Tile t;
-                if (!tile_at(r, t) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
+                if (!tile_at(r, t, ubits) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
                 const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
                 // V_j once the previous unit's last dP^T is done, K_j once its last dQ is
@@ -298,7 +311,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 // the next unit's K and V tiles into L2 while this unit runs
                 if (kDyn && lane == 0) {
                     Tile t2;
-                    if (r_next < T && tile_at(r_next, t2) && t2.nq > 0) {
+                    if (r_next < T && tile_at(r_next, t2, &bits_next) && t2.nq > 0) {
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x) {
                             tma_prefetch_l2_3d(&tm_k, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
@@ -409,7 +422,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     const int r = consumer_rank(k);
                     if (r >= T) break;
                     Tile t;
-                    if (!tile_at(r, t) || t.nq == 0) continue;
+                    if (!tile_at(r, t, ubits) || t.nq == 0) continue;
                     ok = wait_phase(bar(C::kBarKFull), n_t & 1, p.ctl, abort_flag);
                     if (ok) ok = wait_q(gbase);
                     if (!ok) break;
@@ -517,7 +530,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             const int r = consumer_rank(k);
             if (r >= T) break;
             Tile t;
-            if (!tile_at(r, t) || t.nq == 0) continue;
+            if (!tile_at(r, t, ubits) || t.nq == 0) continue;
             const int row0 = p.g.tma_row0(t.start) + q4 * 32, slab = p.g.tma_slab(t.b, t.h);
             for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
                 const int gi = gbase + it;
@@ -568,7 +581,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             const int r = consumer_rank(k);
             if (r >= T) break;
             Tile t;
-            if (!tile_at(r, t)) continue;
+            if (!tile_at(r, t, ubits)) continue;
             const int key = t.kv0 + kr;
             if (t.nq == 0) {
                 // The tile mask leaves key tile j no query tile: dV = dK = 0 for its keys
