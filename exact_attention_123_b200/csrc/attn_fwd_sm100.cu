@@ -631,7 +631,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // unit without waiting for the global writes; a block reaching past the
             // sequence's end (which a packed layout could not clip) is stored row by row.
             const int row_w0 = row - lane;
-            const bool by_tma = len - row_w0 >= 32;
+            // (one tile per CTA at d = 64: direct stores, whose latency the other CTA of the SM
+            // hides; measured 4 % faster there, neutral at d = 128)
+            const bool by_tma = (NT == 2 || D == 128) && len - row_w0 >= 32;
             const uint32_t stage = sbase + C::kOffStage + warp * 2048;
 #pragma unroll 1  // (unrolled, the 128-wide key loop above runs out of registers)
             for (int q = 0; q < D / 32; ++q) {
