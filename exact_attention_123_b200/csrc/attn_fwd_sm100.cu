@@ -160,6 +160,27 @@ struct FwdUnit {
         const int r = min(a < ts0.hi ? a : INT_MAX, b < ts1.hi ? b : INT_MAX);
         return r == INT_MAX ? nkv_max() : r;
     }
+    // Sweep order.  Causal, without a tile mask, Q1 reaches one key tile past Q0 (its
+    // diagonal tile): that tile goes first, then the shared tiles in increasing order,
+    // so that both tiles finish a unit on the same step -- the step Q1 runs alone falls
+    // at the start of the next unit, where Q0's warps spend it writing the previous
+    // unit's output, instead of at the end, where both would wait.  (The online
+    // softmax does not depend on the order of the key tiles.)
+    // (Used at d = 64, where a unit is short; at d = 128 the extra code cost more than the
+    // idle step, measured.)
+    bool diag_first;
+    template <bool DF>
+    __device__ __forceinline__ int ufirst() const { return (DF && diag_first) ? nkv1 - 1 : unext(0); }
+    template <bool DF>
+    __device__ __forceinline__ int uafter(int j) const {  // the unit's key tile after j (nkv_max(): none)
+        if (!(DF && diag_first)) return unext(j + 1);
+        if (j == nkv1 - 1) return nkv1 > 1 ? 0 : nkv1;
+        return j + 1 < nkv1 - 1 ? j + 1 : nkv1;
+    }
+    template <bool DF>
+    __device__ __forceinline__ int ulast(int t) const {  // Q_t's last key tile in sweep order
+        return (t == 1 && DF && diag_first) ? (nkv1 > 1 ? nkv1 - 2 : 0) : (t ? ts1.last() : ts0.last());
+    }
 };
 
 // The unit of rank r.  Sets: also build the tile sets (the epilogue needs only the
@@ -185,6 +206,7 @@ __device__ __forceinline__ bool fwd_unit(const FwdParams &p, int r, FwdUnit &u, 
     const int r1 = u.m0 + 128;
     u.nkv0 = p.causal ? min(nkv_all, u.m0 / 128 + 1) : nkv_all;
     u.nkv1 = (NT == 1 || r1 >= u.len) ? 0 : (p.causal ? min(nkv_all, r1 / 128 + 1) : nkv_all);
+    u.diag_first = !SP && p.causal && u.nkv1 == u.nkv0 + 1;
     if constexpr (Sets) {
         if (bits != nullptr) {
             u.ts0 = TileSet{*bits, 0, u.nkv0, SP};
@@ -227,6 +249,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // publishes {rank, Q0's key-tile bits} to the other roles through a 4-entry ring (so
     // only the producer reads the mask); n_ranks ends the walk.
     constexpr bool kDyn = DYN;
+    constexpr bool kDiagFirst = D == 64;  // see FwdUnit::ufirst
     volatile uint64_t *unit_ring = reinterpret_cast<volatile uint64_t *>(tmem_holder + 2);  // 8-byte aligned
     uint64_t unit_bits = 0;  // key-tile bits of the unit of the role's last rank (dynamic deal)
     auto claim_rank = [&](int k) -> int {  // producer
@@ -315,7 +338,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint8_t *keep = p.g.key_keep ? p.g.key_keep + p.g.keep_base(u.b, u.start) : nullptr;
                 // the key tiles either query tile attends (with a tile mask, NT = 1: those of
                 // the CTA's one tile)
-                for (int j = u.unext(0); j < nkv_max && ok; j = u.unext(j + 1)) {
+                for (int j = u.ufirst<kDiagFirst>(); j < nkv_max && ok; j = u.uafter<kDiagFirst>(j)) {
                     if (keep != nullptr) {
                         prefetch_l1(keep + 128 * j);
                         prefetch_l1(keep + 128 * j + 127);
@@ -393,7 +416,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             FOR_EACH_UNIT(u, consumer_rank) {
                 if (!ok) break;
                 const int hi = u.nkv_max();
-                int j = u.unext(0);  // the unit's key tiles are j, unext(j + 1), ... (< hi)
+                int j = u.ufirst<kDiagFirst>();  // the unit's key tiles are j, uafter(j), ... (< hi)
                 if (j >= hi) continue;  // no tile pair to compute (tile mask)
                 int pos = base;         // ring position of K_j (V_j follows it)
                 ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
@@ -405,10 +428,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int t = 0; t < 2; ++t)
                     if (u.live(t, j)) issue_S(t, pos);
                 tc_commit(bar(C::kBarEmpty + pos % C::kStages));
-                int nxt = u.unext(j + 1);
+                int nxt = u.uafter<kDiagFirst>(j);
                 if (nxt >= hi) tc_commit(bar(C::kBarQEmpty));
                 bool started[2] = {false, false};
-                const int last[2] = {u.ts0.last(), u.ts1.last()};
+                const int last[2] = {u.ulast<kDiagFirst>(0), u.ulast<kDiagFirst>(1)};
                 while (ok) {
                     ok = wait_phase(bar(C::kBarFull + (pos + 1) % C::kStages), ((pos + 1) / C::kStages) & 1, p.ctl,
                                     abort_flag);
@@ -441,7 +464,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     pos += 2;
                     if (nxt >= hi) break;
                     j = nxt;
-                    nxt = u.unext(j + 1);
+                    nxt = u.uafter<kDiagFirst>(j);
                     if (nxt >= hi) tc_commit(bar(C::kBarQEmpty));  // the S products just issued were the unit's last
                 }
                 if (!ok) break;
@@ -474,7 +497,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float m_used = -INFINITY, l = 0.f;
         const TileSet ts = t ? u.ts1 : u.ts0;  // the key tiles this tile attends
         bool first_step = true;
-        for (int j = ts.next(0); j < ts.hi; j = ts.next(j + 1), ++gs) {
+        // (Q1 with its diagonal tile first: see FwdUnit::ufirst)
+        const bool df = kDiagFirst && t == 1 && u.diag_first;
+        for (int j = df ? ts.hi - 1 : ts.next(0); j < ts.hi;
+             j = df ? (j == ts.hi - 1 ? (ts.hi > 1 ? 0 : ts.hi) : (j + 1 < ts.hi - 1 ? j + 1 : ts.hi)) : ts.next(j + 1),
+             ++gs) {
             const int kbase = j * 128;
             ok = wait_phase(bar(C::kBarS + t), gs & 1, p.ctl, abort_flag);
             if (!ok) break;
