@@ -42,8 +42,12 @@
  *   lse = -inf (never NaN), as the _safe_softmax discussion of the same page
  *   asks; its gradients are 0 and it contributes nothing to dK/dV.
  * - Ownership: every pointer is caller-owned DEVICE memory (except where noted);
- *   the library allocates nothing per call and keeps no per-call state, so calls
- *   on different streams are independent.  Base pointers must be 16-byte aligned.
+ *   the library allocates nothing per call, so calls on different streams are
+ *   independent.  (The kernels that claim their work units at run time -- tile
+ *   masks, packed sequences, very large backward problems -- take one of 1,024
+ *   library-owned counter pairs per launch, round-robin, and return it to zero when
+ *   they finish; a device runs at most 128 kernels at once.)  Base pointers must
+ *   be 16-byte aligned.
  * - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
  *   Every compute call is asynchronous on that stream.
  * - Errors: a non-OK code returned from a call means nothing was launched
