@@ -51,6 +51,13 @@
 // K_j once its last dQ is, and the following unit's K/V tiles are prefetched into L2
 // meanwhile.
 //
+// Units are dealt to the CTAs heaviest first in a snake order (SCHED 0), or -- with a
+// tile mask, whose units' costs are uneven -- claimed at run time from a global
+// counter by the loader, one unit ahead, and published with the unit's query-tile
+// bits to the other roles through a shared-memory ring (SCHED 1); when the slices'
+// Q, dO and dQ far exceed the L2 cache, the claimed ranks also walk the slices in
+// bands that fit it (SCHED 2, rank_to_unit).
+//
 // Every wait is bounded (see attn_common.cuh); an expired wait stops every role,
 // drains the copies in flight and returns with ATTN_ERR_TIMEOUT in the status word.
 #include <cuda_bf16.h>

@@ -34,6 +34,12 @@
 // a snake order.  Every barrier counts phases across units and the key/value ring
 // runs on, so the next unit's Q tiles load as soon as the current unit's last
 // S products are done and its first S products overlap the current epilogue.
+// With a tile mask or packed sequences (units of uneven cost) the CTAs instead
+// claim the units at run time (DYN: a global counter; the producer publishes each
+// claimed unit to the other roles through a small shared-memory ring), in bands of
+// slices whose K/V fit the L2 cache when all of it would not (rank_to_unit).  At
+// d = 64, causal Q1's extra diagonal key tile is swept first, so that both tiles
+// end a unit on the same step (FwdUnit::ufirst).
 //
 // Exponentials are base 2: p = 2^(s * scale * log2(e) - m).  The running max is
 // only moved when a row's new max exceeds the one in use by more than 8 (log2
