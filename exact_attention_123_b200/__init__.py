@@ -11,7 +11,12 @@ The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen
 ``attn_fwd_fp8_varlen``,
 ``attn_bwd_workspace_bytes``, ``attn_bwd_deterministic_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
-``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``, ``attn_debug_force_band``.
+``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``, ``attn_debug_force_band``,
+``attn_debug_checks``, ``attn_debug_corrupt_tag``.
+
+With the environment variable ``LIBATTN_DEBUG=1`` at import, the binding loads
+``libattn_debug.so`` instead: the same kernels with pipeline consistency checks
+(``attn_debug_checks``); ``use_debug_library`` switches between the two at run time.
 """
 from __future__ import annotations
 
@@ -24,6 +29,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libattn_debug.so")
 
 ATTN_OK = 0
 ATTN_ERR_INVALID_ARG = 1
@@ -32,8 +38,11 @@ ATTN_ERR_MISALIGNED = 3
 ATTN_ERR_WORKSPACE = 4
 ATTN_ERR_CUDA = 5
 ATTN_ERR_TIMEOUT = 6
+ATTN_ERR_DEBUG_CHECK = 7
 
 _lib = None
+_debug = os.environ.get("LIBATTN_DEBUG", "0") not in ("", "0")
+_loaded = {}
 
 
 class AttnError(RuntimeError):
@@ -42,15 +51,31 @@ class AttnError(RuntimeError):
         super().__init__(f"{where}: libattn status {code}: {attn_strerror(code)}")
 
 
+def use_debug_library(debug: bool) -> bool:
+    """Route later calls to libattn_debug.so (True) or libattn.so (False); returns the
+    previous choice.  The two libraries keep separate device state (status word,
+    hooks), so a status is read from the library that ran the kernels."""
+    global _lib, _debug
+    prev = _debug
+    _debug = bool(debug)
+    _lib = None
+    return prev
+
+
 def lib() -> ctypes.CDLL:
-    """Load libattn.so from the package directory (built by ``build.py``)."""
+    """Load libattn.so (or libattn_debug.so, see ``use_debug_library``) from the
+    package directory (built by ``build.py``)."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"libattn.so not found at {LIB_PATH}; build it with "
+    path = DEBUG_LIB_PATH if _debug else LIB_PATH
+    if path in _loaded:
+        _lib = _loaded[path]
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{os.path.basename(path)} not found at {path}; build it with "
                            "`python -m exact_attention_123_b200.build` (no fallback exists)")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
     L.attn_fwd_masked.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp, vp]
@@ -78,13 +103,17 @@ def lib() -> ctypes.CDLL:
     L.attn_set_wait_limit_ms.argtypes = [i]
     L.attn_debug_skip_load.argtypes = [i]
     L.attn_debug_force_band.argtypes = [i]
+    L.attn_debug_checks.argtypes = []
+    L.attn_debug_corrupt_tag.argtypes = [i]
     L.attn_debug_ex2_poly.argtypes = [vp, vp, ctypes.c_longlong, vp]
     for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_deterministic",
                  "attn_bwd_varlen", "attn_bwd_phase",
                  "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked",
                  "attn_fwd_fp8_varlen", "attn_status", "attn_set_wait_limit_ms",
-                 "attn_debug_skip_load", "attn_debug_ex2_poly", "attn_debug_force_band"):
+                 "attn_debug_skip_load", "attn_debug_ex2_poly", "attn_debug_force_band", "attn_debug_checks",
+                 "attn_debug_corrupt_tag"):
         getattr(L, name).restype = i
+    _loaded[path] = L
     _lib = L
     return L
 
@@ -424,6 +453,17 @@ def attn_debug_force_band(slices: int) -> int:
     """Test hook: force bands of `slices` slices in the banded unit order (0: automatic).
     Returns the previous value."""
     return int(lib().attn_debug_force_band(int(slices)))
+
+
+def attn_debug_checks() -> bool:
+    """True when the loaded library is the debug build (pipeline consistency checks)."""
+    return bool(lib().attn_debug_checks())
+
+
+def attn_debug_corrupt_tag(fill_index: int) -> int:
+    """Test hook (debug library): the forward producer writes a wrong check tag for ring
+    fill `fill_index` of each CTA (-1: off).  Returns the previous value."""
+    return int(lib().attn_debug_corrupt_tag(int(fill_index)))
 
 
 def attn_debug_ex2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:

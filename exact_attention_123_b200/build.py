@@ -14,6 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn.so")
+# the same kernels with pipeline consistency checks (LIBATTN_DEBUG=1; see attn_debug_checks)
+LIB_DEBUG = os.path.join(HERE, "libattn_debug.so")
 SOURCES = ["attn_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "attn_bwd_fused_sm100.cu", "attn_noalloc.cu"]
 HEADERS = ["sm100_ptx.cuh", "attn_common.cuh", "attn_launch.h", "../../include/libattn.h"]
 
@@ -25,26 +27,33 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Builds libattn.so and (debug=True) libattn_debug.so, each only if stale or
+    forced, the two compilations side by side.  Returns the release library's path."""
     flags = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
              "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
              "-shared", "-cudart", "static"]
     if verbose:
         flags += ["-Xptxas", "-v"]
     srcs = [os.path.join(CSRC, f) for f in SOURCES]
-    tmp = LIB + ".tmp"
-    subprocess.run([nvcc()] + flags + srcs + ["-o", tmp], check=True)
-    os.replace(tmp, LIB)
+    jobs = []
+    for lib, extra in ((LIB, []), (LIB_DEBUG, ["-DLIBATTN_DEBUG=1"])):
+        if (lib == LIB_DEBUG and not debug) or not (force or _stale(lib)):
+            continue
+        jobs.append((lib, subprocess.Popen([nvcc()] + flags + extra + srcs + ["-o", lib + ".tmp"])))
+    failed = [lib for lib, proc in jobs if proc.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(os.path.basename(f) for f in failed)})")
+    for lib, _ in jobs:
+        os.replace(lib + ".tmp", lib)
     return LIB
 
 

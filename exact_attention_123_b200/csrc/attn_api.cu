@@ -36,6 +36,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
 
 std::atomic<int> g_wait_limit_ms{4000};
 std::atomic<int> g_skip_load{-1};
+std::atomic<int> g_bad_tag{-1};
 std::atomic<int> g_force_band{0};  // test hook: slices per band forced (0: automatic)
 
 struct DeviceState {
@@ -165,6 +166,7 @@ attn::SyncCtl ctl_of(DeviceState *ds) {
     c.status = ds->status;
     c.wait_limit_ns = static_cast<unsigned long long>(g_wait_limit_ms.load()) * 1000000ull;
     c.inject_skip_load = g_skip_load.load();
+    c.inject_bad_tag = g_bad_tag.load();
     return c;
 }
 
@@ -455,6 +457,7 @@ const char *attn_strerror(int code) {
         case ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
         case ATTN_ERR_CUDA: return "a CUDA call or kernel launch failed";
         case ATTN_ERR_TIMEOUT: return "a device-side pipeline wait exceeded its time limit";
+        case ATTN_ERR_DEBUG_CHECK: return "a pipeline consistency check of the debug library failed";
         default: return "unknown status code";
     }
 }
@@ -481,5 +484,9 @@ int attn_debug_skip_load(int load_index) {
 }
 
 int attn_debug_force_band(int slices) { return g_force_band.exchange(slices > 0 ? slices : 0); }
+
+int attn_debug_checks(void) { return attn::kDebugChecks ? 1 : 0; }
+
+int attn_debug_corrupt_tag(int fill_index) { return g_bad_tag.exchange(fill_index < 0 ? -1 : fill_index); }
 
 }  // extern "C"

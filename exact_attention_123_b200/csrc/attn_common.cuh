@@ -8,11 +8,20 @@
 
 #include "sm100_ptx.cuh"
 
+// LIBATTN_DEBUG=1 builds the debug library (libattn_debug.so): the same kernels with
+// pipeline consistency checks that record ATTN_ERR_DEBUG_CHECK in the status word and
+// stop the CTA the way an expired wait does (never a trap or an assert).
+#ifndef LIBATTN_DEBUG
+#define LIBATTN_DEBUG 0
+#endif
+
 namespace attn {
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusUnsupported = 2;  // ATTN_ERR_UNSUPPORTED (a launch that cannot run as configured)
 constexpr int kStatusTimeout = 6;      // ATTN_ERR_TIMEOUT
+constexpr int kStatusDebugCheck = 7;   // ATTN_ERR_DEBUG_CHECK (debug library only)
+constexpr bool kDebugChecks = LIBATTN_DEBUG != 0;
 
 // Geometry of one (sequence, head) slice, common to dense and packed layouts.
 // A tensor element (row r, column c) of slice (b, h) sits at
@@ -132,6 +141,7 @@ struct SyncCtl {
     int *status;             // device status word (first error wins)
     unsigned long long wait_limit_ns;
     int inject_skip_load;    // test hook: index of a pipeline load to skip, or -1
+    int inject_bad_tag;      // test hook (debug library): ring fill whose check tag is written wrong, or -1
 };
 
 // Record an error once and raise the CTA-wide abort flag.
@@ -141,15 +151,31 @@ __device__ __forceinline__ void raise_abort(const SyncCtl &ctl, volatile int *ab
     __threadfence_block();
 }
 
+// Debug library: a waiter that has just seen phase k of `bar` complete must find phase
+// k+1 still open.  Every barrier here is built so that its next phase needs an action
+// that follows this wait (the waiter's own arrive, or a release it gates), so a
+// completed k+1 means a producer ran two phases ahead of a consumer: the parity
+// protocol can no longer tell the phases apart.  Release library: always true.
+__device__ __forceinline__ bool phase_consistent(uint32_t bar, uint32_t parity, const SyncCtl &ctl,
+                                                 volatile int *abort_flag) {
+    if constexpr (kDebugChecks) {
+        if (mbar_test_wait(bar, parity ^ 1u)) {
+            raise_abort(ctl, abort_flag, kStatusDebugCheck);
+            return false;
+        }
+    }
+    return true;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false (and raises the abort flag on
 // expiry) if the wait gave up, either because the limit passed or because another
 // role of the CTA already aborted.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const SyncCtl &ctl,
                                            volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return phase_consistent(bar, parity, ctl, abort_flag);
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait(bar, parity)) return phase_consistent(bar, parity, ctl, abort_flag);
         if ((it & 15u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > ctl.wait_limit_ns) {

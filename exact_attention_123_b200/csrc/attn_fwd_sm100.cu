@@ -127,7 +127,9 @@ struct FwdCfg {
     static constexpr int kOffBar = kOffStage + 4 * NT * 2048;
     // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
     // ({rank, key-tile bits}, 16 bytes each)
-    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 96;
+    // debug library, after the ring: a check tag per K/V slot and the roles' final counts
+    static constexpr int kDebugBytes = kDebugChecks ? 8 * kStages + 32 : 0;
+    static constexpr int kSmemBytes = 1024 + kOffBar + kNumBars * 8 + 96 + kDebugBytes;
     static_assert(kTileBytes % 1024 == 0, "swizzled shared-memory tiles must be 1024-byte aligned");
     // 227 KB per CTA; two CTAs share an SM's 228 KB less 1 KB reserved per CTA
     static_assert(kSmemBytes <= (NT == 1 ? 115712 : 232448), "exceeds the per-CTA shared-memory limit");
@@ -277,6 +279,25 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return r;
     };
     auto static_rank = [&](int k) -> int { return k * G + ((k & 1) ? (G - 1 - cta) : cta); };
+    // Debug library: the producer tags each ring fill with {unit rank, key tile, fill
+    // number}, which the issuer checks against its own walk when the fill lands; at exit
+    // the roles' counts (units, fills, S phases per tile) must agree.
+    uint64_t *const dbg_tag = reinterpret_cast<uint64_t *>(sptr + C::kOffBar + C::kNumBars * 8 + 96);
+    uint32_t *const dbg_cnt = reinterpret_cast<uint32_t *>(dbg_tag + C::kStages);
+    auto fill_tag = [](int r, int j, int fill) -> uint64_t {
+        return (static_cast<uint64_t>(static_cast<uint32_t>(r)) << 32) |
+               (static_cast<uint64_t>(static_cast<uint32_t>(j) & 0xFFFFu) << 16) |
+               (static_cast<uint32_t>(fill) & 0xFFFFu);
+    };
+    auto tag_ok = [&](int r, int fill, int j) -> bool {  // issuer, after the fill's full barrier
+        if constexpr (kDebugChecks) {
+            if (dbg_tag[fill % C::kStages] != fill_tag(r, j, fill)) {
+                raise_abort(p.ctl, abort_flag, kStatusDebugCheck);
+                return false;
+            }
+        }
+        return true;
+    };
     // walks this CTA's units in order (RANK(k): the role's way to get its k-th rank;
     // the static deal's last round can hold ranks past the end); every role sees the
     // same ranks
@@ -306,6 +327,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
+        if constexpr (kDebugChecks)
+            for (int i = 0; i < 8; ++i) dbg_cnt[i] = 0;
         fence_mbar_init();
     }
     tc_fence_before();
@@ -357,6 +380,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             break;
                         }
                         if (idx == p.ctl.inject_skip_load) continue;  // test hook: this slot never fills
+                        if constexpr (kDebugChecks)  // (test hook: one fill's tag written wrong)
+                            dbg_tag[s] = fill_tag(r_, j, idx) ^ (idx == p.ctl.inject_bad_tag ? 1ull : 0ull);
                         mbar_arrive_expect_tx(bar(C::kBarFull + s), C::kTileBytes);
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x)
@@ -365,6 +390,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         n_issued = idx + 1;
                     }
                 }
+            }
+            if constexpr (kDebugChecks) {
+                dbg_cnt[0] = static_cast<uint32_t>(n_qload);
+                dbg_cnt[1] = static_cast<uint32_t>(idx);
             }
         }
     } else if (warp == C::kIssuerWarp) {
@@ -427,6 +456,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 int pos = base;         // ring position of K_j (V_j follows it)
                 ok = wait_phase(bar(C::kBarQ), n_u & 1, p.ctl, abort_flag);
                 if (ok) ok = wait_phase(bar(C::kBarFull + pos % C::kStages), (pos / C::kStages) & 1, p.ctl, abort_flag);
+                if (ok) ok = tag_ok(r_, pos, j);
                 if (!ok) break;
                 tc_fence_after();
                 // The unit's first S_t may overwrite S_t / P_t: PV_t of the previous unit
@@ -441,6 +471,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 while (ok) {
                     ok = wait_phase(bar(C::kBarFull + (pos + 1) % C::kStages), ((pos + 1) / C::kStages) & 1, p.ctl,
                                     abort_flag);
+                    if (ok) ok = tag_ok(r_, pos + 1, j);
                     if (!ok) break;
                     bool k_next = false;
                     for (int t = 0; t < 2 && ok; ++t) {
@@ -457,6 +488,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             if (!k_next) {
                                 ok = wait_phase(bar(C::kBarFull + (pos + 2) % C::kStages), ((pos + 2) / C::kStages) & 1,
                                                 p.ctl, abort_flag);
+                                if (ok) ok = tag_ok(r_, pos + 2, nxt);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_next = true;
@@ -476,6 +508,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (!ok) break;
                 base = pos;
                 ++n_u;
+            }
+            if constexpr (kDebugChecks) {
+                dbg_cnt[2] = static_cast<uint32_t>(n_u);
+                dbg_cnt[3] = static_cast<uint32_t>(base);
+                dbg_cnt[4] = static_cast<uint32_t>(gs[0]);
+                dbg_cnt[5] = static_cast<uint32_t>(gs[1]);
             }
             // Every MMA issued above must have finished before TMEM / smem go away.
             tc_commit(bar(C::kBarDone));
@@ -701,6 +739,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         }
         if (lane == 0) bulk_wait0();  // this warp's output stores are complete
+        if constexpr (kDebugChecks)
+            if (q4 == 0 && lane == 0) dbg_cnt[6 + t] = static_cast<uint32_t>(gs);
     }
 #undef FOR_EACH_UNIT
 
@@ -720,6 +760,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (warp == C::kIssuerWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if constexpr (kDebugChecks) {
+        // without an abort, every role walked the same units, fills and S phases
+        if (threadIdx.x == 0 && !*abort_flag) {
+            bool agree = dbg_cnt[0] == dbg_cnt[2] && dbg_cnt[1] == dbg_cnt[3] && dbg_cnt[4] == dbg_cnt[6];
+            if (NT == 2) agree = agree && dbg_cnt[5] == dbg_cnt[7];
+            if (!agree) atomicCAS(p.ctl.status, 0, kStatusDebugCheck);
+        }
     }
     if constexpr (kDyn) {
         // the last CTA to finish returns the counters to zero for the slot's next launch

@@ -78,7 +78,8 @@ typedef enum {
     ATTN_ERR_MISALIGNED = 3,  /* a base pointer is not 16-byte aligned             */
     ATTN_ERR_WORKSPACE = 4,   /* backward workspace missing or too small           */
     ATTN_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed       */
-    ATTN_ERR_TIMEOUT = 6      /* a device-side bounded wait expired (attn_status)  */
+    ATTN_ERR_TIMEOUT = 6,     /* a device-side bounded wait expired (attn_status)  */
+    ATTN_ERR_DEBUG_CHECK = 7  /* a consistency check of the debug library failed   */
 } attn_status_t;
 
 /*
@@ -306,8 +307,9 @@ ATTN_API int attn_bwd_noalloc(const void *q, const void *k, const void *v, const
  * Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait
  * expired since the last call, ATTN_ERR_UNSUPPORTED if a kernel found its shared
- * memory laid out in a way it cannot run with (and did nothing), or ATTN_ERR_CUDA
- * if synchronisation failed.
+ * memory laid out in a way it cannot run with (and did nothing),
+ * ATTN_ERR_DEBUG_CHECK if a pipeline consistency check of the debug library failed
+ * (see attn_debug_checks), or ATTN_ERR_CUDA if synchronisation failed.
  */
 ATTN_API int attn_status(void *stream);
 
@@ -358,6 +360,33 @@ ATTN_API int attn_debug_ex2_poly(const float *x, float *y, long long n, void *st
  * to the order of its fp32 additions).  Returns the previous value.
  */
 ATTN_API int attn_debug_force_band(int slices);
+
+/*
+ * 1 in the debug library (libattn_debug.so, built from the same sources with
+ * LIBATTN_DEBUG=1), 0 in the release library.  The debug library runs the same kernels
+ * with pipeline consistency checks; a failed check records ATTN_ERR_DEBUG_CHECK in the
+ * status word (attn_status) and stops the kernel the way an expired wait does, never
+ * with a trap or an assert.  The checks:
+ *   - every bounded mbarrier wait: once phase k of a barrier is seen complete, phase
+ *     k+1 must still be open (a producer two phases ahead of a consumer would make the
+ *     parity protocol misread the phase; every kernel);
+ *   - forward: each K/V ring fill carries a tag {unit rank, key tile, fill number}
+ *     written by the TMA producer, which the MMA issuer compares with its own walk when
+ *     the fill lands; at exit the producer, issuer and softmax warps must agree on the
+ *     units, fills and S phases they processed.
+ * Results are identical to the release library's.
+ */
+ATTN_API int attn_debug_checks(void);
+
+/*
+ * Test hook for the debug library's ring-tag check.  For later launches from this
+ * process, the forward's TMA producer in every CTA writes a wrong tag for its K/V ring
+ * fill number `fill_index` (counting the K and V tile loads of one CTA from 0); the
+ * issuer's check then fails, the kernel stops cleanly and attn_status() reports
+ * ATTN_ERR_DEBUG_CHECK.  No effect in the release library, which writes no tags.  -1
+ * (the default) disables it.  Returns the previous value.
+ */
+ATTN_API int attn_debug_corrupt_tag(int fill_index);
 
 #ifdef __cplusplus
 }

@@ -33,16 +33,32 @@ def test_header_declares_the_expected_entry_points():
         assert n in names
 
 
-def test_every_declared_symbol_is_exported(L):
-    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(ROOT, "exact_attention_123_b200", "libattn.so")],
-                         capture_output=True, text=True, check=True).stdout
+@pytest.mark.parametrize("name", ["libattn.so", "libattn_debug.so"])
+def test_every_declared_symbol_is_exported(L, name):
+    path = os.path.join(ROOT, "exact_attention_123_b200", name)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    handle = ctypes.CDLL(path)
     for n in declared_functions():
         assert n in exported, n
-        assert hasattr(L, n)
+        assert hasattr(handle, n)
     # nothing else of ours leaks out of the library
     ours = {e for e in exported if e.startswith("attn")}
     assert ours == set(declared_functions())
+
+
+def test_release_and_debug_libraries_identify_themselves(L):
+    import exact_attention_123_b200 as ea
+    lib_dir = os.path.join(ROOT, "exact_attention_123_b200")
+    assert ctypes.CDLL(os.path.join(lib_dir, "libattn.so")).attn_debug_checks() == 0
+    assert ctypes.CDLL(os.path.join(lib_dir, "libattn_debug.so")).attn_debug_checks() == 1
+    prev = ea.use_debug_library(True)
+    try:
+        assert ea.attn_debug_checks()
+        assert ea.attn_debug_corrupt_tag(5) == -1 and ea.attn_debug_corrupt_tag(-1) == 5  # host-side hook only
+    finally:
+        ea.use_debug_library(prev)
+    assert not ea.attn_debug_checks()
 
 
 def test_header_compiles_as_c(tmp_path):

@@ -92,15 +92,35 @@ def test_blocksparse_matches_oracle(ea, B, H, N, d, causal, density, seed, er, e
 @pytest.mark.parametrize("causal", [False, True])
 def test_full_mask_is_the_dense_path(ea, d, causal):
     # every pair kept: the block-sparse kernels do the dense kernels' arithmetic, so
-    # O, lse, dK and dV match bit for bit; dQ too up to the order in which the key
-    # tiles' fp32 contributions reach its accumulator (a few bf16 ulps at most)
-    inp = make_dense(2, 2, 520, d, seed=9100 + d, causal=causal, with_grad=True)
+    # O and lse match bit for bit where both sweep the key tiles in the same order, and
+    # dK, dV (from the same O and lse) bit for bit; dQ up to the order in which the key
+    # tiles' fp32 contributions reach its accumulator (a few bf16 ulps at most).  The
+    # one order difference: at d = 64 the dense causal forward sweeps the second query
+    # tile of each 256-row unit (rows 128-255 of it) from its diagonal key tile, where
+    # the running max moves at other tiles.  P is rounded to bf16 (relative error <= 2^-9)
+    # on that running max's scale before P V, so those rows' O may differ by twice that
+    # times sum_j P_j |v_j| / l <= max |v|, plus a bf16 rounding step of O; lse by at
+    # most twice the relative error of the exponentials (at d = 64 one column pair in
+    # eight comes from the FMA-pipe cubic, relative error <= 1.02e-4, whose arguments
+    # shift with the running max), plus float rounding.
+    N = 520
+    inp = make_dense(2, 2, N, d, seed=9100 + d, causal=causal, with_grad=True)
     q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
     bm = torch.ones((2, 5, 5), dtype=torch.uint8)
     o, lse, dq, dk, dv = _run(ea, inp, bm, causal)
     o2, lse2 = ea.attn_fwd(q, k, v, scale=inp.scale, causal=causal)
-    dq2, dk2, dv2 = ea.attn_bwd(q, k, v, o2, lse2, do, scale=inp.scale, causal=causal)
-    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    dq2, dk2, dv2 = ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=causal)
+    reordered = torch.zeros(N, dtype=torch.bool)
+    if d == 64 and causal:
+        for u0 in range(0, N, 256):
+            reordered[u0 + 128:u0 + 256] = True
+    same = ~reordered
+    assert torch.equal(o[:, :, same], o2[:, :, same]) and torch.equal(lse[:, :, same], lse2[:, :, same])
+    if reordered.any():
+        a, b = o[:, :, reordered].double(), o2[:, :, reordered].double()
+        vmax = inp.v.double().abs().max().item()
+        assert torch.all((a - b).abs() <= 2 ** -7 * b.abs() + 2 ** -8 * vmax)
+        assert torch.all((lse[:, :, reordered] - lse2[:, :, reordered]).abs() <= 2 * 1.02e-4 + 1e-5)
     assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
     a, b = dq.double(), dq2.double()
     assert torch.all((a - b).abs() <= 2 ** -6 * b.abs() + 1e-3)
