@@ -622,14 +622,20 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 int lim = p.causal ? key - qb : 0;  // columns c < lim are masked
                 if (!kvalid) lim = 64;
                 float pf[64];
+                const uint64_t c2x2 = f2_pack(c2, c2);
 #pragma unroll
                 for (int c4 = 0; c4 < 16; ++c4) {
                     const float4 l2 = vec[c4];
-                    const float l2v[4] = {l2.x, l2.y, l2.z, l2.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < 4; e += 2) {  // column pairs: scale and shift on the f32x2 pipe
                         const int c = c4 * 4 + e;
-                        pf[c] = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), c2, -l2v[e]));
+                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[c >> 5][c & 31]),
+                                                           __uint_as_float(sr[c >> 5][(c & 31) + 1])),
+                                                   c2x2, e ? f2_pack(-l2.z, -l2.w) : f2_pack(-l2.x, -l2.y));
+                        float x0, x1;
+                        f2_unpack(x2, x0, x1);
+                        pf[c] = ex2_approx(x0);
+                        pf[c + 1] = ex2_approx(x1);
                     }
                 }
                 if (lim > 0) {
