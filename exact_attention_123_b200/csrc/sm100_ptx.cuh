@@ -350,11 +350,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 
 // Two base-2 exponentials on the FMA pipe instead of the MUFU unit.  2^x = 2^j 2^f
 // with j = rint(x) and f = x - j in [-1/2, 1/2]; 2^f is the cubic
