@@ -120,7 +120,9 @@ struct FusedCfg {
     static constexpr int kNumBars = kBarSFull + 17;
     // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
     // ({rank, query-tile bits}, 16 bytes each)
-    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 80;  // from a 1024-byte-aligned base
+    // debug library, after the ring: a check tag per Q stage and the roles' final counts
+    static constexpr int kDebugBytes = kDebugChecks ? 8 * kStages + 32 : 0;
+    static constexpr int kSmemUsed = kOffBar + kNumBars * 8 + 80 + kDebugBytes;  // from a 1024-byte-aligned base
     static constexpr int kSmemMax = 232448;
     // The base of dynamic shared memory is expected to be 1024-byte aligned; the
     // kernel checks, and where the slack below cannot cover the misalignment it
@@ -231,6 +233,25 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         mbar_arrive(bar(C::kBarUFull + (k & 3)));
         return r;
     };
+    // Debug library: the loader tags each Q stage fill with {unit rank, query tile, pair
+    // number}, which the issuer checks against its own walk when the fill lands; at exit
+    // the loader, issuer, math and drain warps must agree on the units and pairs they did.
+    uint64_t *const dbg_tag = reinterpret_cast<uint64_t *>(sptr + C::kOffBar + C::kNumBars * 8 + 80);
+    uint32_t *const dbg_cnt = reinterpret_cast<uint32_t *>(dbg_tag + C::kStages);
+    auto fill_tag = [](int r, int i, int gi) -> uint64_t {
+        return (static_cast<uint64_t>(static_cast<uint32_t>(r)) << 32) |
+               (static_cast<uint64_t>(static_cast<uint32_t>(i) & 0xFFFFu) << 16) |
+               (static_cast<uint32_t>(gi) & 0xFFFFu);
+    };
+    auto tag_ok = [&](int r, int i, int gi) -> bool {  // issuer, after the fill's full barrier
+        if constexpr (kDebugChecks) {
+            if (dbg_tag[gi % C::kStages] != fill_tag(r, i, gi)) {
+                raise_abort(p.ctl, abort_flag, kStatusDebugCheck);
+                return false;
+            }
+        }
+        return true;
+    };
     auto consumer_rank = [&](int k) -> int {  // issuer, drain and math threads
         if constexpr (kDyn) {
             if (!wait_phase(bar(C::kBarUFull + (k & 3)), (k >> 2) & 1, p.ctl, abort_flag)) return T;
@@ -256,6 +277,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             mbar_init(bar(i), cnt);
         }
         *abort_flag = 0;
+        if constexpr (kDebugChecks)
+            for (int i = 0; i < 8; ++i) dbg_cnt[i] = 0;
         fence_mbar_init();
     }
     tc_fence_before();
@@ -367,6 +390,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     }
                     __syncwarp();
                     if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
+                        if constexpr (kDebugChecks)  // (test hook: one fill's tag written wrong)
+                            dbg_tag[st] = fill_tag(r, i, gi) ^ (gi == p.ctl.inject_bad_tag ? 1ull : 0ull);
                         mbar_arrive_expect_tx(bar(C::kBarQFull + st), C::kTile);
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x)
@@ -388,6 +413,11 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     }
                     ++n_do;
                 }
+            }
+            if (kDebugChecks && lane == 0) {
+                dbg_cnt[0] = static_cast<uint32_t>(n_kv);
+                dbg_cnt[1] = static_cast<uint32_t>(n_q);
+                dbg_cnt[2] = static_cast<uint32_t>(n_do);
             }
         } else if (warp == 13) {
             // ------------------------------------------------------------ MMA issuer
@@ -432,6 +462,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     if (!tile_at(r, t, ubits) || t.nq == 0) continue;
                     ok = wait_phase(bar(C::kBarKFull), n_t & 1, p.ctl, abort_flag);
                     if (ok) ok = wait_q(gbase);
+                    int dbg_i = t.qs.next(t.i0);  // (debug library: the query tile of pair gi)
+                    if (ok) ok = tag_ok(r, dbg_i, gbase);
                     if (!ok) break;
                     tc_fence_after();
                     // S^T's columns are free: the previous unit's last dV, which read P^T from
@@ -465,6 +497,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                         // (the math warps keep their P in registers for dS).
                         if (more) {
                             ok = wait_q(gi + 1);
+                            if constexpr (kDebugChecks) dbg_i = t.qs.next(dbg_i + 1);
+                            if (ok) ok = tag_ok(r, dbg_i, gi + 1);
                             if (!ok) break;
                             tc_fence_after();
                             issue_s(gi + 1);
@@ -504,6 +538,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     tc_commit(bar(C::kBarKdv));
                     gbase += t.nq;
                     ++n_t;
+                }
+                if constexpr (kDebugChecks) {
+                    dbg_cnt[3] = static_cast<uint32_t>(n_t);
+                    dbg_cnt[4] = static_cast<uint32_t>(gbase);
                 }
                 // Every MMA issued above must have finished before TMEM / smem go away.
                 tc_commit(bar(C::kBarDone));
@@ -568,6 +606,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             if (!ok) break;
             gbase += t.nq;
         }
+        if (kDebugChecks && warp == 8 && lane == 0) dbg_cnt[7] = static_cast<uint32_t>(gbase);
         if (lane == 0) bulk_wait0();  // every reduce-add of this warp has landed
     } else {
         setmaxnreg_inc<C::kRegsMath>();
@@ -717,6 +756,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             gbase += t.nq;
             ++n_t;
         }
+        if (kDebugChecks && warp == 0 && lane == 0) {
+            dbg_cnt[5] = static_cast<uint32_t>(n_t);
+            dbg_cnt[6] = static_cast<uint32_t>(gbase);
+        }
     }
 
     __syncwarp();
@@ -737,6 +780,15 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if constexpr (kDebugChecks) {
+        // without an abort, every role walked the same units and pairs
+        if (threadIdx.x == 0 && !*abort_flag) {
+            const uint32_t *c = dbg_cnt;
+            const bool agree = c[0] == c[3] && c[3] == c[5] && c[1] == c[4] && c[2] == c[4] && c[4] == c[6] &&
+                               c[4] == c[7];
+            if (!agree) atomicCAS(p.ctl.status, 0, kStatusDebugCheck);
+        }
     }
     if constexpr (kDyn) {
         // the last CTA to finish returns the counters to zero for the pair's next launch

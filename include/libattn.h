@@ -373,7 +373,10 @@ ATTN_API int attn_debug_force_band(int slices);
  *   - forward: each K/V ring fill carries a tag {unit rank, key tile, fill number}
  *     written by the TMA producer, which the MMA issuer compares with its own walk when
  *     the fill lands; at exit the producer, issuer and softmax warps must agree on the
- *     units, fills and S phases they processed.
+ *     units, fills and S phases they processed;
+ *   - single-pass backward: each Q stage fill carries a tag {unit rank, query tile, pair
+ *     number} from the loader, checked by the issuer; at exit the loader, issuer, math
+ *     and dQ-drain warps must agree on the units and tile pairs they processed.
  * Results are identical to the release library's.
  */
 ATTN_API int attn_debug_checks(void);
@@ -381,9 +384,10 @@ ATTN_API int attn_debug_checks(void);
 /*
  * Test hook for the debug library's ring-tag check.  For later launches from this
  * process, the forward's TMA producer in every CTA writes a wrong tag for its K/V ring
- * fill number `fill_index` (counting the K and V tile loads of one CTA from 0); the
- * issuer's check then fails, the kernel stops cleanly and attn_status() reports
- * ATTN_ERR_DEBUG_CHECK.  No effect in the release library, which writes no tags.  -1
+ * fill number `fill_index` (counting the K and V tile loads of one CTA from 0), and the
+ * single-pass backward's loader for its Q stage fill number `fill_index` (the CTA's
+ * tile pairs, from 0); the issuer's check then fails, the kernel stops cleanly and
+ * attn_status() reports ATTN_ERR_DEBUG_CHECK.  No effect in the release library, which writes no tags.  -1
  * (the default) disables it.  Returns the previous value.
  */
 ATTN_API int attn_debug_corrupt_tag(int fill_index);

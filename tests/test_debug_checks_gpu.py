@@ -3,7 +3,9 @@
 Its pipeline consistency checks (every bounded mbarrier wait finds the next phase of
 its barrier still open; the forward's K/V ring fills carry {unit rank, key tile, fill
 number} tags that the MMA issuer checks; at exit the forward's roles agree on the units,
-fills and S phases they processed) must pass on every entry point and leave the results
+fills and S phases they processed; the single-pass backward's Q stage fills carry {unit
+rank, query tile, pair number} tags and its loader, issuer, math and drain warps agree
+on their units and pairs) must pass on every entry point and leave the results
 unchanged: each call is made with the release library and with the debug library on
 the same inputs, and the outputs must agree bit for bit (dQ of the single-pass backward
 up to the order in which the key tiles' fp32 contributions reach its accumulator, as in
@@ -150,5 +152,27 @@ def test_corrupted_ring_tag_is_reported_then_clean(ea):
             ea.attn_debug_corrupt_tag(-1)
         same(ref, ea.attn_fwd(q, k, v, scale=inp.scale, causal=False))
         assert ea.attn_status() == ea.ATTN_OK
+    finally:
+        ea.use_debug_library(False)
+
+
+def test_corrupted_backward_tag_is_reported_then_clean(ea):
+    inp = make_dense(1, 2, 1024, 128, seed=9991, causal=True, with_grad=True)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+    o, lse = ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
+    ref = ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True)
+    assert ea.attn_status() == ea.ATTN_OK
+    ea.use_debug_library(True)
+    try:
+        ea.attn_debug_corrupt_tag(2)  # the third tile pair of every CTA
+        try:
+            ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True)
+            assert ea.attn_status() == ea.ATTN_ERR_DEBUG_CHECK
+        finally:
+            ea.attn_debug_corrupt_tag(-1)
+        got = ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True)
+        assert ea.attn_status() == ea.ATTN_OK
+        dq_close(got[0], ref[0])
+        same(got[1:], ref[1:])
     finally:
         ea.use_debug_library(False)
