@@ -286,6 +286,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     int n_q = 0, n_do = 0, n_kv = 0;  // loader: Q, dO and K/V loads started (for the abort drain)
+    int n_v = 0;                      // loader: V loads started (V goes before K: n_v >= n_kv)
 
     if (warp >= 12) {
         setmaxnreg_dec<C::kRegsCtl>();
@@ -322,48 +323,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 if (!tile_at(r, t, ubits) || t.nq == 0) continue;  // (nq == 0: the math warps write zeros)
                 const int row0 = p.g.tma_row0(t.start), slab = p.g.tma_slab(t.b, t.h);
                 const long long lrow0 = p.g.base(t.b, t.h, t.start, 1), lrs = p.g.row_stride(1);
-                // V_j once the previous unit's last dP^T is done, K_j once its last dQ is
-#pragma unroll
-                for (int kv = 1; kv >= 0; --kv) {
-                    const int full = kv ? C::kBarVFull : C::kBarKFull, empty = kv ? C::kBarVEmpty : C::kBarKEmpty;
-                    ok = __all_sync(0xffffffffu, wait_phase(bar(empty), (n_kv & 1) ^ 1, p.ctl, abort_flag));
-                    if (!ok) break;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(bar(full), C::kTile);
-#pragma unroll
-                        for (int x = 0; x < C::kBoxes; ++x)
-                            tma_load_3d(sbase + (kv ? C::kOffV : C::kOffK) + x * 16384, kv ? &tm_v : &tm_k, bar(full),
-                                        x * 64, row0 + t.kv0, slab);
-                    }
-                }
-                if (!ok) break;
-                ++n_kv;
-                // the next unit's K and V tiles into L2 while this unit runs
-                if (kDyn && lane == 0) {
-                    Tile t2;
-                    if (r_next < T && tile_at(r_next, t2, &bits_next) && t2.nq > 0) {
-#pragma unroll
-                        for (int x = 0; x < C::kBoxes; ++x) {
-                            tma_prefetch_l2_3d(&tm_k, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
-                            tma_prefetch_l2_3d(&tm_v, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
-                        }
-                    }
-                }
-                if (!kDyn && lane == 0) {
-                    for (int k2 = k + 1;; ++k2) {
-                        const int r2 = rank_of(k2);
-                        if (r2 >= T) break;
-                        Tile t2;
-                        if (!tile_at(r2, t2) || t2.nq == 0) continue;
-#pragma unroll
-                        for (int x = 0; x < C::kBoxes; ++x) {
-                            tma_prefetch_l2_3d(&tm_k, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
-                            tma_prefetch_l2_3d(&tm_v, x * 64, p.g.tma_row0(t2.start) + t2.kv0, p.g.tma_slab(t2.b, t2.h));
-                        }
-                        break;
-                    }
-                }
-                for (int it = 0, i = t.qs.next(t.i0); it < t.nq; ++it, i = t.qs.next(i + 1)) {
+                // Q_i, dO_i and the row terms of the unit's pair with query tile i
+                auto load_pair = [&](int i) -> bool {
                     const int gi = n_q, st = gi % C::kStages;
                     const int q0 = i * 128;
                     // the step's row terms, read before waiting for the stage so that their
@@ -379,9 +340,9 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                             dd[u] = p.dvec[lrow0 + q * lrs];
                         }
                     }
-                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
-                                                            p.ctl, abort_flag));
-                    if (!ok) break;
+                    if (!__all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
+                                                            p.ctl, abort_flag)))
+                        return false;
                     float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -401,9 +362,9 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     ++n_q;
                     // dO_i once dV of the step that last used its buffer is done
                     const int db = gi % C::kDoStages;
-                    ok = __all_sync(0xffffffffu, wait_phase(bar(C::kBarDOEmpty + db), ((gi / C::kDoStages) & 1) ^ 1,
-                                                            p.ctl, abort_flag));
-                    if (!ok) break;
+                    if (!__all_sync(0xffffffffu, wait_phase(bar(C::kBarDOEmpty + db), ((gi / C::kDoStages) & 1) ^ 1,
+                                                            p.ctl, abort_flag)))
+                        return false;
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bar(C::kBarDOFull + db), C::kTile);
 #pragma unroll
@@ -412,6 +373,61 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                                         x * 64, row0 + q0, slab);
                     }
                     ++n_do;
+                    return true;
+                };
+                // K_j or V_j once the previous unit has released it
+                auto load_kv = [&](int kv) -> bool {
+                    const int full = kv ? C::kBarVFull : C::kBarKFull, empty = kv ? C::kBarVEmpty : C::kBarKEmpty;
+                    if (!__all_sync(0xffffffffu, wait_phase(bar(empty), (n_kv & 1) ^ 1, p.ctl, abort_flag))) return false;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(full), C::kTile);
+#pragma unroll
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            tma_load_3d(sbase + (kv ? C::kOffV : C::kOffK) + x * 16384, kv ? &tm_v : &tm_k, bar(full),
+                                        x * 64, row0 + t.kv0, slab);
+                    }
+                    if (kv) ++n_v;
+                    return true;
+                };
+                // In the order the previous unit releases the buffers: V_j after its last dP^T,
+                // the first Q_i and dO_i (their stages free up before its last products are
+                // done), K_j after its last dQ.
+                const int i_first = t.qs.next(t.i0);
+                ok = load_kv(1);
+                if (ok) ok = load_pair(i_first);
+                if (ok) ok = load_kv(0);
+                if (!ok) break;
+                ++n_kv;
+                // the next unit's K and V tiles, and its first Q and dO tiles, into L2 while
+                // this unit runs
+                auto prefetch_unit = [&](const Tile &t2) {
+                    const int r2 = p.g.tma_row0(t2.start), s2 = p.g.tma_slab(t2.b, t2.h);
+                    const int q2 = t2.qs.next(t2.i0) * 128;
+#pragma unroll
+                    for (int x = 0; x < C::kBoxes; ++x) {
+                        tma_prefetch_l2_3d(&tm_k, x * 64, r2 + t2.kv0, s2);
+                        tma_prefetch_l2_3d(&tm_v, x * 64, r2 + t2.kv0, s2);
+                        tma_prefetch_l2_3d(&tm_q, x * 64, r2 + q2, s2);
+                        tma_prefetch_l2_3d(&tm_do, x * 64, r2 + q2, s2);
+                    }
+                };
+                if (kDyn && lane == 0) {
+                    Tile t2;
+                    if (r_next < T && tile_at(r_next, t2, &bits_next) && t2.nq > 0) prefetch_unit(t2);
+                }
+                if (!kDyn && lane == 0) {
+                    for (int k2 = k + 1;; ++k2) {
+                        const int r2 = rank_of(k2);
+                        if (r2 >= T) break;
+                        Tile t2;
+                        if (!tile_at(r2, t2) || t2.nq == 0) continue;
+                        prefetch_unit(t2);
+                        break;
+                    }
+                }
+                for (int it = 1, i = t.qs.next(i_first + 1); it < t.nq; ++it, i = t.qs.next(i + 1)) {
+                    ok = load_pair(i);
+                    if (!ok) break;
                 }
             }
             if (kDebugChecks && lane == 0) {
@@ -767,10 +783,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     __syncthreads();
     if (warp == 12 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        if (n_kv > 0) {
-            drain_phase(bar(C::kBarKFull), (n_kv - 1) & 1, p.ctl, abort_flag);
-            drain_phase(bar(C::kBarVFull), (n_kv - 1) & 1, p.ctl, abort_flag);
-        }
+        if (n_kv > 0) drain_phase(bar(C::kBarKFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        if (n_v > 0) drain_phase(bar(C::kBarVFull), (n_v - 1) & 1, p.ctl, abort_flag);
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
             if (gi != p.ctl.inject_skip_load)
                 drain_phase(bar(C::kBarQFull + gi % C::kStages), (gi / C::kStages) & 1, p.ctl, abort_flag);
