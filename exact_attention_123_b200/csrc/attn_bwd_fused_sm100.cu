@@ -47,9 +47,10 @@
 // (32 KB: two 4 KB boxes per warp, reused as soon as the TMA has read them).
 // The next dS is written only after dP^T_{i+1} is complete, which (tensor-core
 // operations completing in issue order) implies dQ_i and dK_i, the products that
-// read dS, are done.  At a unit's end V_j is reloaded once its last dP^T is done and
-// K_j once its last dQ is, and the following unit's K/V tiles are prefetched into L2
-// meanwhile.
+// read dS, are done.  At a unit's end the loader issues the next unit's loads in the
+// order their buffers free up: V_j once the last dP^T is done, the first Q_i and dO_i,
+// then K_j once the last dQ is; that unit's K/V tiles and first Q_i and dO_i have been
+// prefetched into L2 meanwhile.
 //
 // Units are dealt to the CTAs heaviest first in a snake order (SCHED 0), or -- with a
 // tile mask, whose units' costs are uneven -- claimed at run time from a global
