@@ -486,6 +486,19 @@ def run_ours(args):
     st = ea.attn_status(stream)
     if st != ea.ATTN_OK:
         raise RuntimeError(f"end-to-end steps reported status {st}")
+    # The pipeline's longest stream alone: the steps' host-to-device copies back to back, no
+    # kernels and no copies out (which run alongside and only slow them) -- a lower bound on
+    # the end-to-end step that the host link sets.
+    torch.cuda.synchronize(dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(s_in)
+    with torch.cuda.stream(s_in):
+        for s in range(e2e_n):
+            for n in ("q", "k", "v", "do"):
+                bufs[s % 2][n].copy_(pin[n], non_blocking=True)
+    c1.record(s_in)
+    torch.cuda.synchronize(dev)
+    copy_ms = max_over_ranks(c0.elapsed_time(c1), device=dev)
 
     peaks, peak_src = measured_peaks()
     peak = float(peaks["bf16_tflops"])
@@ -607,7 +620,11 @@ def run_ours(args):
                                      "(no MEASURED_PEAKS.json beside bench.py)")},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_n, "pipeline": "copy in, kernels, copy out on three streams over two buffer sets"},
+                "steps": e2e_n, "pipeline": "copy in, kernels, copy out on three streams over two buffer sets",
+                "ms_per_step": e2e_ms / e2e_n,
+                # the host-to-device copies alone, back to back: the host link's bound on a step
+                "h2d_only_ms_per_step": copy_ms / e2e_n,
+                "frac_of_copy_bound": (copy_ms / e2e_ms) if e2e_ms > 0 else None},
         "gpu_launches": n_k * args.steps,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
@@ -714,7 +731,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--cpu-heads", type=int, default=32,
                     help="(b,h) slices in the CPU-oracle baseline sample (32 = the whole workload, about 14 s on 16 cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
