@@ -88,7 +88,7 @@ def test_sharded_ranks_reproduce_the_whole_tensor(world):
         assert torch.equal(torch.cat([p_[i] for p_ in parts], dim=1), full)
     assert ea.attn_status() == ea.ATTN_OK
     # each rank's shard, as the fast backward computes it, against the float64 oracle on
-    # that rank's heads (the benchmark spec bands)
+    # that rank's heads (the parity tests' bands)
     ro, rl = oracle.fwd(inp.q, inp.k, inp.v, inp.scale, True)
     rg = oracle.bwd(inp.q, inp.k, inp.v, inp.do, inp.scale, True)
     for r in range(world):
