@@ -103,7 +103,7 @@ struct FusedCfg {
     static constexpr int kBarKEmpty = 1;                       // K_j no longer read (the unit's last dQ done)
     static constexpr int kBarVFull = 2;
     static constexpr int kBarVEmpty = 3;                       // V_j no longer read (the unit's last dP^T done)
-    static constexpr int kBarQFull = 4;                        // + st
+    static constexpr int kBarQFull = 4;                        // + st: Q_i landed and its row terms stored (2 arrivals)
     static constexpr int kBarQEmpty = kBarQFull + kStages;     // + st
     static constexpr int kBarDOFull = kBarQEmpty + kStages;    // + buffer
     static constexpr int kBarDOEmpty = kBarDOFull + kDoStages; // + buffer
@@ -274,6 +274,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             uint32_t cnt = 1;
             if (i == C::kBarPFull || i == C::kBarDSFull || i == C::kBarAccFree) cnt = 256;
             if (i == C::kBarDQFree) cnt = 128;
+            if (i >= C::kBarQFull && i < C::kBarQFull + C::kStages) cnt = 2;  // the Q copy, then the row terms
             if (i >= C::kBarUEmpty && i < C::kBarUEmpty + 4) cnt = 1 + 128 + 256;  // issuer, drain, math
             mbar_init(bar(i), cnt);
         }
@@ -344,14 +345,10 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     if (!__all_sync(0xffffffffu, wait_phase(bar(C::kBarQEmpty + st), ((gi / C::kStages) & 1) ^ 1,
                                                             p.ctl, abort_flag)))
                         return false;
-                    float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        vec[u * 32 + lane] = l2[u];
-                        vec[128 + u * 32 + lane] = dd[u];
-                    }
-                    __syncwarp();
-                    if (lane == 0 && gi != p.ctl.inject_skip_load) {  // (test hook: this stage never fills)
+                    // Q_i's copy first, then the row terms once their loads are in: the stage's
+                    // full barrier takes both arrivals, so the copy does not wait for them
+                    const bool fill = gi != p.ctl.inject_skip_load;  // (test hook: this stage never fills)
+                    if (lane == 0 && fill) {
                         if constexpr (kDebugChecks)  // (test hook: one fill's tag written wrong)
                             dbg_tag[st] = fill_tag(r, i, gi) ^ (gi == p.ctl.inject_bad_tag ? 1ull : 0ull);
                         mbar_arrive_expect_tx(bar(C::kBarQFull + st), C::kTile);
@@ -361,6 +358,14 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                                         x * 64, row0 + q0, slab);
                     }
                     ++n_q;
+                    float *vec = reinterpret_cast<float *>(sptr + C::kOffVec + st * 1024);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        vec[u * 32 + lane] = l2[u];
+                        vec[128 + u * 32 + lane] = dd[u];
+                    }
+                    __syncwarp();
+                    if (lane == 0 && fill) mbar_arrive(bar(C::kBarQFull + st));
                     // dO_i once dV of the step that last used its buffer is done
                     const int db = gi % C::kDoStages;
                     if (!__all_sync(0xffffffffu, wait_phase(bar(C::kBarDOEmpty + db), ((gi / C::kDoStages) & 1) ^ 1,
@@ -410,6 +415,14 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                         tma_prefetch_l2_3d(&tm_v, x * 64, r2 + t2.kv0, s2);
                         tma_prefetch_l2_3d(&tm_q, x * 64, r2 + q2, s2);
                         tma_prefetch_l2_3d(&tm_do, x * 64, r2 + q2, s2);
+                    }
+                    if (!p.g.varlen) {  // and its first row terms (dense: 128 consecutive floats each)
+                        const long long b2 = p.g.base(t2.b, t2.h, t2.start, 1) + q2;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            prefetch_l2(p.lse2 + b2 + 32 * c);
+                            prefetch_l2(p.dvec + b2 + 32 * c);
+                        }
                     }
                 };
                 if (kDyn && lane == 0) {
