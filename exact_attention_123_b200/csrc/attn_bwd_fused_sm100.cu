@@ -49,7 +49,8 @@
 // operations completing in issue order) implies dQ_i and dK_i, the products that
 // read dS, are done.  At a unit's end the loader issues the next unit's loads in the
 // order their buffers free up: V_j once the last dP^T is done, the first Q_i and dO_i,
-// then K_j once the last dQ is; that unit's K/V tiles and first Q_i and dO_i have been
+// then K_j once the last dQ is (at d = 64 K_j alternates between two buffers, so it
+// need not wait); that unit's K/V tiles and first Q_i, dO_i and row terms have been
 // prefetched into L2 meanwhile.
 //
 // Units are dealt to the CTAs heaviest first in a snake order (SCHED 0), or -- with a
@@ -98,7 +99,12 @@ struct FusedCfg {
     static constexpr int kOffDS = kOffDO + kDoStages * kTile;  // 128 keys x 128 queries bf16, two 64-query boxes
     static constexpr int kOffStage = kOffDS + 32768;           // + warp * 8192: two {32 x 32} fp32 boxes
     static constexpr int kOffVec = kOffStage + 32768;          // + st * 1024: lse2[128], D[128]
-    static constexpr int kOffBar = kOffVec + kStages * 1024;
+    // K_j buffers: two at d = 64, alternating by unit, so that the next unit's K_j loads
+    // while the current unit's last dQ products still read the other (a unit otherwise
+    // starts by waiting out that load); at d = 128 shared memory has room for one.
+    static constexpr int kKBufs = (D == 64) ? 2 : 1;
+    static constexpr int kOffK1 = kOffVec + kStages * 1024;  // the second K_j buffer
+    static constexpr int kOffBar = kOffK1 + (kKBufs == 2 ? kTile : 0);
     static constexpr int kBarKFull = 0;
     static constexpr int kBarKEmpty = 1;                       // K_j no longer read (the unit's last dQ done)
     static constexpr int kBarVFull = 2;
@@ -118,7 +124,9 @@ struct FusedCfg {
     static constexpr int kBarDone = kBarSFull + 8;
     static constexpr int kBarUFull = kBarSFull + 9;       // + entry: a claimed unit rank is published
     static constexpr int kBarUEmpty = kBarSFull + 13;     // + entry: every role has read it (385)
-    static constexpr int kNumBars = kBarSFull + 17;
+    static constexpr int kBarKFull1 = kBarSFull + 17;     // the second K_j buffer: loaded / free again
+    static constexpr int kBarKEmpty1 = kBarSFull + 18;
+    static constexpr int kNumBars = kBarSFull + 17 + (kKBufs == 2 ? 2 : 0);
     // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
     // ({rank, query-tile bits}, 16 bytes each)
     // debug library, after the ring: a check tag per Q stage and the roles' final counts
@@ -130,7 +138,7 @@ struct FusedCfg {
     // reports ATTN_ERR_UNSUPPORTED instead of running.
     static constexpr int kSmemBytes = (kSmemUsed + 1024 <= kSmemMax) ? kSmemUsed + 1024 : kSmemMax;
     static_assert(kSmemUsed <= kSmemMax, "exceeds the 227 KB per-CTA shared-memory limit");
-    static_assert(kTile % 1024 == 0 && kOffDS % 1024 == 0 && kOffStage % 1024 == 0,
+    static_assert(kTile % 1024 == 0 && kOffDS % 1024 == 0 && kOffStage % 1024 == 0 && kOffK1 % 1024 == 0,
                   "swizzled tiles must be 1024-byte aligned");
 };
 
@@ -181,6 +189,12 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
     uint8_t *sptr = smem_raw + (sbase - raw_u32);
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
+    // K_j buffer of the n-th unit with work, its barriers and the phase of its use
+    auto kbuf = [](int n) -> int { return C::kKBufs == 2 ? (n & 1) : 0; };
+    auto kpar = [](int n) -> uint32_t { return static_cast<uint32_t>(C::kKBufs == 2 ? (n >> 1) & 1 : n & 1); };
+    auto koff = [&](int n) -> uint32_t { return sbase + (kbuf(n) ? C::kOffK1 : C::kOffK); };
+    auto bar_kfull = [&](int n) -> uint32_t { return bar(kbuf(n) ? C::kBarKFull1 : C::kBarKFull); };
+    auto bar_kempty = [&](int n) -> uint32_t { return bar(kbuf(n) ? C::kBarKEmpty1 : C::kBarKEmpty); };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sptr + C::kOffBar + C::kNumBars * 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -383,13 +397,15 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 };
                 // K_j or V_j once the previous unit has released it
                 auto load_kv = [&](int kv) -> bool {
-                    const int full = kv ? C::kBarVFull : C::kBarKFull, empty = kv ? C::kBarVEmpty : C::kBarKEmpty;
-                    if (!__all_sync(0xffffffffu, wait_phase(bar(empty), (n_kv & 1) ^ 1, p.ctl, abort_flag))) return false;
+                    const uint32_t full = kv ? bar(C::kBarVFull) : bar_kfull(n_kv);
+                    const uint32_t empty = kv ? bar(C::kBarVEmpty) : bar_kempty(n_kv);
+                    const uint32_t par = kv ? static_cast<uint32_t>(n_kv & 1) : kpar(n_kv);
+                    if (!__all_sync(0xffffffffu, wait_phase(empty, par ^ 1, p.ctl, abort_flag))) return false;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(bar(full), C::kTile);
+                        mbar_arrive_expect_tx(full, C::kTile);
 #pragma unroll
                         for (int x = 0; x < C::kBoxes; ++x)
-                            tma_load_3d(sbase + (kv ? C::kOffV : C::kOffK) + x * 16384, kv ? &tm_v : &tm_k, bar(full),
+                            tma_load_3d((kv ? sbase + C::kOffV : koff(n_kv)) + x * 16384, kv ? &tm_v : &tm_k, full,
                                         x * 64, row0 + t.kv0, slab);
                     }
                     if (kv) ++n_v;
@@ -460,11 +476,12 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 // columns 64-95 of the S^T region (each math warp writes only inside the
                 // columns it read).
                 auto acol = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 64 + (kk - 4) * 8; };
+                uint32_t ks = sbase + C::kOffK;  // the current unit's K_j buffer
                 auto issue_s = [&](int gi) {
                     const uint32_t qs = sbase + C::kOffQ + (gi % C::kStages) * C::kTile;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + C::kColS, sw128_desc(sbase + C::kOffK + kstep(kk), 16, 1024),
+                        mma_ss(tmem + C::kColS, sw128_desc(ks + kstep(kk), 16, 1024),
                                sw128_desc(qs + kstep(kk), 16, 1024), idS, kk > 0);
                     tc_commit(bar(C::kBarSFull));
                 };
@@ -490,7 +507,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                     if (r >= T) break;
                     Tile t;
                     if (!tile_at(r, t, ubits) || t.nq == 0) continue;
-                    ok = wait_phase(bar(C::kBarKFull), n_t & 1, p.ctl, abort_flag);
+                    ok = wait_phase(bar_kfull(n_t), kpar(n_t), p.ctl, abort_flag);
+                    ks = koff(n_t);
                     if (ok) ok = wait_q(gbase);
                     int dbg_i = t.qs.next(t.i0);  // (debug library: the query tile of pair gi)
                     if (ok) ok = tag_ok(r, dbg_i, gbase);
@@ -543,9 +561,9 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
                             mma_ss(tmem + C::kColDQ, sw128_desc(ds + kk * 2048, 16384, 1024),
-                                   sw128_desc(sbase + C::kOffK + kk * 2048, 16384, 1024), idDQ, kk > 0 ? 1u : 0u);
+                                   sw128_desc(ks + kk * 2048, 16384, 1024), idDQ, kk > 0 ? 1u : 0u);
                         tc_commit(bar(C::kBarDQFull));
-                        if (!more) tc_commit(bar(C::kBarKEmpty));  // the unit's last reader of K_j
+                        if (!more) tc_commit(bar_kempty(n_t));  // the unit's last reader of K_j
                         // dK += dS^T Q_i  (K = 128 queries; A = dS as stored, keys x queries)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
@@ -797,7 +815,8 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     __syncthreads();
     if (warp == 12 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        if (n_kv > 0) drain_phase(bar(C::kBarKFull), (n_kv - 1) & 1, p.ctl, abort_flag);
+        for (int n = max(0, n_kv - C::kKBufs); n < n_kv; ++n)  // the last load of each K_j buffer
+            drain_phase(bar_kfull(n), kpar(n), p.ctl, abort_flag);
         if (n_v > 0) drain_phase(bar(C::kBarVFull), (n_v - 1) & 1, p.ctl, abort_flag);
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
             if (gi != p.ctl.inject_skip_load)
