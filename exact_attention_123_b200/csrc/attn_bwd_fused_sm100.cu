@@ -413,11 +413,13 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                 };
                 // In the order the previous unit releases the buffers: V_j after its last dP^T,
                 // the first Q_i and dO_i (their stages free up before its last products are
-                // done), K_j after its last dQ.
+                // done), K_j after its last dQ -- or, with two K_j buffers (free since the unit
+                // before), K_j right after V_j, ahead of the first pair's row-term loads.
                 const int i_first = t.qs.next(t.i0);
                 ok = load_kv(1);
+                if (C::kKBufs == 2 && ok) ok = load_kv(0);
                 if (ok) ok = load_pair(i_first);
-                if (ok) ok = load_kv(0);
+                if (C::kKBufs == 1 && ok) ok = load_kv(0);
                 if (!ok) break;
                 ++n_kv;
                 // the next unit's K and V tiles, and its first Q and dO tiles, into L2 while
