@@ -302,7 +302,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     int n_q = 0, n_do = 0, n_kv = 0;  // loader: Q, dO and K/V loads started (for the abort drain)
-    int n_v = 0;                      // loader: V loads started (V goes before K: n_v >= n_kv)
+    int n_v = 0, n_k = 0;             // loader: V and K loads started (a unit counts in n_kv once both are)
 
     if (warp >= 12) {
         setmaxnreg_dec<C::kRegsCtl>();
@@ -409,6 +409,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                                         x * 64, row0 + t.kv0, slab);
                     }
                     if (kv) ++n_v;
+                    else ++n_k;
                     return true;
                 };
                 // In the order the previous unit releases the buffers: V_j after its last dP^T,
@@ -817,7 +818,7 @@ attn_bwd_fused_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     __syncthreads();
     if (warp == 12 && lane == 0 && *abort_flag) {
         // After an abort, every copy the loader started must land before the CTA exits.
-        for (int n = max(0, n_kv - C::kKBufs); n < n_kv; ++n)  // the last load of each K_j buffer
+        for (int n = max(0, n_k - C::kKBufs); n < n_k; ++n)  // the last load of each K_j buffer
             drain_phase(bar_kfull(n), kpar(n), p.ctl, abort_flag);
         if (n_v > 0) drain_phase(bar(C::kBarVFull), (n_v - 1) & 1, p.ctl, abort_flag);
         for (int gi = max(0, n_q - C::kStages); gi < n_q; ++gi)
