@@ -176,3 +176,19 @@ def test_corrupted_backward_tag_is_reported_then_clean(ea):
         same(got[1:], ref[1:])
     finally:
         ea.use_debug_library(False)
+
+
+def test_bench_shape_under_checks(ea):
+    # the bench workload at full size (512 forward units and 1024 backward units on 148
+    # CTAs): no check fires and the results equal the release library's
+    inp = make_dense(2, 16, 4096, 128, seed=5, causal=True, with_grad=True)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+
+    def run():
+        o, lse = ea.attn_fwd(q, k, v, scale=inp.scale, causal=True)
+        return (o, lse) + tuple(ea.attn_bwd(q, k, v, o, lse, do, scale=inp.scale, causal=True))
+
+    rel, dbg = both(ea, run)
+    same(rel[:2], dbg[:2])
+    dq_close(dbg[2], rel[2])
+    same(rel[3:], dbg[3:])
