@@ -192,3 +192,24 @@ def test_bench_shape_under_checks(ea):
     same(rel[:2], dbg[:2])
     dq_close(dbg[2], rel[2])
     same(rel[3:], dbg[3:])
+
+
+def test_packed_workload_under_checks(ea):
+    # 8 packed sequences of U[256, 4096] tokens, 32 heads, d = 128, key padding: large enough
+    # that the forward and the single-pass backward walk their claimed units in L2-sized bands
+    # of slices on their own
+    from attn_inputs import draw_lengths
+    lengths = draw_lengths(8, 256, 4096, 40)
+    keep = padding_key_mask(lengths, 41).cuda()
+    inp = make_varlen(lengths, 32, 128, 4, True, keep.cpu(), with_grad=True)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+    kw = dict(scale=inp.scale, causal=True, cu_seqlens=inp.cu_seqlens.cuda(), key_keep=keep, max_seqlen=max(lengths))
+
+    def run():
+        o, lse = ea.attn_fwd(q, k, v, **kw)
+        return (o, lse) + tuple(ea.attn_bwd(q, k, v, o, lse, do, **kw))
+
+    rel, dbg = both(ea, run)
+    same(rel[:2], dbg[:2])
+    dq_close(dbg[2], rel[2])
+    same(rel[3:], dbg[3:])
