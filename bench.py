@@ -554,6 +554,17 @@ def run_ours(args):
         f8_tf = flops_fwd() / (f8_ms * 1e-3) / 1e12
         pk8 = 2.0 * peak
         fp8 = {"fwd_ms": round(f8_ms, 4), "fwd_tflops": round(f8_tf, 1), "pct_of_2x_bf16_peak": round(100 * f8_tf / pk8, 1)}
+        if bsp is not None:
+            # e4m3 with the block-sparse variant's tile mask (FLOPs of the pairs computed)
+            for _ in range(3):
+                ea.attn_fwd_fp8_blocksparse(q8, k8, v8, qf, kf, vf, bmd, o, lse, **kw)
+            fs_ms = _median_ms(lambda: ea.attn_fwd_fp8_blocksparse(q8, k8, v8, qf, kf, vf, bmd, o, lse, **kw),
+                               flush, stream, reps)
+            st = ea.attn_status(stream)
+            if st != ea.ATTN_OK:
+                raise RuntimeError(f"fp8 block-sparse forward reported status {st}")
+            fp8.update({"blocksparse_fwd_ms": round(fs_ms, 4),
+                        "blocksparse_fwd_tflops": round(fl_fwd / (fs_ms * 1e-3) / 1e12, 1)})
 
     shapes = None
     if not args.no_shapes and ws == 1:

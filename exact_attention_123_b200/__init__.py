@@ -8,7 +8,7 @@ missing, importing the entry points raises.
 The names follow the C ABI: ``attn_fwd``, ``attn_fwd_masked``, ``attn_fwd_varlen``,
 ``attn_bwd``, ``attn_bwd_deterministic``, ``attn_bwd_varlen``, ``attn_bwd_phase``, ``attn_bwd_noalloc``,
 ``attn_fwd_blocksparse``, ``attn_bwd_blocksparse``, ``attn_fwd_fp8``, ``attn_fwd_fp8_masked``,
-``attn_fwd_fp8_varlen``,
+``attn_fwd_fp8_varlen``, ``attn_fwd_fp8_blocksparse``,
 ``attn_bwd_workspace_bytes``, ``attn_bwd_deterministic_workspace_bytes``,
 ``attn_bwd_varlen_workspace_bytes``, ``attn_status``, ``attn_strerror``,
 ``attn_set_wait_limit_ms``, ``attn_debug_skip_load``, ``attn_debug_ex2_poly``, ``attn_debug_force_band``,
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
     L.attn_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp]
     L.attn_fwd_fp8_masked.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp, vp]
     L.attn_fwd_fp8_varlen.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, i, vp, vp, vp]
+    L.attn_fwd_fp8_blocksparse.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, f, i, vp, vp]
     L.attn_status.argtypes = [vp]
     L.attn_strerror.argtypes = [i]
     L.attn_strerror.restype = ctypes.c_char_p
@@ -109,7 +110,7 @@ def lib() -> ctypes.CDLL:
     for name in ("attn_fwd", "attn_fwd_masked", "attn_fwd_varlen", "attn_bwd", "attn_bwd_deterministic",
                  "attn_bwd_varlen", "attn_bwd_phase",
                  "attn_fwd_blocksparse", "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked",
-                 "attn_fwd_fp8_varlen", "attn_status", "attn_set_wait_limit_ms",
+                 "attn_fwd_fp8_varlen", "attn_fwd_fp8_blocksparse", "attn_status", "attn_set_wait_limit_ms",
                  "attn_debug_skip_load", "attn_debug_ex2_poly", "attn_debug_force_band", "attn_debug_checks",
                  "attn_debug_corrupt_tag"):
         getattr(L, name).restype = i
@@ -382,6 +383,29 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, o=None
         rc = lib().attn_fwd_fp8_masked(_ptr(q), _ptr(k), _ptr(v), *sc, _ptr(o), _ptr(lse), B, H, N, d, float(scale),
                                        int(causal), _ptr(key_keep), _stream(stream))
         _check(rc, "attn_fwd_fp8_masked")
+    return o, lse
+
+
+def attn_fwd_fp8_blocksparse(q, k, v, q_scale: float, k_scale: float, v_scale: float, block_mask, o=None, lse=None,
+                             *, scale: Optional[float] = None, causal: bool = True, stream=None):
+    """FP8 forward with a tile mask.  q, k, v: e4m3 codes (torch.float8_e4m3fn, or uint8
+    views of them) [B,H,N,d] whose values are code * {q,k,v}_scale; block_mask: uint8
+    device tensor [H, ceil(N/128), ceil(N/128)] as for ``attn_fwd_blocksparse``.
+    Returns (o bf16, lse fp32)."""
+    _inputs([("q", q), ("k", k), ("v", v)], (torch.float8_e4m3fn, torch.uint8), False)
+    B, H, N, d = q.shape
+    nb = (N + 127) // 128
+    _shaped(block_mask, (H, nb, nb), torch.uint8, "block_mask", q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16) if o is None else o
+    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _shaped(o, q.shape, torch.bfloat16, "o", q.device)
+    _shaped(lse, (B, H, N), torch.float32, "lse", q.device)
+    rc = lib().attn_fwd_fp8_blocksparse(_ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale), float(v_scale),
+                                        _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal), _ptr(block_mask),
+                                        _stream(stream))
+    _check(rc, "attn_fwd_fp8_blocksparse")
     return o, lse
 
 

@@ -195,7 +195,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, c
 }
 
 int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, float k_scale, float v_scale, void *o,
-                 float *lse, const Shape &s, float scale, int is_causal, const uint8_t *key_keep, void *stream) {
+                 float *lse, const Shape &s, float scale, int is_causal, const uint8_t *key_keep, void *stream,
+                 const uint8_t *block_mask = nullptr) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
     int rc = check_common(s, scale);
     if (rc) return rc;
@@ -217,7 +218,7 @@ int fwd_fp8_impl(const void *q, const void *k, const void *v, float q_scale, flo
         (rc = make_map_u8(&a.tm_v, v, s.d, rows, slabs, rstride, sstride, 128)) ||
         (rc = map_for(&a.tm_o_st, o, s, 32, false, 32)))
         return rc;
-    a.g = geom_of(s, key_keep);
+    a.g = geom_of(s, key_keep, block_mask);
     a.ctl = ctl_of(ds);
     a.o = o;
     a.lse = lse;
@@ -369,6 +370,15 @@ int attn_fwd_fp8_varlen(const void *q, const void *k, const void *v, float q_sca
     if (!cu_seqlens) return ATTN_ERR_INVALID_ARG;
     Shape s{num_seqs, H, max_seqlen, d, total_tokens, cu_seqlens};
     return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, key_keep, stream);
+}
+
+int attn_fwd_fp8_blocksparse(const void *q, const void *k, const void *v, float q_scale, float k_scale,
+                             float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
+                             int is_causal, const uint8_t *block_mask, void *stream) {
+    if (!block_mask) return ATTN_ERR_INVALID_ARG;
+    if (N > 64 * 128) return ATTN_ERR_UNSUPPORTED;  // the kernels hold a row of the mask in 64 bits
+    Shape s{B, H, N, d, 0, nullptr};
+    return fwd_fp8_impl(q, k, v, q_scale, k_scale, v_scale, o, lse, s, scale, is_causal, nullptr, stream, block_mask);
 }
 
 int attn_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,

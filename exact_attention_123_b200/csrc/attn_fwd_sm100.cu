@@ -84,9 +84,11 @@ struct FwdCfg {
     // d bytes per row (128-byte swizzle at d = 128, 64-byte swizzle at d = 64)
     static constexpr int kBoxes = F8 ? 1 : D / 64;
     static constexpr int kKSteps = D * kEsz / 32;          // 32-byte K steps of S = Q K^T
-    static_assert(NT == 2 || (NT == 1 && !F8), "one tile per CTA: bf16 only");
-    // K/V ring: at NT = 1 what half an SM's shared memory leaves after Q and the stage
-    static constexpr int kStages = NT == 1 ? (D == 128 ? 2 : 5) : F8 ? (D == 128 ? 8 : 16) : (D == 128) ? 4 : 8;
+    static_assert(NT == 1 || NT == 2, "one or two query tiles per CTA");
+    // K/V ring: at NT = 1 what half an SM's shared memory leaves after Q, P (e4m3) and
+    // the output stage
+    static constexpr int kStages = NT == 1 ? (F8 ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 5))
+                                           : F8 ? (D == 128 ? 8 : 16) : (D == 128) ? 4 : 8;
     // NT + 1 warpgroups: NT softmax groups, and one with the TMA producer, the MMA
     // issuer and two idle warps (registers move by whole warpgroups).  Launched at the
     // most registers per thread the CTAs of one SM allow (NT = 2: 384 threads, 168;
@@ -122,8 +124,8 @@ struct FwdCfg {
     static constexpr int kBarUEmpty = 13 + 2 * kStages;      // + entry: every role has read it
     static constexpr int kNumBars = 17 + 2 * kStages;
     static constexpr int kSmemTiles = (NT + kStages) * kTileBytes;
-    static constexpr int kOffP = kSmemTiles;                   // e4m3 P_0, P_1: 128 x 128 bytes each
-    static constexpr int kOffStage = kOffP + (F8 ? 2 * 16384 : 0);  // 2 KB output stage per softmax warp
+    static constexpr int kOffP = kSmemTiles;                   // e4m3 P_t: 128 x 128 bytes per tile
+    static constexpr int kOffStage = kOffP + (F8 ? NT * 16384 : 0);  // 2 KB output stage per softmax warp
     static constexpr int kOffBar = kOffStage + 4 * NT * 2048;
     // after the barriers: TMEM base, abort flag, 4-entry ring of claimed units
     // ({rank, key-tile bits}, 16 bytes each)
@@ -240,6 +242,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o_st,
                       const __grid_constant__ FwdParams p) {
     using C = FwdCfg<D, F8, NT>;
+    static_assert(!(SP && DYN && NT == 2), "a run-time claim publishes the key-tile bits of one tile");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
@@ -827,8 +830,17 @@ static cudaError_t launch_fwd_d(const FwdLaunch &a, cudaStream_t stream) {
 
 cudaError_t launch_fwd_fp8(const FwdLaunch &a, cudaStream_t stream) {
     const bool dyn = a.g.varlen != 0;  // packed sequences: uneven units, claimed at run time
-    if (a.g.d == 128) return dyn ? launch_fwd_d<128, false, true, 2, true>(a, stream) : launch_fwd_d<128, false, true>(a, stream);
-    if (a.g.d == 64) return dyn ? launch_fwd_d<64, false, true, 2, true>(a, stream) : launch_fwd_d<64, false, true>(a, stream);
+    // a tile mask: one query tile per CTA, two CTAs per SM, units claimed at run time
+    // (as the bf16 kernel)
+    const bool sp = a.g.block_mask != nullptr;
+    if (a.g.d == 128) {
+        if (sp) return launch_fwd_d<128, true, true, 1, true>(a, stream);
+        return dyn ? launch_fwd_d<128, false, true, 2, true>(a, stream) : launch_fwd_d<128, false, true>(a, stream);
+    }
+    if (a.g.d == 64) {
+        if (sp) return launch_fwd_d<64, true, true, 1, true>(a, stream);
+        return dyn ? launch_fwd_d<64, false, true, 2, true>(a, stream) : launch_fwd_d<64, false, true>(a, stream);
+    }
     return cudaErrorInvalidValue;
 }
 

@@ -271,6 +271,20 @@ ATTN_API int attn_fwd_fp8_varlen(const void *q, const void *k, const void *v, fl
                                  int H, int d, float scale, int is_causal, const int32_t *cu_seqlens,
                                  const uint8_t *key_keep, void *stream);
 
+/*
+ * FP8 forward with a block-sparse tile mask: attn_fwd_fp8's e4m3 operands, scales and
+ * rounding combined with attn_fwd_blocksparse's tile mask (codechina FlashAttention
+ * article, §7.1 Block-Sparse FlashAttention and §9 FP8).  Dense layout, no key mask.
+ *   block_mask  DEVICE uint8 [H][nb][nb], nb = ceil(N / 128), as for
+ *               attn_fwd_blocksparse (must not be NULL: ATTN_ERR_INVALID_ARG); a
+ *               query row left with no key gets O = 0 and lse = -inf.
+ *   N <= 8192, else ATTN_ERR_UNSUPPORTED.  Other arguments as attn_fwd_fp8.
+ * Nothing is allocated and no workspace is needed.
+ */
+ATTN_API int attn_fwd_fp8_blocksparse(const void *q, const void *k, const void *v, float q_scale, float k_scale,
+                                      float v_scale, void *o, float *lse, int B, int H, int N, int d, float scale,
+                                      int is_causal, const uint8_t *block_mask, void *stream);
+
 /* Size of the library-owned scratch array that attn_bwd_noalloc uses (8 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

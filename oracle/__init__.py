@@ -171,10 +171,12 @@ def e4m3_decode(codes, factor=1.0):
 
 
 def fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, scale, causal, cu_seqlens=None, key_keep=None, slices=None,
-            nthreads=None, N=None):
+            nthreads=None, N=None, block_mask=None):
     """Forward of e4m3 inputs (dense [B,H,N,d] or packed [total,H,d] with cu_seqlens):
     the attention of the decoded values (code value x per-tensor factor), with the
-    same masks as ``fwd``.  Returns (o, lse) float64 like ``fwd``."""
+    same masks as ``fwd`` (the tile mask included).  Returns (o, lse) float64 like
+    ``fwd``."""
     return fwd(e4m3_decode(q8, q_scale), e4m3_decode(k8, k_scale), e4m3_decode(v8, v_scale), scale, causal,
-               cu_seqlens=cu_seqlens, key_keep=key_keep, slices=slices, nthreads=nthreads, N=N)
+               cu_seqlens=cu_seqlens, key_keep=key_keep, slices=slices, nthreads=nthreads, N=N,
+               block_mask=block_mask)
 

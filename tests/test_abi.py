@@ -29,7 +29,8 @@ def test_header_declares_the_expected_entry_points():
     for n in ("attn_fwd", "attn_fwd_masked", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status",
               "attn_bwd_deterministic", "attn_bwd_deterministic_workspace_bytes", "attn_bwd_noalloc",
               "attn_strerror", "attn_fwd_varlen", "attn_bwd_varlen", "attn_fwd_blocksparse",
-              "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked", "attn_fwd_fp8_varlen"):
+              "attn_bwd_blocksparse", "attn_fwd_fp8", "attn_fwd_fp8_masked", "attn_fwd_fp8_varlen",
+              "attn_fwd_fp8_blocksparse"):
         assert n in names
 
 
@@ -168,6 +169,14 @@ def test_fp8_host_argument_errors(L):
                                  None, None, None) == ea.ATTN_ERR_INVALID_ARG
     assert L.attn_fwd_fp8_masked(*p5, f(1.0), f(1.0), f(1.0), vp(FAKE), vp(FAKE), 1, 1, 256, 96, f(0.1), 1,
                                  vp(FAKE), None) == ea.ATTN_ERR_UNSUPPORTED
+    # with a tile mask: the mask is required, N <= 8192, and the scales are checked as above
+    def sparse(mask, N=256, d=128, scales=(1.0, 1.0, 1.0)):
+        return L.attn_fwd_fp8_blocksparse(*p5, *(f(x) for x in scales), vp(FAKE), vp(FAKE), 1, 1, N, d, f(0.1), 1,
+                                          mask, None)
+    assert sparse(None) == ea.ATTN_ERR_INVALID_ARG
+    assert sparse(vp(FAKE), N=8193) == ea.ATTN_ERR_UNSUPPORTED
+    assert sparse(vp(FAKE), d=96) == ea.ATTN_ERR_UNSUPPORTED
+    assert sparse(vp(FAKE), scales=(1.0, 1.0, -2.0)) == ea.ATTN_ERR_INVALID_ARG
 
 
 def test_wait_limit_and_fault_hook_setters(L):

@@ -56,15 +56,18 @@ def gpu_fp8(ea, inp, causal=None, key_keep=None, cu_seqlens=None):
     return o.double().cpu().numpy(), lse.double().cpu().numpy()
 
 
-def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref, keep=None):
+def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref, keep=None, pairs=None):
     """Elementwise error bound for one (sequence, head) slice (float64 numpy, n x d),
-    over the rows that see at least one key (the others are checked exactly)."""
+    over the rows that see at least one key (the others are checked exactly).
+    ``pairs``: n x n booleans, the (query, key) pairs a tile mask keeps."""
     n = qd.shape[0]
     S = scale * (qd @ kd.T)
     if causal:
         S[np.triu_indices(n, 1)] = -np.inf
     if keep is not None:
         S[:, ~keep] = -np.inf
+    if pairs is not None:
+        S[~pairs] = -np.inf
     live = np.isfinite(lse_ref)
     S, o_l, lse_l = S[live], o_ref[live], lse_ref[live]
     m = S.max(axis=1)
@@ -77,8 +80,8 @@ def bound_slice(qd, kd, vd, scale, causal, o_ref, lse_ref, keep=None):
     return tol, live
 
 
-def check_slice(tag, qd, kd, vd, scale, causal, got_o, got_l, ro, rl, keep=None):
-    tol, live = bound_slice(qd, kd, vd, scale, causal, ro, rl, keep)
+def check_slice(tag, qd, kd, vd, scale, causal, got_o, got_l, ro, rl, keep=None, pairs=None):
+    tol, live = bound_slice(qd, kd, vd, scale, causal, ro, rl, keep, pairs)
     assert not np.isnan(got_o).any(), f"NaN in {tag}"
     # rows that see no key: exactly O = 0 and lse = -inf
     assert np.all(got_o[~live] == 0.0) and np.all(np.isneginf(got_l[~live])), f"{tag}: empty rows"
@@ -93,10 +96,17 @@ def check_slice(tag, qd, kd, vd, scale, causal, got_o, got_l, ro, rl, keep=None)
     return float((err[live] / tol[live]).max()) if live.any() else 0.0
 
 
-def check(inp, got_o, got_l, causal, slices=None, key_keep=None):
+def tile_pairs(bm_h, n):
+    """n x n booleans: the (query, key) pairs that one head's tile mask keeps."""
+    t = np.arange(n) // 128
+    return bm_h[t][:, t] != 0
+
+
+def check(inp, got_o, got_l, causal, slices=None, key_keep=None, block_mask=None):
     keep = None if key_keep is None else key_keep.numpy().astype(bool)
+    bm = None if block_mask is None else block_mask.numpy()
     ro, rl = oracle.fwd_fp8(inp.q8, inp.k8, inp.v8, inp.q_scale, inp.k_scale, inp.v_scale, inp.scale, causal,
-                            key_keep=key_keep, slices=slices)
+                            key_keep=key_keep, slices=slices, block_mask=bm)
     qd = oracle.e4m3_decode(inp.q8, inp.q_scale)
     kd = oracle.e4m3_decode(inp.k8, inp.k_scale)
     vd = oracle.e4m3_decode(inp.v8, inp.v_scale)
@@ -105,7 +115,8 @@ def check(inp, got_o, got_l, causal, slices=None, key_keep=None):
         b, h = divmod(int(sidx), inp.H)
         worst = max(worst, check_slice(f"slice {sidx}", qd[b, h], kd[b, h], vd[b, h], inp.scale, causal,
                                        got_o[b, h], got_l[b, h], ro[b, h], rl[b, h],
-                                       None if keep is None else keep[b]))
+                                       None if keep is None else keep[b],
+                                       None if bm is None else tile_pairs(bm[h], inp.N)))
     return worst
 
 
@@ -243,3 +254,62 @@ def test_fp8_d64_varlen_with_padding_mask(ea):
             check_slice(f"seq {b} head {h}", qd[st:en, h], kd[st:en, h], vd[st:en, h], inp.scale, True,
                         o[st:en, h], l[st:en, h], ro[st:en, h], rl[st:en, h], kp[st:en])
 
+
+
+# ---- FP8 with a block-sparse tile mask (attn_fwd_fp8_blocksparse): the same bound, with
+# the pairs the mask leaves out counted as masked scores.
+
+def gpu_fp8_sparse(ea, inp, bm, causal):
+    q8, k8, v8 = inp.q8.cuda(), inp.k8.cuda(), inp.v8.cuda()
+    o = torch.full(q8.shape, float("nan"), device="cuda", dtype=torch.bfloat16)
+    lse = torch.full(q8.shape[:3], float("nan"), device="cuda")
+    ea.attn_fwd_fp8_blocksparse(q8, k8, v8, inp.q_scale, inp.k_scale, inp.v_scale, bm.cuda(), o, lse,
+                                scale=inp.scale, causal=causal)
+    assert ea.attn_status() == ea.ATTN_OK
+    return o.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+SPARSE_CASES = [
+    # B, H, N, d, causal, density, seed, emptied (head, query tile) rows: query tiles
+    # with no key tile (first, last and neighbouring tiles), and a ragged N that ends
+    # the last tile mid-way.
+    (2, 3, 700, 128, False, 0.5, 9301, [(0, 2), (1, 1), (2, 2), (2, 3)]),
+    (2, 3, 700, 128, True, 0.6, 9302, [(0, 4), (1, 1)]),
+    (1, 4, 1024, 64, False, 0.3, 9303, [(3, 6), (3, 7), (0, 0)]),
+    (1, 2, 640, 64, True, 0.5, 9304, [(1, 3), (0, 4)]),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,density,seed,er", SPARSE_CASES)
+def test_fp8_blocksparse_matches_oracle(ea, B, H, N, d, causal, density, seed, er):
+    from attn_inputs import tile_mask
+    inp = make_fp8(B, H, N, d, seed=seed, causal=causal)
+    bm = tile_mask(H, N, seed + 1, density, empty_rows=er)
+    o, l = gpu_fp8_sparse(ea, inp, bm, causal)
+    check(inp, o, l, causal, block_mask=bm)
+    for h, i in er:  # emptied query tiles: O = 0 and lse = -inf exactly
+        rows = slice(i * 128, min(N, (i + 1) * 128))
+        assert np.all(o[:, h, rows] == 0.0) and np.all(np.isneginf(l[:, h, rows]))
+
+
+@pytest.mark.parametrize("d,causal", [(128, True), (128, False), (64, False)])
+def test_fp8_full_mask_is_the_dense_fp8_path(ea, d, causal):
+    # every pair kept: the masked kernel (one query tile per CTA) does the dense e4m3
+    # kernel's arithmetic in the same key-tile order, so O and lse match bit for bit (at
+    # d = 64 the dense causal kernel sweeps a unit's second tile from its diagonal
+    # tile, another order)
+    inp = make_fp8(2, 2, 520, d, seed=9310 + d, causal=causal)
+    bm = torch.ones((2, 5, 5), dtype=torch.uint8)
+    o, l = gpu_fp8_sparse(ea, inp, bm, causal)
+    o2, l2 = gpu_fp8(ea, inp, causal=causal)
+    assert np.array_equal(o, o2) and np.array_equal(l, l2)
+
+
+def test_fp8_blocksparse_full_size_sampled_slices(ea):
+    # the benchmark shape (B2 H16 N4096 d128, causal) with half of the tile pairs left
+    # out by a seeded per-head mask, checked on sampled slices
+    from attn_inputs import tile_mask
+    inp = make_fp8(2, 16, 4096, 128, seed=9320, causal=True)
+    bm = tile_mask(16, 4096, 9321, 0.5, empty_rows=[(13, 5)])
+    o, l = gpu_fp8_sparse(ea, inp, bm, True)
+    check(inp, o, l, True, slices=[0, 13, 31], block_mask=bm)
