@@ -130,6 +130,20 @@ def test_fp8_forward(ea, d):
     same(rel, dbg)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_blocksparse_forward(ea, d):
+    inp = make_fp8(2, 3, 700, d, seed=9960 + d, causal=True)
+    q8, k8, v8 = inp.q8.cuda(), inp.k8.cuda(), inp.v8.cuda()
+    bm = tile_mask(3, 700, 9961, 0.5, empty_rows=[(1, 2)]).cuda()
+
+    def run():
+        return ea.attn_fwd_fp8_blocksparse(q8, k8, v8, inp.q_scale, inp.k_scale, inp.v_scale, bm, scale=inp.scale,
+                                           causal=True)
+
+    rel, dbg = both(ea, run)
+    same(rel, dbg)
+
+
 def test_corrupted_ring_tag_is_reported_then_clean(ea):
     inp = make_dense(1, 2, 1024, 128, seed=9990, causal=False)
     q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
