@@ -222,6 +222,12 @@ BWD_PHASES = [
     ("bwd_main", 4, "attn_bwd_fused_sm100_kernel", 2.5),    # all five products of every tile pair
     ("bwd_dq_convert", 5, "attn_bwd_dq_convert_kernel", None),
 ]
+# --deterministic: the two-pass backward (attn_bwd_deterministic) in the step instead
+BWD_PHASES_DET = [
+    ("bwd_pre", 0, "attn_bwd_pre_kernel", None),            # D, lse2
+    ("bwd_dkdv", 1, "attn_bwd_dkdv_sm100_kernel", 2.0),     # S^T, dP^T, dV, dK
+    ("bwd_dq", 2, "attn_bwd_dq_sm100_kernel", 1.5),         # S, dP (recomputed), dQ
+]
 MIN_WARMUP = 10  # warm-up calls before any timing (at least, whatever --warmup says)
 
 
@@ -388,14 +394,15 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream(dev)
     kw = dict(scale=inp.scale, causal=CAUSAL, stream=stream)
-    n_k = 1 + len(BWD_PHASES)  # kernels per step
+    phases = BWD_PHASES_DET if args.deterministic else BWD_PHASES
+    n_k = 1 + len(phases)  # kernels per step
 
     def step(ev=None):
         # attn_bwd == its phases in order; launched one by one here to time each kernel
         if ev is not None:
             ev[0].record(stream)
         ea.attn_fwd(q, k, v, o, lse, **kw)
-        for i, (_, ph, _, _) in enumerate(BWD_PHASES):
+        for i, (_, ph, _, _) in enumerate(phases):
             if ev is not None:
                 ev[1 + i].record(stream)
             ea.attn_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, workspace=wsbuf, **kw)
@@ -461,7 +468,8 @@ def run_ours(args):
         if used[i]:
             stream.wait_event(ev_out[i])  # the gradients of two steps ago have left set i
         ea.attn_fwd(b["q"], b["k"], b["v"], o, lse, **kw)
-        ea.attn_bwd(b["q"], b["k"], b["v"], o, lse, b["do"], b["dq"], b["dk"], b["dv"], workspace=wsbuf, **kw)
+        ea.attn_bwd(b["q"], b["k"], b["v"], o, lse, b["do"], b["dq"], b["dk"], b["dv"], workspace=wsbuf,
+                    deterministic=args.deterministic, **kw)
         ev_run[i].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_run[i])
@@ -583,7 +591,7 @@ def run_ours(args):
     per_kernel = {"attn_fwd_sm100_kernel": (fwd_ms, fwd_tf)}
     breakdown = {"fwd": round(fwd_ms * 1e3, 1)}
     hbm_ms = {}
-    for (name, _, kname, mult), ms in zip(BWD_PHASES, med[1:]):
+    for (name, _, kname, mult), ms in zip(phases, med[1:]):
         breakdown[name] = round(ms * 1e3, 1)
         if mult is None:
             hbm_ms[kname] = ms
@@ -592,9 +600,9 @@ def run_ours(args):
     dominant = max(per_kernel, key=lambda kname: per_kernel[kname][0])
     dom_tf = per_kernel[dominant][1]
     # HBM-bound kernels, algorithmic bytes per launch: the preprocess reads O and dO
-    # (bf16) and lse, writes D and lse2 and zeroes the fp32 dQ accumulator; the
-    # conversion reads the accumulator and writes dQ (bf16)
-    hbm_bytes = {"attn_bwd_pre_kernel": B * H * N * (2 * D * 2 + 4 + 8 + 4 * D),
+    # (bf16) and lse, writes D and lse2 and (single pass) zeroes the fp32 dQ accumulator;
+    # the conversion reads the accumulator and writes dQ (bf16)
+    hbm_bytes = {"attn_bwd_pre_kernel": B * H * N * (2 * D * 2 + 4 + 8 + (0 if args.deterministic else 4 * D)),
                  "attn_bwd_dq_convert_kernel": B * H * N * (4 * D + 2 * D)}
     hbm = {k: {"achieved": round(hbm_bytes[k] / (ms * 1e-3) / 1e9, 1), "bytes_per_launch": hbm_bytes[k]}
            for k, ms in hbm_ms.items() if k in hbm_bytes}
@@ -623,6 +631,7 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": D, "causal": CAUSAL, "seed": SEED,
                    "l2": "flushed (256 MiB write) before every timed step, outside the timed bracket",
                    "warmup_steps_run": n_warm,
+                   "backward": "deterministic (two passes)" if args.deterministic else "single pass",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "traffic": recorded_traffic(dominant),
@@ -749,6 +758,8 @@ def main():
     ap.add_argument("--no-blocksparse", action="store_true", help="skip the block-sparse variant's timing")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward's timing")
     ap.add_argument("--no-shapes", action="store_true", help="skip the table of the other workload shapes")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the deterministic two-pass backward in the step instead of the single pass")
     ap.add_argument("--shape-reps", type=int, default=30, help="timed calls per entry of the shape table (median)")
     ap.add_argument("--ncu-summary", metavar="REPORT",
                     help="print the per-kernel figures of an ncu --set full report (no GPU needed) and exit")
