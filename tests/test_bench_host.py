@@ -27,6 +27,24 @@ def test_flop_conventions(bench):
     assert bench.flops_bwd() == 2.5 * bench.flops_fwd()
 
 
+def test_backward_phase_tables(bench):
+    # each kernel's tensor-core FLOPs in units of the forward's two products: the single
+    # pass does the method's five backward products once (S^T, dP^T, dV, dQ, dK = 2.5
+    # forwards); the two-pass backward recomputes S and dP in its dQ kernel (4 + 3 = 7
+    # products = 3.5 forwards).  Phase numbers as the C ABI's attn_bwd_phase.
+    single = [(ph, k, m) for _, ph, k, m in bench.BWD_PHASES]
+    det = [(ph, k, m) for _, ph, k, m in bench.BWD_PHASES_DET]
+    assert [p for p, _, _ in single] == [3, 4, 5] and [p for p, _, _ in det] == [0, 1, 2]
+    assert sum(m for _, _, m in single if m) == 2.5 and sum(m for _, _, m in det if m) == 3.5
+    assert {k for _, k, m in single + det if m is None} == {"attn_bwd_pre_kernel", "attn_bwd_dq_convert_kernel"}
+    # the tensor-core kernels' names are the record keys of their ncu reports at the bench's
+    # instantiations, which the roofline looks up for its traffic
+    for _, k, m in single + det:
+        if m is not None:
+            args = "128, 0, 0" if "fused" in k else "128, 0"
+            assert bench.ncu_kernel_key(f"void attn::{k}<{args}>(CUtensorMap_st, P)") == k
+
+
 def _copy_sources(tmp_path):
     dst = tmp_path / "exact_attention_123_b200" / "csrc"
     shutil.copytree(os.path.join(ROOT, "exact_attention_123_b200", "csrc"), dst,
